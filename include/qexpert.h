@@ -1,0 +1,223 @@
+/*
+ * qexpert.h -- C ABI of the B200 (sm_100a) quantized MoE expert step.
+ *
+ * The operation is the per-token MoE expert step of LLM decode as the
+ * Flash-MoE pages describe it:
+ *   lilting.ch, "Flash-MoE: running a 397B-parameter model on a 48 GB
+ *   MacBook", sections "Model architecture" (512 experts per layer, 4 active
+ *   per token), "Core technique: SSD expert streaming" (about 6.75 MB per
+ *   4-bit expert) and "Metal Compute Shaders" (4-bit and 2-bit dequant
+ *   matrix-vector products, two-pass RMS normalisation, MoE combine as a
+ *   weighted sum, and the fma(nibble, scale*x, bias*x) dequant rewrite);
+ *   tomo3141592653.github.io summary "Running a 400B-parameter LLM on iPhone
+ *   17 Pro", section "Hybrid quantisation" (MLX-style 4-bit quantisation);
+ *   nzkcom.pages.dev "flash-moe-romance-vs-utility", table of adopted
+ *   optimisations (hot experts at 4 bits, cold ones at 2 bits).
+ *
+ * For one token x (hidden size H) and one layer:
+ *   xn   = x / sqrt(mean(x^2) + eps) * gamma                 (RMSNorm)
+ *   l_e  = W_r[e,:] . xn + offset_e            e = 0..E-1    (router)
+ *   idx  = the K largest l_e, ties to the lower index         (top-K)
+ *   w_k  = exp(l_idx_k - l_max) / sum_j exp(l_idx_j - l_max)  (renormalised softmax)
+ *   g,u  = deq(W_gate) xn, deq(W_up) xn       [I]            (dequant-matvec)
+ *   h    = silu(g) * u                                        (SwiGLU)
+ *   y_k  = deq(W_down) h                      [H]
+ *   out  = sum_k w_k y_k (+ x if a residual is requested)     (combine)
+ * with deq(W)[r,c] = q[r,c] * scale[r, c/64] + bias[r, c/64].
+ *
+ * ---------------------------------------------------------------------
+ * Packed matrix layout (qe_qmat), R rows x C columns, bits b in {4, 2}:
+ *   wq     uint32 [R, C*b/32], row-major; field j of a word (bits
+ *          [b*j, b*j+b), low bits first) is column word*32/b + j.
+ *   scales bf16 bit patterns (uint16) [R, C/64], row-major.
+ *   biases bf16 bit patterns (uint16) [R, C/64], row-major.
+ * An expert is gate [I, H], up [I, H], down [H, I].
+ *
+ * Conventions for every entry point:
+ *   - Pointers named dev_* or documented as device memory are device
+ *     pointers owned by the caller; the library never frees them.  Unless a
+ *     function says otherwise the library allocates nothing.
+ *   - Device pointers must be 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream) and
+ *     launch only kernels, so they can be captured into a CUDA graph, except
+ *     where a function says it synchronises.
+ *   - Every function returns QE_OK (0) or a negative status; the thread-local
+ *     message of the last failure is qe_last_error().  Argument errors are
+ *     reported before anything is launched.  Errors found on the device
+ *     (a bounded wait that gave up, a bad expert descriptor) are recorded in
+ *     the workspace and returned by qe_workspace_status().
+ *   - Shapes: H % 64 == 0, I % 64 == 0, group == 64, 1 <= K <= 16, K <= E,
+ *     E <= 1024, H <= 8192, I <= 8192.
+ *   - Activations entering the dequant-matvecs must satisfy |v| < 2^90.
+ */
+#ifndef QEXPERT_H
+#define QEXPERT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define QE_API __attribute__((visibility("default")))
+#else
+#define QE_API
+#endif
+
+/* A CUDA stream (cudaStream_t). */
+typedef struct CUstream_st* qe_stream_t;
+
+/* Status codes. */
+#define QE_OK 0
+#define QE_ERR_INVALID_ARG (-1) /* bad pointer, shape or descriptor       */
+#define QE_ERR_UNSUPPORTED (-2) /* valid but not supported here            */
+#define QE_ERR_CUDA (-3)        /* a CUDA runtime call failed              */
+#define QE_ERR_TIMEOUT (-4)     /* a bounded device-side wait gave up      */
+#define QE_ERR_OOM (-5)         /* host or device allocation failed        */
+
+/* Activation dtypes. */
+#define QE_F32 0
+#define QE_BF16 1
+
+/* One packed matrix (device pointers). */
+typedef struct {
+  const uint32_t* wq;
+  const uint16_t* scales;
+  const uint16_t* biases;
+  int32_t bits; /* 4 or 2 */
+  int32_t reserved;
+} qe_qmat;
+
+/* One expert: gate [I,H], up [I,H], down [H,I]. */
+typedef struct {
+  qe_qmat gate, up, down;
+} qe_expert;
+
+/* Layer shape. group must be 64. */
+typedef struct {
+  int32_t hidden;    /* H */
+  int32_t n_experts; /* E */
+  int32_t top_k;     /* K */
+  int32_t inter;     /* I: expert intermediate size */
+  int32_t group;     /* quantisation group along the input axis: 64 */
+  float eps;         /* RMSNorm epsilon */
+} qe_cfg;
+
+/* The weights of one MoE layer.  router_w fp32 [E,H] device; logit_offset
+ * fp32 [E] device or NULL (added to the logits before top-K and softmax);
+ * gamma fp32 [H] device or NULL (meaning 1); experts: device array of E
+ * descriptors. */
+typedef struct {
+  const float* router_w;
+  const float* logit_offset;
+  const float* gamma;
+  const qe_expert* experts;
+} qe_layer;
+
+/* Message of the calling thread's last failure ("" if none). */
+QE_API const char* qe_last_error(void);
+
+/* Library version string. */
+QE_API const char* qe_version(void);
+
+/* ------------------------------------------------------------------ pool */
+
+/* Bytes of one expert in the standard pool layout at `bits` (4 or 2):
+ * gate, up and down packed words, then their scales and biases, every
+ * segment 256-byte aligned.  Returns 0 for an invalid shape. */
+QE_API size_t qe_expert_bytes(const qe_cfg* cfg, int bits);
+
+/* Fill `table_out` (HOST array of n descriptors) for n experts stored back to
+ * back from dev_base (device, 256-byte aligned) in the standard layout, with
+ * stride qe_expert_bytes(cfg, bits).  Byte offsets of expert 0's segments are
+ * written to seg_offsets[9] if not NULL, in the order gate wq, up wq, down wq,
+ * gate scales, gate biases, up scales, up biases, down scales, down biases. */
+QE_API int qe_pool_table(const qe_cfg* cfg, void* dev_base, int bits, int n, qe_expert* table_out,
+                  size_t* seg_offsets);
+
+/* ------------------------------------------------------------- workspace */
+
+/* Bytes of device workspace the calls below need for T tokens. */
+QE_API size_t qe_workspace_bytes(const qe_cfg* cfg, int T);
+
+/* Zero a workspace (device).  Call once after allocating it, and again after
+ * a call reported QE_ERR_TIMEOUT. */
+QE_API int qe_workspace_init(void* dev_ws, size_t ws_bytes, qe_stream_t stream);
+
+/* Synchronise `stream`, then return (and clear) the status the device wrote
+ * into the workspace: QE_OK, QE_ERR_TIMEOUT or QE_ERR_INVALID_ARG. */
+QE_API int qe_workspace_status(void* dev_ws, qe_stream_t stream);
+
+/* Time budget of every bounded device-side wait, in nanoseconds (default
+ * 200 ms).  Applies to launches made after the call. */
+QE_API void qe_set_wait_budget_ns(uint64_t ns);
+
+/* ----------------------------------------------------------- entry points */
+
+/* RMSNorm + router + softmax + top-K for T tokens (sections "Model
+ * architecture" and "Metal Compute Shaders" above).
+ *   x          [T,H] device, fp32 (x_dtype QE_F32) or bf16 bits (QE_BF16)
+ *   gamma      [H] device or NULL; router_w [E,H] fp32 device;
+ *   logit_offset [E] device or NULL
+ *   xn         [T,H] fp32 device output (may be NULL)
+ *   topk_idx   [T,K] int32 device output, descending logit order
+ *   topk_w     [T,K] fp32 device output, sums to 1 per token
+ * The norm and the router are evaluated in double precision, so the chosen
+ * experts are those of an fp64 evaluation up to summation order. */
+QE_API int moe_route(const qe_cfg* cfg, const void* x, int x_dtype, const float* gamma,
+              const float* router_w, const float* logit_offset, int T, float* xn,
+              int32_t* topk_idx, float* topk_w, void* dev_ws, size_t ws_bytes,
+              qe_stream_t stream);
+
+/* Expert FFN for T tokens x K selected experts, 4-bit experts only:
+ *   y[t,k,:] = deq(down_e) (silu(deq(gate_e) xn[t]) * deq(up_e) xn[t]),
+ *   e = topk_idx[t,k]  (section "Metal Compute Shaders": 4-bit matvec).
+ *   experts  device table [E] (each selected descriptor must have bits 4)
+ *   xn [T,H] fp32 device; topk_idx [T,K] int32 device; y [T,K,H] fp32 device.
+ * A selected descriptor with other bits, a NULL pointer or a misaligned
+ * pointer leaves its y rows untouched and records QE_ERR_INVALID_ARG. */
+QE_API int moe_expert_ffn_q4(const qe_cfg* cfg, const qe_expert* experts, const float* xn,
+                      const int32_t* topk_idx, int T, float* y, void* dev_ws, size_t ws_bytes,
+                      qe_stream_t stream);
+
+/* Same with 2-bit experts (section "Metal Compute Shaders": 2-bit matvec). */
+QE_API int moe_expert_ffn_q2(const qe_cfg* cfg, const qe_expert* experts, const float* xn,
+                      const int32_t* topk_idx, int T, float* y, void* dev_ws, size_t ws_bytes,
+                      qe_stream_t stream);
+
+/* Same with each expert's own bits (4 or 2), for tiered pools. */
+QE_API int moe_expert_ffn_mixed(const qe_cfg* cfg, const qe_expert* experts, const float* xn,
+                         const int32_t* topk_idx, int T, float* y, void* dev_ws, size_t ws_bytes,
+                         qe_stream_t stream);
+
+/* Weighted combine (section "Metal Compute Shaders": MoE combine):
+ *   out[t,:] = sum_k w[t,k] * y[t,k,:]  (+ residual[t,:] if not NULL),
+ * k summed in ascending order.  y [T,K,H], w [T,K], residual/out [T,H]; all
+ * fp32 device.  out may alias residual. */
+QE_API int moe_combine(const float* y, const float* w, const float* residual, int T, int K, int H,
+                float* out, qe_stream_t stream);
+
+/* The whole layer step: out[t] = combine(expert FFNs of route(x[t]))
+ * (+ x[t] if add_residual).  x [T,H] device fp32 or bf16 (x_dtype); out
+ * [T,H] fp32 device (must not alias x); topk_idx/topk_w [T,K] device outputs
+ * or NULL.  For T == 1 this is one persistent kernel covering the router,
+ * the K experts and the combine.  For T > 1 the tokens are one batch:
+ * assignments are grouped per expert so each selected expert's weights are
+ * read once per step. */
+QE_API int moe_layer_step(const qe_cfg* cfg, const qe_layer* layer, const void* x, int x_dtype, int T,
+                   float* out, int add_residual, int32_t* topk_idx, float* topk_w, void* dev_ws,
+                   size_t ws_bytes, qe_stream_t stream);
+
+/* Test hook: make CTA `cta` of the next fused single-token launches skip its
+ * arrival at the routing barrier (-1 disables).  The other CTAs' bounded
+ * waits then give up and the workspace reports QE_ERR_TIMEOUT. */
+QE_API void qe_test_skip_arrival(int cta);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QEXPERT_H */

@@ -1,0 +1,242 @@
+"""ctypes binding of libqexpert.so: same entry-point names as the C ABI.
+
+Only argument marshalling happens here; every step of the expert path runs in
+the library's CUDA kernels.  Tensors must be CUDA tensors (contiguous);
+``stream`` defaults to torch's current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqexpert.so")
+
+QE_OK = 0
+QE_ERR_INVALID_ARG = -1
+QE_ERR_UNSUPPORTED = -2
+QE_ERR_CUDA = -3
+QE_ERR_TIMEOUT = -4
+QE_ERR_OOM = -5
+QE_F32 = 0
+QE_BF16 = 1
+
+__all__ = [
+    "LIB_PATH", "lib", "QEError", "Cfg", "QMat", "Expert", "Layer", "ExpertPool",
+    "QE_OK", "QE_ERR_INVALID_ARG", "QE_ERR_UNSUPPORTED", "QE_ERR_CUDA", "QE_ERR_TIMEOUT", "QE_ERR_OOM",
+    "QE_F32", "QE_BF16",
+    "qe_last_error", "qe_version", "qe_expert_bytes", "qe_pool_table", "qe_workspace_bytes",
+    "qe_workspace_init", "qe_workspace_status", "qe_set_wait_budget_ns", "qe_test_skip_arrival",
+    "moe_route", "moe_expert_ffn_q4", "moe_expert_ffn_q2", "moe_expert_ffn_mixed", "moe_combine",
+    "moe_layer_step", "workspace",
+]
+
+
+class QEError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+class Cfg(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("n_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("inter", ctypes.c_int32), ("group", ctypes.c_int32), ("eps", ctypes.c_float)]
+
+    def __init__(self, hidden, n_experts, top_k, inter, group=64, eps=1e-6):
+        super().__init__(hidden, n_experts, top_k, inter, group, eps)
+
+
+class QMat(ctypes.Structure):
+    _fields_ = [("wq", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("biases", ctypes.c_void_p),
+                ("bits", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class Expert(ctypes.Structure):
+    _fields_ = [("gate", QMat), ("up", QMat), ("down", QMat)]
+
+
+class Layer(ctypes.Structure):
+    _fields_ = [("router_w", ctypes.c_void_p), ("logit_offset", ctypes.c_void_p), ("gamma", ctypes.c_void_p),
+                ("experts", ctypes.c_void_p)]
+
+
+assert ctypes.sizeof(Expert) == 96
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with quantized_expert_matvec_b200/build.py "
+                          "(or __graft_entry__.build()); there is no CPU fallback")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    P = ctypes.POINTER
+    sigs = {
+        "qe_last_error": (ctypes.c_char_p, []),
+        "qe_version": (ctypes.c_char_p, []),
+        "qe_expert_bytes": (sz, [P(Cfg), i32]),
+        "qe_pool_table": (i32, [P(Cfg), vp, i32, i32, P(Expert), P(ctypes.c_size_t)]),
+        "qe_workspace_bytes": (sz, [P(Cfg), i32]),
+        "qe_workspace_init": (i32, [vp, sz, vp]),
+        "qe_workspace_status": (i32, [vp, vp]),
+        "qe_set_wait_budget_ns": (None, [ctypes.c_uint64]),
+        "qe_test_skip_arrival": (None, [i32]),
+        "moe_route": (i32, [P(Cfg), vp, i32, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
+        "moe_expert_ffn_q4": (i32, [P(Cfg), vp, vp, vp, i32, vp, vp, sz, vp]),
+        "moe_expert_ffn_q2": (i32, [P(Cfg), vp, vp, vp, i32, vp, vp, sz, vp]),
+        "moe_expert_ffn_mixed": (i32, [P(Cfg), vp, vp, vp, i32, vp, vp, sz, vp]),
+        "moe_combine": (i32, [vp, vp, vp, i32, i32, i32, vp, vp]),
+        "moe_layer_step": (i32, [P(Cfg), P(Layer), vp, i32, i32, vp, i32, vp, vp, vp, sz, vp]),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+lib = _load()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int):
+    if rc != QE_OK:
+        raise QEError(rc, lib.qe_last_error().decode())
+    return rc
+
+
+def qe_last_error() -> str:
+    return lib.qe_last_error().decode()
+
+
+def qe_version() -> str:
+    return lib.qe_version().decode()
+
+
+def qe_expert_bytes(cfg: Cfg, bits: int) -> int:
+    return int(lib.qe_expert_bytes(ctypes.byref(cfg), bits))
+
+
+def qe_pool_table(cfg: Cfg, base_ptr: int, bits: int, n: int):
+    """Descriptors (ctypes array of Expert) and segment offsets of n experts
+    stored back to back from base_ptr in the standard layout."""
+    table = (Expert * max(n, 1))()
+    seg = (ctypes.c_size_t * 9)()
+    _check(lib.qe_pool_table(ctypes.byref(cfg), base_ptr, bits, n, table, seg))
+    return table, list(seg)
+
+
+def qe_workspace_bytes(cfg: Cfg, T: int) -> int:
+    return int(lib.qe_workspace_bytes(ctypes.byref(cfg), T))
+
+
+def qe_workspace_init(ws, stream=None):
+    _check(lib.qe_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def qe_workspace_status(ws, stream=None) -> int:
+    """Synchronise and return the device status (0, or a negative QE_ERR_*)."""
+    return int(lib.qe_workspace_status(_ptr(ws), _stream(stream)))
+
+
+def qe_set_wait_budget_ns(ns: int):
+    lib.qe_set_wait_budget_ns(int(ns))
+
+
+def qe_test_skip_arrival(cta: int):
+    lib.qe_test_skip_arrival(int(cta))
+
+
+def workspace(cfg: Cfg, T: int, device="cuda"):
+    """Allocate (through torch) and zero a workspace for T tokens."""
+    import torch
+    n = qe_workspace_bytes(cfg, T)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    qe_workspace_init(ws)
+    return ws
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def moe_route(cfg, x, gamma, router_w, logit_offset, xn, topk_idx, topk_w, ws, stream=None):
+    import torch
+    T = x.shape[0]
+    dt = QE_BF16 if x.dtype == torch.bfloat16 else QE_F32
+    _check(lib.moe_route(ctypes.byref(cfg), _ptr(x), dt, _ptr(gamma), _ptr(router_w), _ptr(logit_offset), T,
+                         _ptr(xn), _ptr(topk_idx), _ptr(topk_w), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def _ffn(fn, cfg, experts, xn, topk_idx, y, ws, stream):
+    T = xn.shape[0]
+    _check(fn(ctypes.byref(cfg), _ptr(experts), _ptr(xn), _ptr(topk_idx), T, _ptr(y), _ptr(ws), _nbytes(ws),
+              _stream(stream)))
+
+
+def moe_expert_ffn_q4(cfg, experts, xn, topk_idx, y, ws, stream=None):
+    _ffn(lib.moe_expert_ffn_q4, cfg, experts, xn, topk_idx, y, ws, stream)
+
+
+def moe_expert_ffn_q2(cfg, experts, xn, topk_idx, y, ws, stream=None):
+    _ffn(lib.moe_expert_ffn_q2, cfg, experts, xn, topk_idx, y, ws, stream)
+
+
+def moe_expert_ffn_mixed(cfg, experts, xn, topk_idx, y, ws, stream=None):
+    _ffn(lib.moe_expert_ffn_mixed, cfg, experts, xn, topk_idx, y, ws, stream)
+
+
+def moe_combine(y, w, residual, out, stream=None):
+    T, K, H = y.shape
+    _check(lib.moe_combine(_ptr(y), _ptr(w), _ptr(residual), T, K, H, _ptr(out), _stream(stream)))
+
+
+def moe_layer_step(cfg, layer: Layer, x, out, add_residual=False, topk_idx=None, topk_w=None, ws=None,
+                   stream=None):
+    import torch
+    T = x.shape[0]
+    dt = QE_BF16 if x.dtype == torch.bfloat16 else QE_F32
+    _check(lib.moe_layer_step(ctypes.byref(cfg), ctypes.byref(layer), _ptr(x), dt, T, _ptr(out),
+                              1 if add_residual else 0, _ptr(topk_idx), _ptr(topk_w), _ptr(ws), _nbytes(ws),
+                              _stream(stream)))
+
+
+class ExpertPool:
+    """n experts of one bit width, back to back in one device buffer
+    (standard layout of qe_pool_table), plus the device descriptor table."""
+
+    def __init__(self, cfg: Cfg, n: int, bits: int, device="cuda"):
+        import torch
+        self.cfg, self.n, self.bits = cfg, n, bits
+        self.stride = qe_expert_bytes(cfg, bits)
+        if self.stride == 0:
+            raise QEError(QE_ERR_INVALID_ARG, qe_last_error())
+        self.buf = torch.empty(self.stride * n + 256, dtype=torch.uint8, device=device)
+        base = self.buf.data_ptr()
+        self.base = (base + 255) // 256 * 256
+        self.host_table, self.seg = qe_pool_table(cfg, self.base, bits, n)
+        raw = bytes(self.host_table)[: ctypes.sizeof(Expert) * n]
+        self.table = torch.frombuffer(bytearray(raw), dtype=torch.uint8).to(device)
+
+    def seg_ptr(self, seg: int, expert: int = 0) -> int:
+        """Device address of segment `seg` (0..8, qe_pool_table order) of an expert."""
+        return self.base + expert * self.stride + self.seg[seg]

@@ -1,0 +1,331 @@
+// qe_abi.cu -- the extern "C" entry points of include/qexpert.h: argument
+// validation, error strings, workspace layout and kernel dispatch.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "qe_internal.h"
+
+namespace qe {
+
+static thread_local char g_err[512] = "";
+static unsigned long long g_budget_ns = 200ull * 1000 * 1000;
+static int g_skip_cta = -1;
+
+static int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+static int cuda_fail(cudaError_t e, const char* what) {
+  return fail(QE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+static size_t al(size_t v) { return (v + 255) & ~(size_t)255; }
+
+WsLayout ws_layout(int H, int E, int K, int I, int T) {
+  WsLayout L{};
+  const size_t t = T > 0 ? (size_t)T : 1;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = al(off + bytes); return o; };
+  L.control = take(sizeof(WsControl));
+  const size_t nlog = (size_t)E * (t > 2 ? t : 2);
+  L.logits = take(8 * nlog);
+  L.rinv = take(8 * t);
+  L.xg = take(8 * t * H);
+  L.xn = take(4 * t * H);
+  L.xp4 = take(4 * t * H);
+  L.xp2 = take(4 * t * H);
+  L.xsum = take(4 * t * (H / 32));
+  L.xexp = take(4 * t);
+  L.h = take(4 * t * K * I);
+  L.hp = take(4 * t * K * I);
+  L.hsum = take(4 * t * K * (I / 32));
+  L.hexp = take(4 * t * K);
+  L.hamax = take(4 * t * K);
+  L.y = take(4 * t * K * H);
+  L.idx = take(4 * t * K);
+  L.w = take(4 * t * K);
+  L.grp_count = take(4 * (size_t)E);
+  L.grp_start = take(4 * ((size_t)E + 1));
+  L.grp_list = take(4 * t * K);
+  L.grp_tiles = take(16 * (t * K + E));
+  L.total = off;
+  return L;
+}
+
+static int check_cfg(const qe_cfg* c) {
+  if (!c) return fail(QE_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->group != kGroup) return fail(QE_ERR_INVALID_ARG, "group must be 64 (got %d)", c->group);
+  if (c->hidden <= 0 || c->hidden % kGroup || c->hidden > kMaxDim)
+    return fail(QE_ERR_INVALID_ARG, "hidden must be a positive multiple of 64 <= %d (got %d)", kMaxDim, c->hidden);
+  if (c->inter <= 0 || c->inter % kGroup || c->inter > kMaxDim)
+    return fail(QE_ERR_INVALID_ARG, "inter must be a positive multiple of 64 <= %d (got %d)", kMaxDim, c->inter);
+  if (c->n_experts <= 0 || c->n_experts > kMaxE)
+    return fail(QE_ERR_INVALID_ARG, "n_experts must be in [1, %d] (got %d)", kMaxE, c->n_experts);
+  if (c->top_k <= 0 || c->top_k > kMaxK || c->top_k > c->n_experts)
+    return fail(QE_ERR_INVALID_ARG, "top_k must be in [1, min(16, n_experts)] (got %d)", c->top_k);
+  if (!(c->eps >= 0.0f)) return fail(QE_ERR_INVALID_ARG, "eps must be >= 0");
+  return QE_OK;
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+static int check_ptr(const void* p, const char* name, bool may_be_null = false) {
+  if (!p) return may_be_null ? QE_OK : fail(QE_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(QE_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return QE_OK;
+}
+
+static int check_ws(const qe_cfg* c, int T, void* ws, size_t bytes) {
+  if (!ws) return fail(QE_ERR_INVALID_ARG, "workspace is NULL");
+  if (((uintptr_t)ws & 255) != 0) return fail(QE_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t need = ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, T).total;
+  if (bytes < need) return fail(QE_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", bytes, need);
+  return QE_OK;
+}
+
+template <typename P>
+static P* at(void* base, size_t off) { return (P*)((char*)base + off); }
+
+struct DevInfo {
+  int sms = 0, optin = 0;
+};
+
+static DevInfo dev_info() {
+  static std::mutex mu;
+  static DevInfo cache[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  DevInfo& d = cache[dev & 63];
+  if (d.sms == 0) {
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&d.optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  }
+  return d;
+}
+
+static int route_impl(const qe_cfg* c, const void* x, int x_dtype, const float* gamma, const float* router_w,
+                      const float* offset, int T, float* xn, int32_t* idx, float* w, void* ws, size_t ws_bytes,
+                      bool want_xprime, cudaStream_t s) {
+  const WsLayout L = ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, T);
+  RouteParams p{};
+  p.H = c->hidden; p.E = c->n_experts; p.K = c->top_k; p.T = T; p.eps = c->eps;
+  p.x = x; p.x_bf16 = x_dtype == QE_BF16; p.gamma = gamma; p.router_w = router_w; p.offset = offset;
+  p.xn_out = xn; p.idx = idx; p.w = w;
+  p.rinv = at<double>(ws, L.rinv); p.xg = at<double>(ws, L.xg); p.logits = at<double>(ws, L.logits);
+  p.xn_ws = at<float>(ws, L.xn);
+  if (want_xprime) {
+    p.xp4 = at<float>(ws, L.xp4); p.xp2 = at<float>(ws, L.xp2); p.xsum = at<float>(ws, L.xsum);
+    p.xexp = at<int>(ws, L.xexp);
+  }
+  p.err = &at<WsControl>(ws, L.control)->err;
+  cudaError_t e = launch_route(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_route launch");
+  return QE_OK;
+}
+
+static int ffn_impl(const qe_cfg* c, const qe_expert* experts, const float* xn, const int32_t* idx, int T, float* y,
+                    void* ws, size_t ws_bytes, int mode, bool skip_xprep, cudaStream_t s) {
+  const WsLayout L = ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, T);
+  FfnParams p{};
+  p.H = c->hidden; p.K = c->top_k; p.I = c->inter; p.T = T; p.mode = mode;
+  p.experts = experts; p.idx = idx; p.xn = xn;
+  p.xp4 = at<float>(ws, L.xp4); p.xp2 = at<float>(ws, L.xp2); p.xsum = at<float>(ws, L.xsum);
+  p.xexp = at<int>(ws, L.xexp);
+  p.h = at<float>(ws, L.h); p.hp = at<float>(ws, L.hp); p.hsum = at<float>(ws, L.hsum);
+  p.hexp = at<int>(ws, L.hexp); p.hamax = at<unsigned>(ws, L.hamax);
+  p.y = y; p.err = &at<WsControl>(ws, L.control)->err; p.skip_xprep = skip_xprep;
+  cudaError_t e = launch_ffn(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn launch");
+  return QE_OK;
+}
+
+}  // namespace qe
+
+using namespace qe;
+
+extern "C" {
+
+const char* qe_last_error(void) { return g_err; }
+
+const char* qe_version(void) { return "qexpert 0.1 (sm_100a)"; }
+
+size_t qe_expert_bytes(const qe_cfg* c, int bits) {
+  if (check_cfg(c) != QE_OK || !(bits == 4 || bits == 2)) return 0;
+  const size_t H = c->hidden, I = c->inter;
+  const size_t wq = al(I * H * bits / 8), sb = al(I * H / kGroup * 2);
+  return 3 * wq + 6 * sb;
+}
+
+int qe_pool_table(const qe_cfg* c, void* base, int bits, int n, qe_expert* out, size_t* seg) {
+  int rc = check_cfg(c);
+  if (rc) return rc;
+  if (!(bits == 4 || bits == 2)) return fail(QE_ERR_INVALID_ARG, "bits must be 4 or 2 (got %d)", bits);
+  if (n < 0 || (n > 0 && (!base || !out))) return fail(QE_ERR_INVALID_ARG, "bad pool arguments");
+  if (((uintptr_t)base & 255) != 0) return fail(QE_ERR_INVALID_ARG, "pool base must be 256-byte aligned");
+  const size_t H = c->hidden, I = c->inter;
+  const size_t wq = al(I * H * bits / 8), sb = al(I * H / kGroup * 2);
+  const size_t offs[9] = {0, wq, 2 * wq, 3 * wq, 3 * wq + sb, 3 * wq + 2 * sb, 3 * wq + 3 * sb,
+                          3 * wq + 4 * sb, 3 * wq + 5 * sb};
+  if (seg) memcpy(seg, offs, sizeof(offs));
+  const size_t stride = 3 * wq + 6 * sb;
+  for (int e = 0; e < n; ++e) {
+    char* b = (char*)base + (size_t)e * stride;
+    qe_expert x{};
+    x.gate = {(const uint32_t*)(b + offs[0]), (const uint16_t*)(b + offs[3]), (const uint16_t*)(b + offs[4]), bits, 0};
+    x.up = {(const uint32_t*)(b + offs[1]), (const uint16_t*)(b + offs[5]), (const uint16_t*)(b + offs[6]), bits, 0};
+    x.down = {(const uint32_t*)(b + offs[2]), (const uint16_t*)(b + offs[7]), (const uint16_t*)(b + offs[8]), bits, 0};
+    out[e] = x;
+  }
+  return QE_OK;
+}
+
+size_t qe_workspace_bytes(const qe_cfg* c, int T) {
+  if (check_cfg(c) != QE_OK || T < 0) return 0;
+  return ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, T).total;
+}
+
+int qe_workspace_init(void* ws, size_t bytes, qe_stream_t stream) {
+  if (!ws || bytes < sizeof(WsControl)) return fail(QE_ERR_INVALID_ARG, "bad workspace");
+  cudaError_t e = cudaMemsetAsync(ws, 0, bytes, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "qe_workspace_init");
+  return QE_OK;
+}
+
+int qe_workspace_status(void* ws, qe_stream_t stream) {
+  if (!ws) return fail(QE_ERR_INVALID_ARG, "workspace is NULL");
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "qe_workspace_status sync");
+  int err = 0;
+  e = cudaMemcpy(&err, &((WsControl*)ws)->err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "qe_workspace_status read");
+  if (err != 0) {
+    const int zero = 0;
+    cudaMemcpy(&((WsControl*)ws)->err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    return fail(err, err == QE_ERR_TIMEOUT ? "a bounded device wait gave up (QE_ERR_TIMEOUT)"
+                                           : "the device rejected an expert descriptor");
+  }
+  return QE_OK;
+}
+
+void qe_set_wait_budget_ns(uint64_t ns) { g_budget_ns = ns ? ns : 1; }
+
+void qe_test_skip_arrival(int cta) { g_skip_cta = cta; }
+
+int moe_route(const qe_cfg* c, const void* x, int x_dtype, const float* gamma, const float* router_w,
+              const float* logit_offset, int T, float* xn, int32_t* topk_idx, float* topk_w, void* ws,
+              size_t ws_bytes, qe_stream_t stream) {
+  int rc = check_cfg(c);
+  if (rc) return rc;
+  if (T < 0) return fail(QE_ERR_INVALID_ARG, "T must be >= 0");
+  if (T == 0) return QE_OK;
+  if (!(x_dtype == QE_F32 || x_dtype == QE_BF16)) return fail(QE_ERR_INVALID_ARG, "x_dtype must be QE_F32 or QE_BF16");
+  if ((rc = check_ptr(x, "x")) || (rc = check_ptr(router_w, "router_w")) || (rc = check_ptr(gamma, "gamma", true)) ||
+      (rc = check_ptr(logit_offset, "logit_offset", true)) || (rc = check_ptr(xn, "xn", true)) ||
+      (rc = check_ptr(topk_idx, "topk_idx")) || (rc = check_ptr(topk_w, "topk_w")) ||
+      (rc = check_ws(c, T, ws, ws_bytes)))
+    return rc;
+  return route_impl(c, x, x_dtype, gamma, router_w, logit_offset, T, xn, topk_idx, topk_w, ws, ws_bytes, false,
+                    (cudaStream_t)stream);
+}
+
+static int ffn_entry(const qe_cfg* c, const qe_expert* experts, const float* xn, const int32_t* idx, int T, float* y,
+                     void* ws, size_t ws_bytes, int mode, cudaStream_t s) {
+  int rc = check_cfg(c);
+  if (rc) return rc;
+  if (T < 0) return fail(QE_ERR_INVALID_ARG, "T must be >= 0");
+  if (T == 0) return QE_OK;
+  if ((rc = check_ptr(experts, "experts")) || (rc = check_ptr(xn, "xn")) || (rc = check_ptr(idx, "topk_idx")) ||
+      (rc = check_ptr(y, "y")) || (rc = check_ws(c, T, ws, ws_bytes)))
+    return rc;
+  return ffn_impl(c, experts, xn, idx, T, y, ws, ws_bytes, mode, false, s);
+}
+
+int moe_expert_ffn_q4(const qe_cfg* c, const qe_expert* experts, const float* xn, const int32_t* idx, int T, float* y,
+                      void* ws, size_t ws_bytes, qe_stream_t stream) {
+  return ffn_entry(c, experts, xn, idx, T, y, ws, ws_bytes, 4, (cudaStream_t)stream);
+}
+
+int moe_expert_ffn_q2(const qe_cfg* c, const qe_expert* experts, const float* xn, const int32_t* idx, int T, float* y,
+                      void* ws, size_t ws_bytes, qe_stream_t stream) {
+  return ffn_entry(c, experts, xn, idx, T, y, ws, ws_bytes, 2, (cudaStream_t)stream);
+}
+
+int moe_expert_ffn_mixed(const qe_cfg* c, const qe_expert* experts, const float* xn, const int32_t* idx, int T,
+                         float* y, void* ws, size_t ws_bytes, qe_stream_t stream) {
+  return ffn_entry(c, experts, xn, idx, T, y, ws, ws_bytes, 0, (cudaStream_t)stream);
+}
+
+int moe_combine(const float* y, const float* w, const float* residual, int T, int K, int H, float* out,
+                qe_stream_t stream) {
+  if (T < 0 || K <= 0 || K > kMaxK || H <= 0) return fail(QE_ERR_INVALID_ARG, "bad combine shape");
+  if (T == 0) return QE_OK;
+  int rc;
+  if ((rc = check_ptr(y, "y")) || (rc = check_ptr(w, "w")) || (rc = check_ptr(residual, "residual", true)) ||
+      (rc = check_ptr(out, "out")))
+    return rc;
+  cudaError_t e = launch_combine(y, w, residual, 0, T, K, H, out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_combine launch");
+  return QE_OK;
+}
+
+int moe_layer_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_dtype, int T, float* out,
+                   int add_residual, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                   qe_stream_t stream) {
+  int rc = check_cfg(c);
+  if (rc) return rc;
+  if (!layer) return fail(QE_ERR_INVALID_ARG, "layer is NULL");
+  if (T < 0) return fail(QE_ERR_INVALID_ARG, "T must be >= 0");
+  if (T == 0) return QE_OK;
+  if (!(x_dtype == QE_F32 || x_dtype == QE_BF16)) return fail(QE_ERR_INVALID_ARG, "x_dtype must be QE_F32 or QE_BF16");
+  if ((rc = check_ptr(x, "x")) || (rc = check_ptr(out, "out")) || (rc = check_ptr(layer->router_w, "router_w")) ||
+      (rc = check_ptr(layer->experts, "experts")) || (rc = check_ptr(layer->gamma, "gamma", true)) ||
+      (rc = check_ptr(layer->logit_offset, "logit_offset", true)) || (rc = check_ptr(topk_idx, "topk_idx", true)) ||
+      (rc = check_ptr(topk_w, "topk_w", true)) || (rc = check_ws(c, T, ws, ws_bytes)))
+    return rc;
+  if ((const void*)out == x) return fail(QE_ERR_INVALID_ARG, "out must not alias x");
+  cudaStream_t s = (cudaStream_t)stream;
+  const WsLayout L = ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, T);
+  FusedParams p{};
+  bool fused = false;
+  if (T == 1) {
+    const DevInfo d = dev_info();
+    fused = fused_geometry(c->hidden, c->n_experts, c->top_k, c->inter, d.sms, d.optin, &p.g) == QE_OK;
+  }
+  if (fused) {
+    p.H = c->hidden; p.E = c->n_experts; p.K = c->top_k; p.I = c->inter; p.eps = c->eps;
+    p.x = x; p.x_bf16 = x_dtype == QE_BF16; p.add_residual = add_residual != 0;
+    p.gamma = layer->gamma; p.router_w = layer->router_w; p.offset = layer->logit_offset;
+    p.experts = layer->experts; p.out = out; p.topk_idx = topk_idx; p.topk_w = topk_w;
+    p.ctl = at<WsControl>(ws, L.control);
+    p.logit_part = at<double>(ws, L.logits);
+    p.hbuf = at<float>(ws, L.h);
+    p.budget_ns = g_budget_ns;
+    p.skip_cta = g_skip_cta;
+    cudaError_t e = launch_fused_layer(p, s);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step fused launch");
+    return QE_OK;
+  }
+  // batched (or a single token whose shape does not fit the fused kernel):
+  // route all tokens, then the expert FFNs, then the combine
+  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);
+  float* w = topk_w ? topk_w : at<float>(ws, L.w);
+  rc = route_impl(c, x, x_dtype, layer->gamma, layer->router_w, layer->logit_offset, T, nullptr, idx, w, ws, ws_bytes,
+                  true, s);
+  if (rc) return rc;
+  rc = ffn_impl(c, layer->experts, at<float>(ws, L.xn), idx, T, at<float>(ws, L.y), ws, ws_bytes, 0, true, s);
+  if (rc) return rc;
+  cudaError_t e = launch_combine(at<float>(ws, L.y), w, add_residual ? x : nullptr, x_dtype == QE_BF16, T,
+                                 c->top_k, c->hidden, out, s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step combine");
+  return QE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,169 @@
+// qe_internal.h -- host/device shared declarations of the CUDA library
+// (kernel parameter blocks, workspace layout, launch wrappers).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/qexpert.h"
+
+namespace qe {
+
+constexpr int kMaxK = 16;
+constexpr int kMaxE = 1024;
+constexpr int kMaxDim = 8192;
+constexpr int kGroup = 64;
+
+// Control words at the start of every workspace.
+struct WsControl {
+  int err;             // first device-side error (QE_ERR_*), 0 if none
+  unsigned route_ctr;  // fused kernel: CTAs past the router
+  unsigned exit_ctr;   // fused kernel: CTAs finished
+  unsigned pad0;
+  unsigned ready[kMaxK];  // fused kernel: CTAs done with expert k's gate/up
+  unsigned pad1[12];
+};
+static_assert(sizeof(WsControl) == 128, "control block");
+
+// Offsets (bytes) of the workspace regions for T tokens.
+struct WsLayout {
+  size_t control;   // WsControl
+  size_t logits;    // double [max(2E, T*E)]
+  size_t rinv;      // double [T]
+  size_t xg;        // double [T*H]   x*gamma for the router
+  size_t xn;        // float  [T*H]   normalised activations
+  size_t xp4;       // float  [T*H]   x' for 4-bit matrices
+  size_t xp2;       // float  [T*H]   x' for 2-bit matrices
+  size_t xsum;      // float  [T*H/32] 32-column sums of xn
+  size_t xexp;      // int    [T]     vector exponent E of xn
+  size_t h;         // float  [T*K*I] SwiGLU outputs
+  size_t hp;        // float  [T*K*I] x' of h (bits of the expert's down matrix)
+  size_t hsum;      // float  [T*K*I/32]
+  size_t hexp;      // int    [T*K]
+  size_t hamax;     // unsigned [T*K] |h| max as float bits
+  size_t y;         // float  [T*K*H] expert outputs
+  size_t idx;       // int32  [T*K]
+  size_t w;         // float  [T*K]
+  size_t grp_count; // int    [E]    assignments per expert
+  size_t grp_start; // int    [E+1]
+  size_t grp_list;  // int    [T*K]  assignment ids (t*K+k) sorted by expert
+  size_t grp_tiles; // int4   [T*K + E] work tiles of the grouped kernels
+  size_t total;
+};
+
+WsLayout ws_layout(int H, int E, int K, int I, int T);
+
+// Geometry of the fused single-token kernel.
+struct FusedGeometry {
+  int RB, RC;            // rows of a gate/up item, rows of a down item
+  int nIB, nB, nCB;      // gate/up items per expert, gate/up items, output blocks
+  int max_own;           // most output blocks one CTA owns
+  int slotB, slotC;      // ring slot bytes
+  int nslotB, nslotC;    // ring slots
+  int off_ringB, off_ringC, off_bars, off_xp4, off_xp2, off_xs, off_hp, off_hs, off_logit,
+      off_ycomb, off_misc;
+  int smem_bytes;
+  int grid;
+};
+
+struct FusedParams {
+  int H, E, K, I;
+  float eps;
+  const void* x;
+  int x_bf16;
+  int add_residual;
+  const float* gamma;
+  const float* router_w;
+  const float* offset;
+  const qe_expert* experts;
+  float* out;
+  int32_t* topk_idx;
+  float* topk_w;
+  WsControl* ctl;
+  double* logit_part;  // [2][E]
+  float* hbuf;         // [K][I]
+  FusedGeometry g;
+  unsigned long long budget_ns;
+  int skip_cta;
+};
+
+// Launch wrappers (defined in the .cu files).  Return cudaError_t.
+cudaError_t launch_fused_layer(const FusedParams& p, cudaStream_t s);
+int fused_geometry(int H, int E, int K, int I, int sms, int smem_optin, FusedGeometry* g);
+
+struct RouteParams {
+  int H, E, K, T;
+  float eps;
+  const void* x;
+  int x_bf16;
+  const float* gamma;
+  const float* router_w;
+  const float* offset;
+  float* xn_out;    // may be null
+  int32_t* idx;
+  float* w;
+  double* rinv;
+  double* xg;
+  double* logits;
+  float* xn_ws;     // normalised activations kept for the expert path (may be null)
+  float* xp4;       // may be null
+  float* xp2;
+  float* xsum;
+  int* xexp;
+  int* err;
+};
+cudaError_t launch_route(const RouteParams& p, cudaStream_t s);
+
+struct FfnParams {
+  int H, K, I, T;
+  int mode;  // 4, 2 or 0 (each expert's own bits)
+  const qe_expert* experts;
+  const int32_t* idx;
+  const float* xn;   // [T,H] (prep kernel input)
+  float* xp4;
+  float* xp2;
+  float* xsum;
+  int* xexp;
+  float* h;
+  float* hp;
+  float* hsum;
+  int* hexp;
+  unsigned* hamax;
+  float* y;          // [T,K,H]
+  int* err;
+  int skip_xprep;    // x' already prepared by the route step
+};
+cudaError_t launch_ffn(const FfnParams& p, cudaStream_t s);
+
+cudaError_t launch_combine(const float* y, const float* w, const void* residual, int res_bf16, int T, int K,
+                           int H, float* out, cudaStream_t s);
+
+struct GroupedParams {
+  int H, E, K, I, T;
+  const qe_expert* experts;
+  const int32_t* idx;
+  const float* w;
+  const float* xp4;
+  const float* xp2;
+  const float* xsum;
+  const int* xexp;
+  float* h;
+  float* hp;
+  float* hsum;
+  int* hexp;
+  unsigned* hamax;
+  float* y;
+  int* grp_count;
+  int* grp_start;
+  int* grp_list;
+  int4* grp_tiles;
+  const void* x;     // residual source
+  int x_bf16;
+  int add_residual;
+  float* out;
+  int* err;
+};
+cudaError_t launch_grouped(const GroupedParams& p, cudaStream_t s);
+
+}  // namespace qe

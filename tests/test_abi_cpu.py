@@ -1,0 +1,93 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol that
+include/qexpert.h declares, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"^QE_API\s+[\w\s\*]+?\b(\w+)\s*\(", src, flags=re.M))
+    return names
+
+
+@pytest.fixture(scope="module")
+def q():
+    import quantized_expert_matvec_b200 as q
+    return q
+
+
+def test_library_exports_every_declared_symbol(q):
+    names = declared_symbols()
+    assert {"moe_route", "moe_expert_ffn_q4", "moe_expert_ffn_q2", "moe_combine", "moe_layer_step"} <= names
+    out = subprocess.run(["nm", "-D", "--defined-only", q.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if ln.strip()}
+    missing = names - exported
+    assert not missing, missing
+    lib = ctypes.CDLL(q.LIB_PATH)
+    for n in names:
+        getattr(lib, n)
+
+
+def test_sizes_and_pool_table(q):
+    c = q.Cfg(4096, 512, 4, 1024)
+    assert q.qe_expert_bytes(c, 4) == 7_077_888
+    assert q.qe_expert_bytes(c, 2) == 3_932_160
+    table, seg = q.qe_pool_table(c, 1 << 24, 4, 3)
+    stride = q.qe_expert_bytes(c, 4)
+    assert table[2].gate.wq == (1 << 24) + 2 * stride + seg[0]
+    assert table[1].down.biases == (1 << 24) + stride + seg[8]
+    assert all(t.bits == 4 for e in range(3) for t in (table[e].gate, table[e].up, table[e].down))
+    assert seg == sorted(seg) and all(s % 256 == 0 for s in seg)
+    assert q.qe_workspace_bytes(c, 1) > 0 and q.qe_workspace_bytes(c, 256) > q.qe_workspace_bytes(c, 1)
+
+
+@pytest.mark.parametrize("cfg,msg", [
+    ((4096, 512, 4, 1000), "inter"),
+    ((4100, 512, 4, 1024), "hidden"),
+    ((4096, 512, 0, 1024), "top_k"),
+    ((4096, 4, 8, 1024), "top_k"),
+    ((4096, 2048, 4, 1024), "n_experts"),
+])
+def test_invalid_shapes_rejected_before_launch(q, cfg, msg):
+    c = q.Cfg(*cfg)
+    layer = q.Layer(16, 0, 0, 16)
+    rc = q.lib.moe_layer_step(ctypes.byref(c), ctypes.byref(layer), 16, 0, 1, 32, 0, None, None, 256, 1 << 20, None)
+    assert rc == q.QE_ERR_INVALID_ARG
+    assert msg in q.qe_last_error()
+    assert q.qe_expert_bytes(c, 4) == 0
+
+
+def test_null_and_misaligned_pointers_rejected(q):
+    c = q.Cfg(256, 16, 2, 64)
+    ws_bytes = q.qe_workspace_bytes(c, 1)
+    layer = q.Layer(0, 0, 0, 4096)
+    rc = q.lib.moe_layer_step(ctypes.byref(c), ctypes.byref(layer), 4096, 0, 1, 8192, 0, None, None, 1 << 20,
+                              ws_bytes, None)
+    assert rc == q.QE_ERR_INVALID_ARG and "router_w" in q.qe_last_error()
+    layer = q.Layer(4096 + 4, 0, 0, 4096)
+    rc = q.lib.moe_layer_step(ctypes.byref(c), ctypes.byref(layer), 4096, 0, 1, 8192, 0, None, None, 1 << 20,
+                              ws_bytes, None)
+    assert rc == q.QE_ERR_INVALID_ARG and "aligned" in q.qe_last_error()
+    layer = q.Layer(4096, 0, 0, 4096)
+    rc = q.lib.moe_layer_step(ctypes.byref(c), ctypes.byref(layer), 4096, 0, 1, 8192, 0, None, None, 1 << 20,
+                              ws_bytes - 256, None)
+    assert rc == q.QE_ERR_INVALID_ARG and "workspace too small" in q.qe_last_error()
+    rc = q.lib.moe_combine(16, 16, None, 1, 0, 64, 32, None)
+    assert rc == q.QE_ERR_INVALID_ARG
+
+
+def test_empty_batches_are_noops(q):
+    c = q.Cfg(256, 16, 2, 64)
+    layer = q.Layer(4096, 0, 0, 4096)
+    assert q.lib.moe_layer_step(ctypes.byref(c), ctypes.byref(layer), 4096, 0, 0, 8192, 0, None, None, None, 0,
+                                None) == q.QE_OK
+    assert q.lib.moe_combine(None, None, None, 0, 2, 64, None, None) == q.QE_OK
