@@ -37,7 +37,9 @@
  *   - Pointers named dev_* or documented as device memory are device
  *     pointers owned by the caller; the library never frees them.  Unless a
  *     function says otherwise the library allocates nothing.
- *   - Device pointers must be 16-byte aligned.
+ *   - Device pointers must be aligned to their element size; router_w rows
+ *     and every packed-weight, scale and bias pointer of an expert descriptor
+ *     must be 16-byte aligned, and the workspace 256-byte aligned.
  *   - Calls are asynchronous on `stream` (NULL = legacy default stream) and
  *     launch only kernels, so they can be captured into a CUDA graph, except
  *     where a function says it synchronises.

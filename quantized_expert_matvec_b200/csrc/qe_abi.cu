@@ -74,11 +74,11 @@ static int check_cfg(const qe_cfg* c) {
   return QE_OK;
 }
 
-static bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
-
-static int check_ptr(const void* p, const char* name, bool may_be_null = false) {
+// Pointers must be aligned to `align` bytes: their element size, or 16 where
+// the kernels read them with 128-bit loads (router rows).
+static int check_ptr(const void* p, const char* name, bool may_be_null = false, unsigned align = 4) {
   if (!p) return may_be_null ? QE_OK : fail(QE_ERR_INVALID_ARG, "%s is NULL", name);
-  if (!aligned16(p)) return fail(QE_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  if (((uintptr_t)p & (align - 1)) != 0) return fail(QE_ERR_INVALID_ARG, "%s is not %u-byte aligned", name, align);
   return QE_OK;
 }
 
@@ -227,7 +227,7 @@ int moe_route(const qe_cfg* c, const void* x, int x_dtype, const float* gamma, c
   if (T < 0) return fail(QE_ERR_INVALID_ARG, "T must be >= 0");
   if (T == 0) return QE_OK;
   if (!(x_dtype == QE_F32 || x_dtype == QE_BF16)) return fail(QE_ERR_INVALID_ARG, "x_dtype must be QE_F32 or QE_BF16");
-  if ((rc = check_ptr(x, "x")) || (rc = check_ptr(router_w, "router_w")) || (rc = check_ptr(gamma, "gamma", true)) ||
+  if ((rc = check_ptr(x, "x", false, x_dtype == QE_BF16 ? 2 : 4)) || (rc = check_ptr(router_w, "router_w", false, 16)) || (rc = check_ptr(gamma, "gamma", true)) ||
       (rc = check_ptr(logit_offset, "logit_offset", true)) || (rc = check_ptr(xn, "xn", true)) ||
       (rc = check_ptr(topk_idx, "topk_idx")) || (rc = check_ptr(topk_w, "topk_w")) ||
       (rc = check_ws(c, T, ws, ws_bytes)))
@@ -242,7 +242,7 @@ static int ffn_entry(const qe_cfg* c, const qe_expert* experts, const float* xn,
   if (rc) return rc;
   if (T < 0) return fail(QE_ERR_INVALID_ARG, "T must be >= 0");
   if (T == 0) return QE_OK;
-  if ((rc = check_ptr(experts, "experts")) || (rc = check_ptr(xn, "xn")) || (rc = check_ptr(idx, "topk_idx")) ||
+  if ((rc = check_ptr(experts, "experts", false, 8)) || (rc = check_ptr(xn, "xn")) || (rc = check_ptr(idx, "topk_idx")) ||
       (rc = check_ptr(y, "y")) || (rc = check_ws(c, T, ws, ws_bytes)))
     return rc;
   return ffn_impl(c, experts, xn, idx, T, y, ws, ws_bytes, mode, false, s);
@@ -285,8 +285,8 @@ int moe_layer_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_
   if (T < 0) return fail(QE_ERR_INVALID_ARG, "T must be >= 0");
   if (T == 0) return QE_OK;
   if (!(x_dtype == QE_F32 || x_dtype == QE_BF16)) return fail(QE_ERR_INVALID_ARG, "x_dtype must be QE_F32 or QE_BF16");
-  if ((rc = check_ptr(x, "x")) || (rc = check_ptr(out, "out")) || (rc = check_ptr(layer->router_w, "router_w")) ||
-      (rc = check_ptr(layer->experts, "experts")) || (rc = check_ptr(layer->gamma, "gamma", true)) ||
+  if ((rc = check_ptr(x, "x", false, x_dtype == QE_BF16 ? 2 : 4)) || (rc = check_ptr(out, "out")) || (rc = check_ptr(layer->router_w, "router_w", false, 16)) ||
+      (rc = check_ptr(layer->experts, "experts", false, 8)) || (rc = check_ptr(layer->gamma, "gamma", true)) ||
       (rc = check_ptr(layer->logit_offset, "logit_offset", true)) || (rc = check_ptr(topk_idx, "topk_idx", true)) ||
       (rc = check_ptr(topk_w, "topk_w", true)) || (rc = check_ws(c, T, ws, ws_bytes)))
     return rc;

@@ -159,6 +159,28 @@ static __device__ __forceinline__ void down_dispatch(int RC, const unsigned char
   else down_item<8, BITS>(slot, I, hp, hsum, hK, y_out, lane);
 }
 
+// The producer publishes how many items of a ring it has issued.  A consumer
+// waits for its item to be issued before it waits on the slot's full
+// barrier: a parity wait only tells the current phase from the one before,
+// so waiting on lap L of a slot whose lap L-1 has not even been issued would
+// return at once.
+static __device__ __forceinline__ void publish_issued(int* ctr, int v) {
+  asm volatile("st.release.cta.shared::cta.s32 [%0], %1;" ::"r"(smem_u32(ctr)), "r"(v) : "memory");
+}
+
+static __device__ __forceinline__ bool wait_issued(int* ctr, int j, uint64_t deadline,
+                                                   volatile int* abort_flag) {
+  unsigned spins = 0;
+  for (;;) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(ctr)) : "memory");
+    if (v > j) return true;
+    if (*abort_flag) return false;
+    if ((++spins & 15u) == 0 && gtimer() > deadline) return false;
+    __nanosleep(20);
+  }
+}
+
 __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const FusedParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const FusedGeometry& g = p.g;
@@ -192,6 +214,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
     for (int i = 0; i < g.nslotB; ++i) { mbar_init(&fullB[i], 1); mbar_init(&emptyB[i], 1); }
     for (int i = 0; i < g.nslotC; ++i) { mbar_init(&fullC[i], 1); mbar_init(&emptyC[i], 1); }
     for (int k = 0; k < K; ++k) { mbar_init(&hready[k], 1); misc->claim[k] = 0; }
+    misc->issuedB = 0;
+    misc->issuedC = 0;
     fence_mbar_init();
   }
 
@@ -367,6 +391,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
         bulk_g2s(sdst + 2 * sbytes, ex.up.scales + (size_t)r0 * gpr_h, sbytes, &fullB[slot], pol);
         bulk_g2s(sdst + 3 * sbytes, ex.up.biases + (size_t)r0 * gpr_h, sbytes, &fullB[slot], pol);
         issuedB = jb + 1;
+        publish_issued(&misc->issuedB, issuedB);
       }
       for (int jc = 0; jc < nCc && !*abort_flag; ++jc) {
         const int k = jc / own, ob = jc - k * own;
@@ -386,9 +411,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
         bulk_g2s(dst + RC * I / 2, d.scales + (size_t)r0 * gpr_i, sbytes, &fullC[slot], pol);
         bulk_g2s(dst + RC * I / 2 + sbytes, d.biases + (size_t)r0 * gpr_i, sbytes, &fullC[slot], pol);
         issuedC = jc + 1;
+        publish_issued(&misc->issuedC, issuedC);
       }
     }
-    if (lane == 0) { misc->issuedB = issuedB; misc->issuedC = issuedC; }
     __syncwarp();
   } else {
     // --------------------------------------------------------- consumers
@@ -398,7 +423,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
         const int gi = cta + G * j;
         const int k = gi / nIB, r0 = (gi - k * nIB) * RB;
         const int slot = j % g.nslotB;
-        if (!mbar_wait(&fullB[slot], (j / g.nslotB) & 1, deadline, abort_flag)) {
+        if (!wait_issued(&misc->issuedB, j, deadline, abort_flag) ||
+            !mbar_wait(&fullB[slot], (j / g.nslotB) & 1, deadline, abort_flag)) {
           if (lane == 0) { set_error(&ctl->err, QE_ERR_TIMEOUT); *abort_flag = 1; }
           break;
         }
@@ -460,7 +486,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
           }
         }
         const int slot = jc % g.nslotC;
-        if (!mbar_wait(&fullC[slot], (jc / g.nslotC) & 1, deadline, abort_flag)) {
+        if (!wait_issued(&misc->issuedC, jc, deadline, abort_flag) ||
+            !mbar_wait(&fullC[slot], (jc / g.nslotC) & 1, deadline, abort_flag)) {
           if (lane == 0) { set_error(&ctl->err, QE_ERR_TIMEOUT); *abort_flag = 1; }
           break;
         }

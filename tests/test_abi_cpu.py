@@ -76,7 +76,7 @@ def test_null_and_misaligned_pointers_rejected(q):
     layer = q.Layer(4096 + 4, 0, 0, 4096)
     rc = q.lib.moe_layer_step(ctypes.byref(c), ctypes.byref(layer), 4096, 0, 1, 8192, 0, None, None, 1 << 20,
                               ws_bytes, None)
-    assert rc == q.QE_ERR_INVALID_ARG and "aligned" in q.qe_last_error()
+    assert rc == q.QE_ERR_INVALID_ARG and "router_w is not 16-byte aligned" in q.qe_last_error()
     layer = q.Layer(4096, 0, 0, 4096)
     rc = q.lib.moe_layer_step(ctypes.byref(c), ctypes.byref(layer), 4096, 0, 1, 8192, 0, None, None, 1 << 20,
                               ws_bytes - 256, None)
