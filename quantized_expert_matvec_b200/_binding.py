@@ -26,7 +26,7 @@ __all__ = [
     "QE_OK", "QE_ERR_INVALID_ARG", "QE_ERR_UNSUPPORTED", "QE_ERR_CUDA", "QE_ERR_TIMEOUT", "QE_ERR_OOM",
     "QE_F32", "QE_BF16",
     "qe_last_error", "qe_version", "qe_expert_bytes", "qe_pool_table", "qe_workspace_bytes",
-    "qe_workspace_init", "qe_workspace_status", "qe_set_wait_budget_ns", "qe_test_skip_arrival",
+    "qe_workspace_init", "qe_workspace_status", "qe_set_wait_budget_ns", "qe_test_skip_arrival", "qe_trace_fused",
     "moe_route", "moe_expert_ffn_q4", "moe_expert_ffn_q2", "moe_expert_ffn_mixed", "moe_combine",
     "moe_layer_step", "workspace",
 ]
@@ -80,6 +80,7 @@ def _load():
         "qe_workspace_status": (i32, [vp, vp]),
         "qe_set_wait_budget_ns": (None, [ctypes.c_uint64]),
         "qe_test_skip_arrival": (None, [i32]),
+        "qe_trace_fused": (None, [vp]),
         "moe_route": (i32, [P(Cfg), vp, i32, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
         "moe_expert_ffn_q4": (i32, [P(Cfg), vp, vp, vp, i32, vp, vp, sz, vp]),
         "moe_expert_ffn_q2": (i32, [P(Cfg), vp, vp, vp, i32, vp, vp, sz, vp]),
@@ -164,6 +165,12 @@ def qe_set_wait_budget_ns(ns: int):
 
 def qe_test_skip_arrival(cta: int):
     lib.qe_test_skip_arrival(int(cta))
+
+
+def qe_trace_fused(buf):
+    """Record per-CTA phase timestamps of fused launches into buf (uint64
+    CUDA tensor [SMs, 64]); None disables."""
+    lib.qe_trace_fused(_ptr(buf) if buf is not None else None)
 
 
 def workspace(cfg: Cfg, T: int, device="cuda"):

@@ -13,6 +13,7 @@ namespace qe {
 static thread_local char g_err[512] = "";
 static unsigned long long g_budget_ns = 200ull * 1000 * 1000;
 static int g_skip_cta = -1;
+static unsigned long long* g_trace = nullptr;
 
 static int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -219,6 +220,8 @@ void qe_set_wait_budget_ns(uint64_t ns) { g_budget_ns = ns ? ns : 1; }
 
 void qe_test_skip_arrival(int cta) { g_skip_cta = cta; }
 
+void qe_trace_fused(void* dev_buf) { g_trace = (unsigned long long*)dev_buf; }
+
 int moe_route(const qe_cfg* c, const void* x, int x_dtype, const float* gamma, const float* router_w,
               const float* logit_offset, int T, float* xn, int32_t* topk_idx, float* topk_w, void* ws,
               size_t ws_bytes, qe_stream_t stream) {
@@ -309,6 +312,7 @@ int moe_layer_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_
     p.hbuf = at<float>(ws, L.h);
     p.budget_ns = g_budget_ns;
     p.skip_cta = g_skip_cta;
+    p.trace = g_trace;
     cudaError_t e = launch_fused_layer(p, s);
     if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step fused launch");
     return QE_OK;

@@ -114,6 +114,24 @@ QE_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, 
       : "memory");
 }
 
+// 16-byte asynchronous global -> shared copy (LDGSTS), L2 evict-first.
+QE_DEV void cp_async16(void* dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "l"(pol)
+               : "memory");
+}
+QE_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+QE_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Copy `bytes` (a multiple of 16) from global to shared with the 32 lanes of
+// a warp, 16 bytes per lane per step.
+QE_DEV void warp_copy_async(void* dst, const void* src, uint32_t bytes, int lane, uint64_t pol) {
+  unsigned char* d = (unsigned char*)dst;
+  const unsigned char* s = (const unsigned char*)src;
+  for (uint32_t o = (uint32_t)lane * 16u; o < bytes; o += 512u) cp_async16(d + o, s + o, pol);
+}
+
 // -------------------------------------------------------- warp reductions
 
 QE_DEV float warp_sum(float v) {
@@ -188,7 +206,7 @@ QE_DEV int lane_of_reduced_row(int row) {
 // word is masked so the field keeps its place below bit 23, and the masked
 // word read as a float is the subnormal q * 2^(p-149), p = the field's bit
 // offset.  The activation is pre-scaled per column by 2^(89-p-E) (see
-// xscale_q4 / xscale_q2), so every product is exactly q*x*2^(-60-E) before
+// xprime_q4 / xprime_q2), so every product is exactly q*x*2^(-60-E) before
 // the single fp32 rounding of the fused multiply-add.  Two products go
 // through one packed f32x2 FMA.  Fields above bit 22 are first shifted down
 // by 12.  Per group the dot product is then
@@ -203,39 +221,49 @@ QE_DEV int q2_field_pos(int j) { return j < 11 ? 2 * j : 2 * j - 12; }
 
 QE_DEV float f_of(uint32_t u) { return __uint_as_float(u); }
 
-// One uint4 of 4-bit weights (32 columns) against pre-scaled x' (16 float2).
-QE_DEV float2 dot32_q4(const uint4 w, const float2* xs, float2 acc) {
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t v = ws[i];
-    const uint32_t hv = v >> 12;
-    acc = __ffma2_rn(make_float2(f_of(v & 0xFu), f_of(v & 0xF0u)), xs[4 * i + 0], acc);
-    acc = __ffma2_rn(make_float2(f_of(v & 0xF00u), f_of(v & 0xF000u)), xs[4 * i + 1], acc);
-    acc = __ffma2_rn(make_float2(f_of(v & 0xF0000u), f_of(hv & 0xF00u)), xs[4 * i + 2], acc);
-    acc = __ffma2_rn(make_float2(f_of(hv & 0xF000u), f_of(hv & 0xF0000u)), xs[4 * i + 3], acc);
-  }
+// Eight 4-bit columns of one word against their x' (4 float2).
+QE_DEV float2 dot8_q4(const uint32_t v, const float2* x, float2 acc) {
+  const uint32_t hv = v >> 12;
+  acc = __ffma2_rn(make_float2(f_of(v & 0xFu), f_of(v & 0xF0u)), x[0], acc);
+  acc = __ffma2_rn(make_float2(f_of(v & 0xF00u), f_of(v & 0xF000u)), x[1], acc);
+  acc = __ffma2_rn(make_float2(f_of(v & 0xF0000u), f_of(hv & 0xF00u)), x[2], acc);
+  acc = __ffma2_rn(make_float2(f_of(hv & 0xF000u), f_of(hv & 0xF0000u)), x[3], acc);
   return acc;
+}
+
+// Sixteen 2-bit columns of one word against their x' (8 float2).
+QE_DEV float2 dot16_q2(const uint32_t v, const float2* x, float2 acc) {
+  const uint32_t hv = v >> 12;
+  acc = __ffma2_rn(make_float2(f_of(v & 0x3u), f_of(v & 0xCu)), x[0], acc);
+  acc = __ffma2_rn(make_float2(f_of(v & 0x30u), f_of(v & 0xC0u)), x[1], acc);
+  acc = __ffma2_rn(make_float2(f_of(v & 0x300u), f_of(v & 0xC00u)), x[2], acc);
+  acc = __ffma2_rn(make_float2(f_of(v & 0x3000u), f_of(v & 0xC000u)), x[3], acc);
+  acc = __ffma2_rn(make_float2(f_of(v & 0x30000u), f_of(v & 0xC0000u)), x[4], acc);
+  acc = __ffma2_rn(make_float2(f_of(v & 0x300000u), f_of(hv & 0xC00u)), x[5], acc);
+  acc = __ffma2_rn(make_float2(f_of(hv & 0x3000u), f_of(hv & 0xC000u)), x[6], acc);
+  acc = __ffma2_rn(make_float2(f_of(hv & 0x30000u), f_of(hv & 0xC0000u)), x[7], acc);
+  return acc;
+}
+
+// One uint4 of 4-bit weights (32 columns) against x' (16 float2); two
+// accumulators so consecutive FMAs do not wait on each other.
+QE_DEV float2 dot32_q4(const uint4 w, const float2* xs, float2 acc) {
+  float2 a2 = make_float2(0.f, 0.f);
+  acc = dot8_q4(w.x, xs, acc);
+  a2 = dot8_q4(w.y, xs + 4, a2);
+  acc = dot8_q4(w.z, xs + 8, acc);
+  a2 = dot8_q4(w.w, xs + 12, a2);
+  return make_float2(acc.x + a2.x, acc.y + a2.y);
 }
 
 // One uint4 of 2-bit weights (64 columns, one group) against x' (32 float2).
 QE_DEV float2 dot64_q2(const uint4 w, const float2* xs, float2 acc) {
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t v = ws[i];
-    const uint32_t hv = v >> 12;
-    const float2* x = xs + 8 * i;
-    acc = __ffma2_rn(make_float2(f_of(v & 0x3u), f_of(v & 0xCu)), x[0], acc);
-    acc = __ffma2_rn(make_float2(f_of(v & 0x30u), f_of(v & 0xC0u)), x[1], acc);
-    acc = __ffma2_rn(make_float2(f_of(v & 0x300u), f_of(v & 0xC00u)), x[2], acc);
-    acc = __ffma2_rn(make_float2(f_of(v & 0x3000u), f_of(v & 0xC000u)), x[3], acc);
-    acc = __ffma2_rn(make_float2(f_of(v & 0x30000u), f_of(v & 0xC0000u)), x[4], acc);
-    acc = __ffma2_rn(make_float2(f_of(v & 0x300000u), f_of(hv & 0xC00u)), x[5], acc);
-    acc = __ffma2_rn(make_float2(f_of(hv & 0x3000u), f_of(hv & 0xC000u)), x[6], acc);
-    acc = __ffma2_rn(make_float2(f_of(hv & 0x30000u), f_of(hv & 0xC0000u)), x[7], acc);
-  }
-  return acc;
+  float2 a2 = make_float2(0.f, 0.f);
+  acc = dot16_q2(w.x, xs, acc);
+  a2 = dot16_q2(w.y, xs + 8, a2);
+  acc = dot16_q2(w.z, xs + 16, acc);
+  a2 = dot16_q2(w.w, xs + 24, a2);
+  return make_float2(acc.x + a2.x, acc.y + a2.y);
 }
 
 // Vector exponent E = exponent(amax) - 30, clamped to [-38, 60]: x' stays
@@ -255,6 +283,21 @@ QE_DEV float xprime_q4(float x, int c, int E) {
 QE_DEV float xprime_q2(float x, int c, int E) {
   return x * __int_as_float((127 + 89 - q2_field_pos(c & 15) - E) << 23);
 }
+// Shared-memory layout of x' in the fused kernel.  A lane reads the whole
+// uint4 chunk of columns it works on (32 columns for 4-bit, 64 for 2-bit) as
+// float4 pieces; stored linearly, the 32 lanes of a warp would hit the same
+// banks (chunks are 128 or 256 bytes apart).  Piece i of chunk ch is stored
+// at position i ^ (ch & 7), so lanes ch..ch+7 reading piece i touch eight
+// different 16-byte bank groups.
+QE_DEV int swz_q4(int c) {
+  const int ch = c >> 5;
+  return (ch << 5) | ((((c >> 2) & 7) ^ (ch & 7)) << 2) | (c & 3);
+}
+QE_DEV int swz_q2(int c) {
+  const int ch = c >> 6;
+  return (ch << 6) | ((((c >> 2) & 15) ^ (ch & 7)) << 2) | (c & 3);
+}
+
 // 2^(60+E): turns acc back into sum q*x.
 QE_DEV float acc_scale(int E) { return __int_as_float((127 + 60 + E) << 23); }
 

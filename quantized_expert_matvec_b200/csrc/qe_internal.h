@@ -59,10 +59,9 @@ struct FusedGeometry {
   int RB, RC;            // rows of a gate/up item, rows of a down item
   int nIB, nB, nCB;      // gate/up items per expert, gate/up items, output blocks
   int max_own;           // most output blocks one CTA owns
-  int slotB, slotC;      // ring slot bytes
-  int nslotB, nslotC;    // ring slots
-  int off_ringB, off_ringC, off_bars, off_xp4, off_xp2, off_xs, off_hp, off_hs, off_logit,
-      off_ycomb, off_misc;
+  int slot;              // bytes of one warp ring slot (largest item)
+  int nslot;             // slots per warp (1 or 2)
+  int off_ring, off_xp4, off_xp2, off_xs, off_hp, off_hs, off_ycomb, off_misc;
   int smem_bytes;
   int grid;
 };
@@ -81,11 +80,12 @@ struct FusedParams {
   int32_t* topk_idx;
   float* topk_w;
   WsControl* ctl;
-  double* logit_part;  // [2][E]
+  double* logit_part;  // [E] routing logits
   float* hbuf;         // [K][I]
   FusedGeometry g;
   unsigned long long budget_ns;
   int skip_cta;
+  unsigned long long* trace;  // [grid][16] phase timestamps, or null
 };
 
 // Launch wrappers (defined in the .cu files).  Return cudaError_t.
