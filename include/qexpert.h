@@ -220,14 +220,12 @@ QE_API void qe_test_skip_arrival(int cta);
 
 /* Tracing: while dev_buf (device, uint64 [SMs][64]) is set, every fused
  * single-token launch writes globaltimer stamps (ns) of its phases per CTA:
- * 0 start, 1 router partials done, 2 routing barrier passed, 3 top-K done,
- * 4 last gate/up copy issued, 5 last down copy issued, 6 first gate/up item
- * landed, 7 last gate/up item done, 8 h of the first expert ready, 9 h of
- * the last expert ready, 10 last down item done, 11 end; slots 12 and 13
- * hold the SM cycle counter at start and end; 16+w and 32+w: consumer warp
- * w's first gate/up item landed and done; 48 consumers joined, 49 combine
- * done, 50 CTA joined, 51 in-flight copies checked, 52 CTA joined again,
- * 53 exit counter bumped.  Slots a CTA does
+ * 0 start, 1 router logits written, 2 routing barrier passed, 3 top-K
+ * done, 7 gate/up phase done, 8 h barrier passed, 9 h staged, 10 last down
+ * row done, 11 end; 12 and 13 the SM cycle counter at start and end; 16+w
+ * and 32+w: warp w done with gate/up and with down; 48 CTA joined after the
+ * expert phase, 49 combine done, 53 exit counter bumped; 56-58 routing
+ * sub-steps (router loop, first barrier, RMSNorm pass 2).  Slots a CTA does
  * not reach keep their old value.  NULL disables tracing. */
 QE_API void qe_trace_fused(void* dev_buf);
 

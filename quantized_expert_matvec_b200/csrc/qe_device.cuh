@@ -124,6 +124,14 @@ QE_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memor
 template <int N>
 QE_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+QE_DEV void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p)); }
+QE_DEV void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
+
+// Named barrier over `count` threads (non-aligned form: counts threads).
+QE_DEV void named_barrier(int id, int count) {
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Copy `bytes` (a multiple of 16) from global to shared with the 32 lanes of
 // a warp, 16 bytes per lane per step.
 QE_DEV void warp_copy_async(void* dst, const void* src, uint32_t bytes, int lane, uint64_t pol) {
@@ -245,6 +253,14 @@ QE_DEV float2 dot16_q2(const uint32_t v, const float2* x, float2 acc) {
   return acc;
 }
 
+// Two words of 2-bit weights (32 columns) against x' (16 float2).
+QE_DEV float2 dot32_q2(const uint2 w, const float2* xs, float2 acc) {
+  float2 a2 = make_float2(0.f, 0.f);
+  acc = dot16_q2(w.x, xs, acc);
+  a2 = dot16_q2(w.y, xs + 8, a2);
+  return make_float2(acc.x + a2.x, acc.y + a2.y);
+}
+
 // One uint4 of 4-bit weights (32 columns) against x' (16 float2); two
 // accumulators so consecutive FMAs do not wait on each other.
 QE_DEV float2 dot32_q4(const uint4 w, const float2* xs, float2 acc) {
@@ -296,6 +312,30 @@ QE_DEV int swz_q4(int c) {
 QE_DEV int swz_q2(int c) {
   const int ch = c >> 6;
   return (ch << 6) | ((((c >> 2) & 15) ^ (ch & 7)) << 2) | (c & 3);
+}
+
+// The 32 x' values of columns [32*lc, 32*lc+32) from a swizzled buffer, as
+// 16 float2 (4-bit form: whole chunk lc; 2-bit form: half lc&1 of chunk lc/2).
+QE_DEV void load_xs32_q4(const float* xp, int lc, float2 (&xs)[16]) {
+  const float4* src = (const float4*)(xp + lc * 32);
+  const int sw = lc & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 v = src[i ^ sw];
+    xs[2 * i] = make_float2(v.x, v.y);
+    xs[2 * i + 1] = make_float2(v.z, v.w);
+  }
+}
+QE_DEV void load_xs32_q2(const float* xp, int lc, float2 (&xs)[16]) {
+  const int ch = lc >> 1, half = lc & 1;
+  const float4* src = (const float4*)(xp + ch * 64);
+  const int sw = ch & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 v = src[(half * 8 + i) ^ sw];
+    xs[2 * i] = make_float2(v.x, v.y);
+    xs[2 * i + 1] = make_float2(v.z, v.w);
+  }
 }
 
 // 2^(60+E): turns acc back into sum q*x.

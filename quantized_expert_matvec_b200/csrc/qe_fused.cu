@@ -10,27 +10,35 @@
 // counter, every CTA ranks all E logits itself: per-warp top-K candidates by
 // redux reductions, then one merge.
 //
-// Expert phase: the selected experts' rows are cut into items, gate/up items
-// (RB rows of gate and of up) and down items (RC rows of one expert's down
-// matrix, for an output block this CTA owns).  Each warp owns a private ring
-// of shared-memory slots and streams its own items into it with 16-byte
-// cp.async copies, so the next item is in flight while the current one is
-// dequantised; there is no producer warp and no cross-warp handshake on the
-// rings.  Down items need h_k = silu(g_k) * u_k in full: every gate/up item of
+// Expert phase.  Gate/up: the selected experts' rows are cut into items of
+// RB rows of gate and of up; the four 4-warp groups take items in turn and
+// each warp of a group copies (16-byte cp.async into the group's ring) and
+// dequantises one column quarter of every row, keeping the x' of its columns
+// in registers; the four quarter sums meet in shared memory behind a named
+// barrier, and h = silu(g) * u goes to global memory.  Down: warp w works on
+// expert w % K and computes full rows (RC-row blocks of the output rows this
+// CTA owns) with h_k in registers; its rows are prefetched to L2 when the
+// expert phase starts.  Down rows need h_k in full: every gate/up item of
 // expert k bumps a global counter ready[k]; the first warp of a CTA that needs
-// h_k waits for the count, stages h_k in x' form in shared memory and raises
-// a flag for the others.  All such waits are bounded (QE_ERR_TIMEOUT).
+// h_k waits for the count, stages h_k in x' form in shared memory and raises a
+// flag for the others.  All such waits are bounded (QE_ERR_TIMEOUT).
 // The last CTA to finish resets the counters for the next launch.
 #include <math.h>
+
+#include <type_traits>
 
 #include "qe_device.cuh"
 
 namespace qe {
 
 constexpr int kWarps = 16;
+constexpr int kGroups = 4;  // 4-warp groups of the gate/up phase
+constexpr int kRB = 4;      // rows of gate (and of up) in one gate/up item
+constexpr int kRC = 4;      // rows of one down block
 constexpr int kFusedThreads = kWarps * 32;
 constexpr int kRouterRows = 8;  // router rows one CTA owns at most: E <= 8 * grid
-constexpr int kChunkMax = 16;   // 32-column chunks one warp converts: H <= 16 * 32 * 16
+constexpr int kRouterBatch = 4; // router rows accumulated together
+constexpr int kChunkMax = 8;    // 32-column chunks one warp converts: H <= 8 * 32 * 16
 
 struct FusedMisc {
   int abort;
@@ -42,7 +50,12 @@ struct FusedMisc {
   unsigned claim[kMaxK];
   int hflag[kMaxK];
   unsigned cand_idx[kWarps][kMaxK];
-  unsigned long long t_lastB, t_lastC;
+  unsigned long long cand_key[kWarps][kMaxK];
+  double cand_val[kWarps][kMaxK];
+  double lsel[kMaxK];
+  float gred[kGroups][2][4][2 * kRB];  // gate/up partial sums [group][item parity][quarter][row]
+  unsigned hamax[kMaxK];               // max |h_k| of this CTA's rows, as float bits
+  unsigned long long t_lastC;
   float redf[kWarps];
   double redd[kWarps];
   double rpart[kRouterRows][kWarps];
@@ -93,164 +106,155 @@ static __device__ __forceinline__ unsigned warp_argmax_key(unsigned long long ke
   return __reduce_min_sync(0xffffffffu, (top && lo == lmax) ? idx : 0xffffffffu);
 }
 
-// ------------------------------------------------------------ gate/up item
-// RB rows of gate and RB rows of up of one expert, staged in a slot as
-// [gate wq | up wq (at RB*H/2) | gate s | gate b | up s | up b].
-template <int RB, int BITS>
-static __device__ __forceinline__ void gateup_item(const unsigned char* slot, int H, const float* xp,
-                                                   const float* xs_sum, float xK, float* h_out,
-                                                   int lane) {
-  constexpr int COLS = BITS == 4 ? 32 : 64;  // columns per uint4 chunk
-  const int nch = H / COLS;
-  const int row_bytes = H * BITS / 8;
-  const int gpr = H / kGroup;
-  const unsigned char* gw = slot;
-  const unsigned char* uw = slot + RB * H / 2;
-  const uint16_t* gs = (const uint16_t*)(slot + RB * H);
-  const uint16_t* gb = gs + RB * gpr;
-  const uint16_t* us = gb + RB * gpr;
-  const uint16_t* ub = us + RB * gpr;
-  float yv[2 * RB];
-#pragma unroll
-  for (int i = 0; i < 2 * RB; ++i) yv[i] = 0.f;
-  for (int ch = lane; ch < nch; ch += 32) {
-    float2 xs[COLS / 2];
-    const float4* src = (const float4*)(xp + ch * COLS);
-    const int sw = ch & 7;
-#pragma unroll
-    for (int i = 0; i < COLS / 4; ++i) {
-      const float4 v = src[i ^ sw];
-      xs[2 * i] = make_float2(v.x, v.y);
-      xs[2 * i + 1] = make_float2(v.z, v.w);
-    }
-    const int g = BITS == 4 ? (ch >> 1) : ch;
-    const float xsum = BITS == 4 ? xs_sum[ch] : xs_sum[2 * ch] + xs_sum[2 * ch + 1];
-#pragma unroll
-    for (int rr = 0; rr < RB; ++rr) {
-      const uint4 wg = *(const uint4*)(gw + rr * row_bytes + ch * 16);
-      const uint4 wu = *(const uint4*)(uw + rr * row_bytes + ch * 16);
-      const float2 ag = BITS == 4 ? dot32_q4(wg, xs, make_float2(0.f, 0.f)) : dot64_q2(wg, xs, make_float2(0.f, 0.f));
-      const float2 au = BITS == 4 ? dot32_q4(wu, xs, make_float2(0.f, 0.f)) : dot64_q2(wu, xs, make_float2(0.f, 0.f));
-      yv[rr] += bf16f(gs[rr * gpr + g]) * xK * (ag.x + ag.y) + bf16f(gb[rr * gpr + g]) * xsum;
-      yv[RB + rr] += bf16f(us[rr * gpr + g]) * xK * (au.x + au.y) + bf16f(ub[rr * gpr + g]) * xsum;
-    }
-  }
-  const float s = warp_reduce_rows<2 * RB>(yv, lane);
-#pragma unroll
-  for (int rr = 0; rr < RB; ++rr) {
-    const float gv = __shfl_sync(0xffffffffu, s, lane_of_reduced_row<2 * RB>(rr));
-    const float uv = __shfl_sync(0xffffffffu, s, lane_of_reduced_row<2 * RB>(RB + rr));
-    if (lane == rr) h_out[rr] = gv / (1.0f + expf(-gv)) * uv;
-  }
-}
+// ------------------------------------------------------- gate/up (groups)
+// A gate/up item is kRB rows of gate and kRB rows of up of one expert.  The
+// four warps of a group split the columns into quarters; warp qd copies and
+// dequantises quarter qd of every row, so the x' of its columns stays in
+// registers.  Slot layout: packed words of (quarter, matrix, row) at
+// ((qd*2 + mat)*kRB + rr) * H/8, then per warp four segments [gate s | gate
+// b | up s | up b] of sseg bytes at kRB*H + qd*4*sseg.  When H is a multiple
+// of 2048 a segment holds only the quarter's groups of each row (H/128 bytes
+// a row); otherwise it holds whole rows.
 
-// --------------------------------------------------------------- down item
-// RC rows of one expert's down matrix: [wq | s (at RC*I/2) | b].
-template <int RC, int BITS>
-static __device__ __forceinline__ void down_item(const unsigned char* slot, int I, const float* hp,
-                                                 const float* hsum, float hK, float* y_out, int lane) {
-  constexpr int COLS = BITS == 4 ? 32 : 64;
-  const int nch = I / COLS;
-  const int row_bytes = I * BITS / 8;
-  const int gpr = I / kGroup;
-  const uint16_t* ds = (const uint16_t*)(slot + RC * I / 2);
-  const uint16_t* db = ds + RC * gpr;
-  float yv[RC];
-#pragma unroll
-  for (int i = 0; i < RC; ++i) yv[i] = 0.f;
-  for (int ch = lane; ch < nch; ch += 32) {
-    float2 xs[COLS / 2];
-    const float4* src = (const float4*)(hp + ch * COLS);
-    const int sw = ch & 7;
-#pragma unroll
-    for (int i = 0; i < COLS / 4; ++i) {
-      const float4 v = src[i ^ sw];
-      xs[2 * i] = make_float2(v.x, v.y);
-      xs[2 * i + 1] = make_float2(v.z, v.w);
-    }
-    const int g = BITS == 4 ? (ch >> 1) : ch;
-    const float xsum = BITS == 4 ? hsum[ch] : hsum[2 * ch] + hsum[2 * ch + 1];
-#pragma unroll
-    for (int rr = 0; rr < RC; ++rr) {
-      const uint4 w = *(const uint4*)(slot + rr * row_bytes + ch * 16);
-      const float2 a = BITS == 4 ? dot32_q4(w, xs, make_float2(0.f, 0.f)) : dot64_q2(w, xs, make_float2(0.f, 0.f));
-      yv[rr] += bf16f(ds[rr * gpr + g]) * hK * (a.x + a.y) + bf16f(db[rr * gpr + g]) * xsum;
-    }
-  }
-  const float s = warp_reduce_rows<RC>(yv, lane);
-#pragma unroll
-  for (int rr = 0; rr < RC; ++rr)
-    if (lane == lane_of_reduced_row<RC>(rr)) y_out[rr] = s;
-}
-
-template <int BITS>
-static __device__ __forceinline__ void gateup_dispatch(int RB, const unsigned char* slot, int H, const float* xp,
-                                                       const float* xs_sum, float xK, float* h_out, int lane) {
-  if (RB == 1) gateup_item<1, BITS>(slot, H, xp, xs_sum, xK, h_out, lane);
-  else if (RB == 2) gateup_item<2, BITS>(slot, H, xp, xs_sum, xK, h_out, lane);
-  else if (RB == 4) gateup_item<4, BITS>(slot, H, xp, xs_sum, xK, h_out, lane);
-  else gateup_item<8, BITS>(slot, H, xp, xs_sum, xK, h_out, lane);
-}
-
-template <int BITS>
-static __device__ __forceinline__ void down_dispatch(int RC, const unsigned char* slot, int I, const float* hp,
-                                                     const float* hsum, float hK, float* y_out, int lane) {
-  if (RC == 4) down_item<4, BITS>(slot, I, hp, hsum, hK, y_out, lane);
-  else down_item<8, BITS>(slot, I, hp, hsum, hK, y_out, lane);
-}
-
-// Item j of this CTA's list (gate/up items, then down items k-major).
-struct ItemRef {
-  bool gateup;
-  int k;   // position in the top-K list
-  int r0;  // first row (gate/up: row of I; down: row of H)
-  int ob;  // down: index of the owned output block
+struct GateUpCtx {
+  int H, gpr, nlc;  // nlc: 32-column lane chunks per quarter
+  int qsc;          // segments hold quarter rows
+  int sseg;         // bytes of one segment
+  int srow;         // entries (uint16) per row in a segment
 };
 
-static __device__ __forceinline__ ItemRef item_ref(int j, int nBc, int own, int cta, int G, const FusedGeometry& g) {
-  ItemRef it;
-  if (j < nBc) {
-    const int gi = cta + G * j;
-    it.gateup = true;
-    it.k = gi / g.nIB;
-    it.r0 = (gi - it.k * g.nIB) * g.RB;
-    it.ob = 0;
-  } else {
-    const int jc = j - nBc;
-    it.gateup = false;
-    it.k = jc / own;
-    it.ob = jc - it.k * own;
-    it.r0 = (cta + G * it.ob) * g.RC;
-  }
-  return it;
+static __device__ __forceinline__ GateUpCtx make_gateup_ctx(int H) {
+  GateUpCtx c;
+  c.H = H;
+  c.gpr = H / kGroup;
+  c.nlc = H / 128;
+  c.qsc = (H % 2048) == 0;
+  c.srow = c.qsc ? H / 256 : c.gpr;
+  c.sseg = kRB * c.srow * 2;
+  return c;
 }
 
-// Issue the copies of one item into a slot (all lanes), then commit.
-static __device__ __forceinline__ void issue_item(const ItemRef& it, unsigned char* slot, const FusedMisc* misc,
-                                                  int H, int I, const FusedGeometry& g, int lane, uint64_t pol) {
-  const qe_expert& ex = misc->ex[it.k];
-  if (it.gateup) {
-    const int bits = ex.gate.bits;
-    const uint32_t wbytes = (uint32_t)(g.RB * H * bits / 8);
-    const uint32_t sbytes = (uint32_t)(g.RB * (H / kGroup) * 2);
-    const size_t wrow = (size_t)H * bits / 32;
-    const size_t srow = (size_t)(H / kGroup);
-    warp_copy_async(slot, ex.gate.wq + (size_t)it.r0 * wrow, wbytes, lane, pol);
-    warp_copy_async(slot + g.RB * H / 2, ex.up.wq + (size_t)it.r0 * wrow, wbytes, lane, pol);
-    unsigned char* sd = slot + g.RB * H;
-    warp_copy_async(sd, ex.gate.scales + (size_t)it.r0 * srow, sbytes, lane, pol);
-    warp_copy_async(sd + sbytes, ex.gate.biases + (size_t)it.r0 * srow, sbytes, lane, pol);
-    warp_copy_async(sd + 2 * sbytes, ex.up.scales + (size_t)it.r0 * srow, sbytes, lane, pol);
-    warp_copy_async(sd + 3 * sbytes, ex.up.biases + (size_t)it.r0 * srow, sbytes, lane, pol);
+static __device__ __forceinline__ void issue_gateup(const qe_expert& ex, int r0, unsigned char* slot, int qd,
+                                                    const GateUpCtx& c, int lane, uint64_t pol) {
+  const int bits = ex.gate.bits;
+  const uint32_t qb = (uint32_t)(c.H * bits / 32);  // bytes of one row quarter
+  const size_t rowb = (size_t)c.H * bits / 8;
+  const unsigned char* gsrc = (const unsigned char*)ex.gate.wq + (size_t)r0 * rowb + qd * qb;
+  const unsigned char* usrc = (const unsigned char*)ex.up.wq + (size_t)r0 * rowb + qd * qb;
+#pragma unroll
+  for (int rr = 0; rr < kRB; ++rr) {
+    warp_copy_async(slot + ((qd * 2 + 0) * kRB + rr) * (c.H / 8), gsrc + rr * rowb, qb, lane, pol);
+    warp_copy_async(slot + ((qd * 2 + 1) * kRB + rr) * (c.H / 8), usrc + rr * rowb, qb, lane, pol);
+  }
+  unsigned char* sd = slot + kRB * c.H + qd * 4 * c.sseg;
+  const uint16_t* segsrc[4] = {ex.gate.scales, ex.gate.biases, ex.up.scales, ex.up.biases};
+  if (c.qsc) {
+    const int npc = c.H / 2048;  // 16-byte pieces of one quarter row
+    const int per_seg = kRB * npc;
+    for (int u = lane; u < 4 * per_seg; u += 32) {
+      const int seg = u / per_seg, rem = u - seg * per_seg;
+      const int rr = rem / npc, pc = rem - rr * npc;
+      const unsigned char* src = (const unsigned char*)(segsrc[seg] + (size_t)(r0 + rr) * c.gpr + qd * (c.H / 256)) + pc * 16;
+      cp_async16(sd + seg * c.sseg + rr * (c.H / 128) + pc * 16, src, pol);
+    }
   } else {
-    const qe_qmat& d = ex.down;
-    const uint32_t wbytes = (uint32_t)(g.RC * I * d.bits / 8);
-    const uint32_t sbytes = (uint32_t)(g.RC * (I / kGroup) * 2);
-    warp_copy_async(slot, d.wq + (size_t)it.r0 * I * d.bits / 32, wbytes, lane, pol);
-    warp_copy_async(slot + g.RC * I / 2, d.scales + (size_t)it.r0 * (I / kGroup), sbytes, lane, pol);
-    warp_copy_async(slot + g.RC * I / 2 + sbytes, d.biases + (size_t)it.r0 * (I / kGroup), sbytes, lane, pol);
+#pragma unroll
+    for (int seg = 0; seg < 4; ++seg)
+      warp_copy_async(sd + seg * c.sseg, segsrc[seg] + (size_t)r0 * c.gpr, (uint32_t)c.sseg, lane, pol);
   }
   cp_async_commit();
+}
+
+// Partial sums of the 2*kRB rows over this warp's quarter; returns the
+// warp-reduced value (row reduced_row_of_lane<2*kRB>(lane)).
+template <int BITS>
+static __device__ __forceinline__ float gateup_partial(const unsigned char* slot, int qd, const GateUpCtx& c,
+                                                       const float* xp, const float* xs_sum, float xK,
+                                                       float2 (&xs)[16], bool xs_cached, int lane) {
+  float yv[2 * kRB];
+#pragma unroll
+  for (int i = 0; i < 2 * kRB; ++i) yv[i] = 0.f;
+  const uint16_t* sc = (const uint16_t*)(slot + kRB * c.H + qd * 4 * c.sseg);
+  const int segs = c.sseg / 2;  // uint16 entries per segment
+  const int goff = c.qsc ? qd * (c.H / 256) : 0;
+  for (int l = lane; l < c.nlc; l += 32) {
+    const int lc = qd * c.nlc + l;  // 32-column chunk of the full row
+    if (!xs_cached) {
+      if (BITS == 4) load_xs32_q4(xp, lc, xs);
+      else load_xs32_q2(xp, lc, xs);
+    }
+    const int gi = (lc >> 1) - goff;
+    const float xsum = xs_sum[lc];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+#pragma unroll
+      for (int rr = 0; rr < kRB; ++rr) {
+        const unsigned char* wp = slot + ((qd * 2 + m) * kRB + rr) * (c.H / 8);
+        float2 a;
+        if (BITS == 4) a = dot32_q4(*(const uint4*)(wp + l * 16), xs, make_float2(0.f, 0.f));
+        else a = dot32_q2(*(const uint2*)(wp + l * 8), xs, make_float2(0.f, 0.f));
+        const float sv = bf16f(sc[(2 * m) * segs + rr * c.srow + gi]);
+        const float bv = bf16f(sc[(2 * m + 1) * segs + rr * c.srow + gi]);
+        yv[m * kRB + rr] += sv * xK * (a.x + a.y) + bv * xsum;
+      }
+    }
+  }
+  return warp_reduce_rows<2 * kRB>(yv, lane);
+}
+
+// ------------------------------------------------------------ down (warps)
+// A warp computes full rows of one expert's down matrix: RC-row blocks of the
+// output blocks this CTA owns, up to 8 rows per batch; batch row i is row
+// (i % RC) of block wi + nwk * (i / RC).  Each lane takes one 32-column chunk
+// of every row; the packed words and the scale/bias pair of that chunk are
+// loaded into registers (before h is ready, for the first chunk).
+struct DownRows {
+  uint4 w[8];       // 4-bit: one uint4; 2-bit: .x, .y
+  uint32_t sb[8];   // bf16 scale (low half) and bias (high half)
+};
+
+static __device__ __forceinline__ int down_row(int cta, int G, int RC, int wi, int nwk, int ri) {
+  const int blk = ri / RC;
+  return (cta + G * (wi + nwk * blk)) * RC + (ri - blk * RC);
+}
+
+static __device__ __forceinline__ void down_load(const qe_qmat& d, int cta, int G, int RC, int wi, int nwk, int b0,
+                                                 int nr, int I, int lc, DownRows& R) {
+  const int gpr = I / kGroup;
+  const size_t rowb = (size_t)I * d.bits / 8;
+  const int g = lc >> 1;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (i < nr) {
+      const int row = down_row(cta, G, RC, wi, nwk, b0 + i);
+      const unsigned char* rp = (const unsigned char*)d.wq + (size_t)row * rowb;
+      if (d.bits == 4) {
+        R.w[i] = __ldcs((const uint4*)rp + lc);
+      } else {
+        const uint2 v = __ldcs((const uint2*)rp + lc);
+        R.w[i] = make_uint4(v.x, v.y, 0u, 0u);
+      }
+      R.sb[i] = (uint32_t)__ldg(d.scales + (size_t)row * gpr + g) |
+                ((uint32_t)__ldg(d.biases + (size_t)row * gpr + g) << 16);
+    }
+  }
+}
+
+template <int BITS>
+static __device__ __forceinline__ void down_accum(const DownRows& R, int nr, int lc, const float* hpk,
+                                                  const float* hsk, float hK, float (&yv)[8]) {
+  float2 xs[16];
+  if (BITS == 4) load_xs32_q4(hpk, lc, xs);
+  else load_xs32_q2(hpk, lc, xs);
+  const float xsum = hsk[lc];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (i < nr) {
+      const float2 a = BITS == 4 ? dot32_q4(R.w[i], xs, make_float2(0.f, 0.f))
+                                 : dot32_q2(make_uint2(R.w[i].x, R.w[i].y), xs, make_float2(0.f, 0.f));
+      yv[i] += bf16f(R.sb[i] & 0xFFFFu) * hK * (a.x + a.y) + bf16f(R.sb[i] >> 16) * xsum;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const FusedParams p) {
@@ -269,12 +273,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   float* hp = (float*)(smem + g.off_hp);    // [K][I]
   float* hsum = (float*)(smem + g.off_hs);  // [K][I/32]
   float* ycomb = (float*)(smem + g.off_ycomb);
-  unsigned char* ring = smem + g.off_ring + (size_t)warp * g.nslot * g.slot;
   WsControl* ctl = p.ctl;
 
   if (tid == 0) {
     misc->abort = 0;
-    misc->t_lastB = 0;
     misc->t_lastC = 0;
     QE_TRACE(kTrStart);
     if (p.trace) p.trace[(size_t)cta * 64 + 12] = clock64();
@@ -294,45 +296,53 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   {
     const int S = H / kWarps;
     double ss = 0.0;
-    double acc[kRouterRows];
+    for (int r0 = 0; r0 < (nrows > 0 ? nrows : 1); r0 += kRouterBatch) {
+      double acc[kRouterBatch];
 #pragma unroll
-    for (int m = 0; m < kRouterRows; ++m) acc[m] = 0.0;
-    for (int i = lane; i < S / 4; i += 32) {
-      const int c = warp * S + 4 * i;
-      float4 wv[kRouterRows];
+      for (int m = 0; m < kRouterBatch; ++m) acc[m] = 0.0;
+      for (int i = lane; i < S / 4; i += 32) {
+        const int c = warp * S + 4 * i;
+        float4 wv[kRouterBatch];
 #pragma unroll
-      for (int m = 0; m < kRouterRows; ++m)
-        if (m < nrows) wv[m] = __ldg((const float4*)(p.router_w + (size_t)(cta + G * m) * H + c));
-      double xv[4];
-      load_x4(p, c, xv);
-      ss += xv[0] * xv[0] + xv[1] * xv[1] + xv[2] * xv[2] + xv[3] * xv[3];
-      if (p.gamma) {
-        const float4 gm = *(const float4*)(p.gamma + c);
-        xv[0] *= (double)gm.x; xv[1] *= (double)gm.y; xv[2] *= (double)gm.z; xv[3] *= (double)gm.w;
+        for (int m = 0; m < kRouterBatch; ++m)
+          if (r0 + m < nrows) wv[m] = __ldg((const float4*)(p.router_w + (size_t)(cta + G * (r0 + m)) * H + c));
+        double xv[4];
+        load_x4(p, c, xv);
+        if (r0 == 0) {
+          ss += xv[0] * xv[0] + xv[1] * xv[1] + xv[2] * xv[2] + xv[3] * xv[3];
+          // raw x for RMSNorm pass 2 (the x' buffer is free until then)
+          *(float4*)(xp4 + c) = make_float4((float)xv[0], (float)xv[1], (float)xv[2], (float)xv[3]);
+        }
+        if (p.gamma) {
+          const float4 gm = *(const float4*)(p.gamma + c);
+          xv[0] *= (double)gm.x; xv[1] *= (double)gm.y; xv[2] *= (double)gm.z; xv[3] *= (double)gm.w;
+        }
+#pragma unroll
+        for (int m = 0; m < kRouterBatch; ++m) {
+          if (r0 + m < nrows) {
+            double a = acc[m];
+            a = fma((double)wv[m].x, xv[0], a);
+            a = fma((double)wv[m].y, xv[1], a);
+            a = fma((double)wv[m].z, xv[2], a);
+            a = fma((double)wv[m].w, xv[3], a);
+            acc[m] = a;
+          }
+        }
       }
 #pragma unroll
-      for (int m = 0; m < kRouterRows; ++m) {
-        if (m < nrows) {
-          double a = acc[m];
-          a = fma((double)wv[m].x, xv[0], a);
-          a = fma((double)wv[m].y, xv[1], a);
-          a = fma((double)wv[m].z, xv[2], a);
-          a = fma((double)wv[m].w, xv[3], a);
-          acc[m] = a;
+      for (int m = 0; m < kRouterBatch; ++m) {
+        if (r0 + m < nrows) {
+          const double t = warp_sum_d(acc[m]);
+          if (lane == 0) misc->rpart[r0 + m][warp] = t;
         }
       }
     }
+    if (tid == 0) QE_TRACE(56);
     ss = warp_sum_d(ss);
-#pragma unroll
-    for (int m = 0; m < kRouterRows; ++m) {
-      if (m < nrows) {
-        const double t = warp_sum_d(acc[m]);
-        if (lane == 0) misc->rpart[m][warp] = t;
-      }
-    }
     if (lane == 0) misc->redd[warp] = ss;
   }
   __syncthreads();
+  if (tid == 0) QE_TRACE(57);
   double rinv;
   {
     double tot = 0.0;
@@ -347,8 +357,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   }
   // RMSNorm pass 2 in 32-column chunks (lane = column): xn stays in
   // registers until the vector exponent of x' is known
+  // (fp32 suffices here: xn feeds the expert matvecs, not the routing)
   float xnv[kChunkMax];
   {
+    const float rinv_f = (float)rinv;
     float amax = 0.f;
 #pragma unroll
     for (int q = 0; q < kChunkMax; ++q) {
@@ -356,14 +368,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
       xnv[q] = 0.f;
       if (ch < H / 32) {
         const int c = ch * 32 + lane;
-        const double gm = p.gamma ? (double)p.gamma[c] : 1.0;
-        xnv[q] = (float)((double)load_x(p, c) * rinv * gm);
+        const float gm = p.gamma ? p.gamma[c] : 1.0f;
+        xnv[q] = xp4[c] * rinv_f * gm;
         amax = fmaxf(amax, fabsf(xnv[q]));
       }
     }
     amax = warp_max(amax);
     if (lane == 0) misc->redf[warp] = amax;
   }
+  if (tid == 0) QE_TRACE(58);
   __syncthreads();
   if (tid == 0) {
     QE_TRACE(kTrRouterDone);
@@ -398,19 +411,25 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
 
   // ---------------------------------------------------------------- top-K
   // Thread t ranks logits t and t+512.  Each warp finds its own top-K by K
-  // rounds of warp_argmax_key (a sorted candidate list); warp 0 then merges
-  // the 16 lists, one list per lane.
+  // rounds of warp_argmax_key (a sorted candidate list, keys and values kept
+  // in shared memory); warp 0 then merges the 16 lists, one list per lane.
   if (!*abort_flag) {
     const unsigned iA = (unsigned)tid, iB = (unsigned)(tid + kFusedThreads);
     bool hasA = tid < E, hasB = tid + kFusedThreads < E;
-    const unsigned long long kA = hasA ? dkey(__ldcg(&p.logit_part[iA])) : 0ull;
-    const unsigned long long kB = hasB ? dkey(__ldcg(&p.logit_part[iB])) : 0ull;
+    const double vA = hasA ? __ldcg(&p.logit_part[iA]) : 0.0;
+    const double vB = hasB ? __ldcg(&p.logit_part[iB]) : 0.0;
+    const unsigned long long kA = dkey(vA), kB = dkey(vB);
     for (int k = 0; k < K; ++k) {
       const bool useA = hasA && (!hasB || kA >= kB);  // equal keys: A has the lower index
       const unsigned bi = (hasA || hasB) ? (useA ? iA : iB) : 0xffffffffu;
       const unsigned win = warp_argmax_key(useA ? kA : kB, bi);
       if (lane == 0) misc->cand_idx[warp][k] = win;
       if (bi != 0xffffffffu && bi == win) {
+        misc->cand_key[warp][k] = useA ? kA : kB;
+        misc->cand_val[warp][k] = useA ? vA : vB;
+        // warm L1 with the candidate's descriptor while the rounds go on
+        prefetch_l1(&p.experts[win]);
+        prefetch_l1((const unsigned char*)&p.experts[win] + 64);
         if (useA) hasA = false;
         else hasB = false;
       }
@@ -419,22 +438,27 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   __syncthreads();
   if (warp == 0 && !*abort_flag) {
     int ptr = 0;
+    double myval = 0.0;
     for (int k = 0; k < K; ++k) {
       unsigned bi = 0xffffffffu;
       unsigned long long bk = 0;
       if (lane < kWarps && ptr < K) {
         bi = misc->cand_idx[lane][ptr];
-        if (bi != 0xffffffffu) bk = dkey(__ldcg(&p.logit_part[bi]));
+        if (bi != 0xffffffffu) bk = misc->cand_key[lane][ptr];
       }
       const unsigned win = warp_argmax_key(bk, bi);
-      if (lane == 0) misc->idx[k] = (int)win;
-      if (bi != 0xffffffffu && bi == win) ++ptr;
+      if (bi != 0xffffffffu && bi == win) {
+        misc->idx[k] = (int)win;
+        myval = misc->cand_val[lane][ptr];
+        ++ptr;
+        misc->lsel[k] = myval;
+      }
     }
     __syncwarp();
     // renormalised softmax over the K kept logits (sum in k order); lanes
     // k < K also fetch and check the K expert descriptors
-    const double lmax = __ldcg(&p.logit_part[misc->idx[0]]);
-    const double ev = lane < K ? exp(__ldcg(&p.logit_part[misc->idx[lane]]) - lmax) : 0.0;
+    const double lmax = misc->lsel[0];
+    const double ev = lane < K ? exp(misc->lsel[lane] - lmax) : 0.0;
     double s = 0.0;
     for (int k = 0; k < K; ++k) s += __shfl_sync(0xffffffffu, ev, k);
     if (lane < K) {
@@ -454,112 +478,186 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   __syncthreads();
   if (tid == 0) QE_TRACE(kTrTopK);
 
-  // ------------------------------------------------ expert phase (per warp)
+  // ---------------------------------------------------------- expert phase
   const int nBc = g.nB > cta ? (g.nB - cta + G - 1) / G : 0;
   const int own = g.nCB > cta ? (g.nCB - cta + G - 1) / G : 0;
-  const int nItems = nBc + K * own;
-  const int MR = g.max_own * g.RC;  // rows of one expert's slice of ycomb
-  const int nmine = warp < nItems ? (nItems - warp + kWarps - 1) / kWarps : 0;
-  if (!*abort_flag && nmine > 0) {
+  const int MR = g.max_own * kRC;  // rows of one expert's slice of ycomb
+  // down work of this warp: expert k = warp % K, blocks wi, wi + nwk, ...
+  const int ck = warp % K, wi = warp / K, nwk = (kWarps - ck + K - 1) / K;
+  const int myblocks = wi < own ? (own - wi + nwk - 1) / nwk : 0;
+
+  const qe_qmat dmat = misc->ex[ck].down;
+  const int nrow = myblocks * kRC;  // down rows of this warp
+  DownRows R;
+  if (tid < kMaxK) misc->hamax[tid] = 0u;
+  __syncthreads();
+
+  if (!*abort_flag) {
+    // ------------------------------------------------ gate/up, 4-warp groups
+    const int gr = warp >> 2, qd = warp & 3;
+    const int ng = nBc > gr ? (nBc - gr + kGroups - 1) / kGroups : 0;
+    unsigned char* gring = smem + g.off_ring + (size_t)gr * g.nslot * g.slot;
+    const GateUpCtx cx = make_gateup_ctx(H);
     const uint64_t pol = policy_evict_first();
-    for (int q = 0; q < g.nslot && q < nmine; ++q)
-      issue_item(item_ref(warp + kWarps * q, nBc, own, cta, G, g), ring + (size_t)q * g.slot, misc, H, I, g,
-                 lane, pol);
-    for (int q = 0; q < nmine; ++q) {
-      const int j = warp + kWarps * q;
-      const ItemRef it = item_ref(j, nBc, own, cta, G, g);
-      unsigned char* sl = ring + (size_t)(q % g.nslot) * g.slot;
-      // groups committed after this item's own: the items already issued ahead
-      const int later = (q + g.nslot <= nmine ? g.nslot : nmine - q) - 1;
-      if (later >= 1) cp_async_wait<1>(); else cp_async_wait<0>();
+    // item t of this group is gate/up item gi = cta + G*(gr + 4t) of the
+    // grid: expert gi / nIB, rows (gi % nIB) * kRB
+    auto item_k = [&](int t, int* r0) {
+      const int gi = cta + G * (gr + kGroups * t);
+      const int k = gi / g.nIB;
+      *r0 = (gi - k * g.nIB) * kRB;
+      return k;
+    };
+    for (int t = 0; t < g.nslot && t < ng; ++t) {
+      int r0;
+      const int k = item_k(t, &r0);
+      issue_gateup(misc->ex[k], r0, gring + (size_t)t * g.slot, qd, cx, lane, pol);
+    }
+    float2 xs[16];
+    int xs_bits = 0;  // bits of the x' form cached in xs (0: none)
+    const bool cache = cx.nlc <= 32;  // one lane chunk of the quarter per lane
+    for (int t = 0; t < ng; ++t) {
+      int r0;
+      const int k = item_k(t, &r0);
+      unsigned char* sl = gring + (size_t)(t % g.nslot) * g.slot;
+      // copy groups committed after this item's: the items already issued ahead
+      const int later = (t + g.nslot <= ng ? g.nslot : ng - t) - 1;
+      if (later >= 2) cp_async_wait<2>();
+      else if (later == 1) cp_async_wait<1>();
+      else cp_async_wait<0>();
       __syncwarp();
-      if (q == 0 && lane == 0) QE_TRACE(16 + warp);
-      if (it.gateup) {
-        float* hdst = p.hbuf + (size_t)it.k * I + it.r0;
-        if (misc->ex[it.k].gate.bits == 4)
-          gateup_dispatch<4>(g.RB, sl, H, xp4, xsum, misc->xK, hdst, lane);
-        else
-          gateup_dispatch<2>(g.RB, sl, H, xp2, xsum, misc->xK, hdst, lane);
-        __syncwarp();
-        if (lane == 0) {
-          __threadfence();
-          red_release_add(&ctl->ready[it.k], 1u);
-          if (p.trace) atomicMax(&misc->t_lastB, (unsigned long long)gtimer());
-        }
-      } else {
-        const int k = it.k;
-        const int dbits = misc->ex[k].down.bits;
-        // stage h_k in shared memory (first warp to need it) or wait for it
-        unsigned won = 0;
-        if (lane == 0) won = atomicCAS(&misc->claim[k], 0u, 1u) == 0u;
-        won = __shfl_sync(0xffffffffu, won, 0);
-        int ok = 1;
-        if (won) {
-          if (lane == 0) ok = wait_geq(&ctl->ready[k], (unsigned)g.nIB, deadline, abort_flag);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (ok) {
-            if (lane == 0 && k == 0) QE_TRACE(kTrHFirst);
-            if (lane == 0 && k == K - 1) QE_TRACE(kTrHLast);
-            float* hpk = hp + (size_t)k * I;
-            float* hsk = hsum + (size_t)k * (I / 32);
-            const float* hsrc = p.hbuf + (size_t)k * I;
-            float am = 0.f;
-            for (int c = lane; c < I; c += 32) am = fmaxf(am, fabsf(__ldcg(hsrc + c)));
-            const int Eh = xscale_exponent(warp_max(am));
-            for (int ch = 0; ch < I / 32; ++ch) {
-              const int c = ch * 32 + lane;
-              const float v = __ldcg(hsrc + c);
-              const float sm = warp_sum(v);
-              if (lane == 0) hsk[ch] = sm;
-              if (dbits == 4) hpk[swz_q4(c)] = xprime_q4(v, c, Eh);
-              else hpk[swz_q2(c)] = xprime_q2(v, c, Eh);
-            }
-            if (lane == 0) misc->hK[k] = acc_scale(Eh);
-            __threadfence_block();
-            __syncwarp();
-            if (lane == 0) *(volatile int*)&misc->hflag[k] = 1;
-          }
-        } else {
-          if (lane == 0) {
-            unsigned spins = 0;
-            while (*(volatile int*)&misc->hflag[k] == 0) {
-              if (*abort_flag || ((++spins & 15u) == 0 && gtimer() > deadline)) { ok = 0; break; }
-              __nanosleep(32);
-            }
-          }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          __threadfence_block();
-        }
-        if (!ok) {
-          if (lane == 0) { set_error(&ctl->err, QE_ERR_TIMEOUT); *abort_flag = 1; }
-          break;
-        }
-        float* ydst = ycomb + (size_t)k * MR + it.ob * g.RC;
-        const float* hpk = hp + (size_t)k * I;
-        const float* hsk = hsum + (size_t)k * (I / 32);
-        if (dbits == 4)
-          down_dispatch<4>(g.RC, sl, I, hpk, hsk, misc->hK[k], ydst, lane);
-        else
-          down_dispatch<2>(g.RC, sl, I, hpk, hsk, misc->hK[k], ydst, lane);
-        if (lane == 0 && p.trace) atomicMax(&misc->t_lastC, (unsigned long long)gtimer());
+      const int bits = misc->ex[k].gate.bits;
+      if (cache && xs_bits != bits && lane < cx.nlc) {
+        if (bits == 4) load_xs32_q4(xp4, qd * cx.nlc + lane, xs);
+        else load_xs32_q2(xp2, qd * cx.nlc + lane, xs);
       }
-      if (q == 0 && lane == 0) QE_TRACE(32 + warp);
+      xs_bits = bits;
+      const float s = bits == 4 ? gateup_partial<4>(sl, qd, cx, xp4, xsum, misc->xK, xs, cache, lane)
+                                : gateup_partial<2>(sl, qd, cx, xp2, xsum, misc->xK, xs, cache, lane);
+      float* red = misc->gred[gr][t & 1][qd];
+#pragma unroll
+      for (int i = 0; i < 2 * kRB; ++i)
+        if (lane == lane_of_reduced_row<2 * kRB>(i)) red[i] = s;
+      named_barrier(1 + gr, 128);
+      if (qd == 0 && lane < kRB) {
+        // lane rr: h of row r0 + rr = silu(g) * u from the four quarter sums
+        float gv = 0.f, uv = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          gv += misc->gred[gr][t & 1][q][lane];
+          uv += misc->gred[gr][t & 1][q][kRB + lane];
+        }
+        const float hv = gv / (1.0f + expf(-gv)) * uv;
+        p.hbuf[(size_t)k * I + r0 + lane] = hv;  // published once per CTA below
+        atomicMax(&misc->hamax[k], __float_as_uint(fabsf(hv)));
+      }
       __syncwarp();
-      // refill this slot with the item nslot places ahead
-      if (q + g.nslot < nmine)
-        issue_item(item_ref(warp + kWarps * (q + g.nslot), nBc, own, cta, G, g), sl, misc, H, I, g, lane, pol);
+      if (t + g.nslot < ng) {
+        int r1;
+        const int k1 = item_k(t + g.nslot, &r1);
+        issue_gateup(misc->ex[k1], r1, sl, qd, cx, lane, pol);
+      }
       if (*abort_flag) break;
     }
     cp_async_wait<0>();  // nothing may still be landing when the CTA exits
+    if (lane == 0) QE_TRACE(16 + warp);
+    // this warp's first down rows do not depend on h: load them now
+    if (nrow > 0 && lane < I / 32) down_load(dmat, cta, G, kRC, wi, nwk, 0, nrow < 8 ? nrow : 8, I, lane, R);
   }
+
+  // ------------------------------------- publish h, wait for every CTA's h
+  __syncthreads();
+  if (tid == 0) {
+    QE_TRACE(kTrLastB);
+    if (!*abort_flag) {
+      for (int k = 0; k < K; ++k) atomicMax(&ctl->hamax[k], misc->hamax[k]);
+      __threadfence();
+      atomicAdd(&ctl->h_ctr, 1u);
+      if (!wait_geq(&ctl->h_ctr, (unsigned)G, deadline, abort_flag)) {
+        set_error(&ctl->err, QE_ERR_TIMEOUT);
+        misc->abort = 1;
+      }
+      for (int k = 0; k < K; ++k) {
+        unsigned v;
+        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&ctl->hamax[k]) : "memory");
+        const int Eh = xscale_exponent(__uint_as_float(v));
+        misc->hK[k] = acc_scale(Eh);
+        misc->hamax[k] = (unsigned)Eh;  // reused: vector exponent of h_k
+      }
+    }
+    QE_TRACE(kTrHFirst);
+  }
+  __syncthreads();
+
+  // stage h in x' form, all warps: chunk ch of the K*I/32 chunks
+  if (!*abort_flag) {
+    const int per = I / 32;
+    // 8 chunks per pass, loads issued before any of them is used
+    for (int ch0 = warp; ch0 < K * per; ch0 += 8 * kWarps) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int ch = ch0 + i * kWarps;
+        if (ch < K * per) {
+          const int k = ch / per, lc = ch - k * per;
+          v[i] = __ldcg(p.hbuf + (size_t)k * I + lc * 32 + lane);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int ch = ch0 + i * kWarps;
+        if (ch < K * per) {
+          const int k = ch / per, lc = ch - k * per;
+          const int c = lc * 32 + lane;
+          const int Eh = (int)misc->hamax[k];
+          const float sm = warp_sum(v[i]);
+          if (lane == 0) hsum[(size_t)k * per + lc] = sm;
+          float* hpk = hp + (size_t)k * I;
+          if (misc->ex[k].down.bits == 4) hpk[swz_q4(c)] = xprime_q4(v[i], c, Eh);
+          else hpk[swz_q2(c)] = xprime_q2(v[i], c, Eh);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (tid == 0) QE_TRACE(kTrHLast);
+
+  // -------------------------------------------------------- down, warps
+  if (!*abort_flag && nrow > 0) {
+    const int k = ck;
+    const float* hpk = hp + (size_t)k * I;
+    const float* hsk = hsum + (size_t)k * (I / 32);
+    const float hK = misc->hK[k];
+    float* yk = ycomb + (size_t)k * MR;
+    for (int b0 = 0; b0 < nrow; b0 += 8) {
+      const int nr = nrow - b0 < 8 ? nrow - b0 : 8;
+      float yv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) yv[i] = 0.f;
+      for (int lc = lane; lc < I / 32; lc += 32) {
+        if (!(b0 == 0 && lc == lane)) down_load(dmat, cta, G, kRC, wi, nwk, b0, nr, I, lc, R);
+        if (dmat.bits == 4) down_accum<4>(R, nr, lc, hpk, hsk, hK, yv);
+        else down_accum<2>(R, nr, lc, hpk, hsk, hK, yv);
+      }
+      const float sred = warp_reduce_rows<8>(yv, lane);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (i < nr && lane == lane_of_reduced_row<8>(i)) {
+          const int ri = b0 + i, blk = ri / kRC;
+          yk[(wi + nwk * blk) * kRC + (ri - blk * kRC)] = sred;
+        }
+      }
+    }
+    if (lane == 0 && p.trace) atomicMax(&misc->t_lastC, (unsigned long long)gtimer());
+  }
+  if (lane == 0) QE_TRACE(32 + warp);
   __syncthreads();
   if (tid == 0) QE_TRACE(48);
 
   // ----------------------------------------------- combine of owned rows
   if (!*abort_flag) {
-    for (int lr = tid; lr < own * g.RC; lr += kFusedThreads) {
-      const int ob = lr / g.RC;
-      const int r = (cta + G * ob) * g.RC + (lr - ob * g.RC);
+    for (int lr = tid; lr < own * kRC; lr += kFusedThreads) {
+      const int ob = lr / kRC;
+      const int r = (cta + G * ob) * kRC + (lr - ob * kRC);
       float acc = 0.f;
       for (int k = 0; k < K; ++k) acc += misc->wk[k] * ycomb[(size_t)k * MR + lr];
       if (p.add_residual) acc += load_x(p, r);
@@ -574,15 +672,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
     QE_TRACE(53);
     if (prev == (unsigned)G - 1) {
       ctl->route_ctr = 0;
-      for (int k = 0; k < kMaxK; ++k) ctl->ready[k] = 0;
+      ctl->h_ctr = 0;
+      for (int k = 0; k < kMaxK; ++k) ctl->hamax[k] = 0;
       __threadfence();
       ctl->exit_ctr = 0;
       __threadfence();
     }
-    if (p.trace) {
-      p.trace[(size_t)cta * 64 + kTrLastB] = misc->t_lastB;
-      p.trace[(size_t)cta * 64 + kTrLastC] = misc->t_lastC;
-    }
+    if (p.trace) p.trace[(size_t)cta * 64 + kTrLastC] = misc->t_lastC;
     QE_TRACE(kTrEnd);
     if (p.trace) p.trace[(size_t)cta * 64 + 13] = clock64();
   }
@@ -595,35 +691,34 @@ static int gcd_int(int a, int b) { while (b) { int t = a % b; a = b; b = t; } re
 
 int fused_geometry(int H, int E, int K, int I, int sms, int smem_optin, FusedGeometry* out) {
   FusedGeometry g{};
-  // rows per item: every copied segment must be a multiple of 16 bytes
-  // (RB*H and RC*I multiples of 512)
-  g.RB = 8 / gcd_int(H / kGroup, 8);
-  g.RC = 8 / gcd_int(I / kGroup, 8);
-  if (g.RC < 4) g.RC = 4;
-  if (I % g.RB || H % g.RC) return QE_ERR_UNSUPPORTED;
+  // gate/up items of kRB rows in column quarters: H a multiple of 256 keeps
+  // every copied quarter row and scale segment a multiple of 16 bytes
+  if (H % 256 != 0 || I % kRB != 0 || H % kRC != 0) return QE_ERR_UNSUPPORTED;
   if (E > kRouterRows * sms) return QE_ERR_UNSUPPORTED;
   if (H > kChunkMax * 32 * kWarps) return QE_ERR_UNSUPPORTED;
-  g.nIB = I / g.RB;
+  g.RB = kRB;
+  g.RC = kRC;
+  g.nIB = I / kRB;
   g.nB = K * g.nIB;
-  g.nCB = H / g.RC;
+  g.nCB = H / kRC;
   g.grid = sms;
   g.max_own = (g.nCB + sms - 1) / sms;
-  const int slotB = g.RB * H + 4 * g.RB * (H / kGroup) * 2;
-  const int slotC = g.RC * I / 2 + 2 * g.RC * (I / kGroup) * 2;
-  g.slot = align_up(slotB > slotC ? slotB : slotC, 128);
+  const int srow = (H % 2048) == 0 ? H / 256 : H / kGroup;
+  g.slot = align_up(kRB * H + 4 * 4 * kRB * srow * 2, 128);
   int off = 0;
   g.off_xp4 = off; off = align_up(off + 4 * H, 128);
   g.off_xp2 = off; off = align_up(off + 4 * H, 128);
   g.off_xs = off; off = align_up(off + 4 * (H / 32), 128);
   g.off_hp = off; off = align_up(off + 4 * K * I, 128);
   g.off_hs = off; off = align_up(off + 4 * K * (I / 32), 128);
-  g.off_ycomb = off; off = align_up(off + 4 * K * g.max_own * g.RC, 128);
+  g.off_ycomb = off; off = align_up(off + 4 * K * g.max_own * kRC, 128);
   g.off_misc = off; off = align_up(off + (int)sizeof(FusedMisc), 1024);
   g.off_ring = off;
   const int budget = smem_optin - off;
-  g.nslot = budget >= 2 * kWarps * g.slot ? 2 : (budget >= kWarps * g.slot ? 1 : 0);
-  if (g.nslot == 0) return QE_ERR_UNSUPPORTED;
-  g.smem_bytes = off + g.nslot * kWarps * g.slot;
+  g.nslot = budget / (kGroups * g.slot);
+  if (g.nslot > 3) g.nslot = 3;
+  if (g.nslot < 1) return QE_ERR_UNSUPPORTED;
+  g.smem_bytes = off + g.nslot * kGroups * g.slot;
   *out = g;
   return QE_OK;
 }

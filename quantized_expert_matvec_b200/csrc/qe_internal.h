@@ -20,11 +20,11 @@ struct WsControl {
   int err;             // first device-side error (QE_ERR_*), 0 if none
   unsigned route_ctr;  // fused kernel: CTAs past the router
   unsigned exit_ctr;   // fused kernel: CTAs finished
-  unsigned pad0;
-  unsigned ready[kMaxK];  // fused kernel: CTAs done with expert k's gate/up
-  unsigned pad1[12];
+  unsigned h_ctr;      // fused kernel: CTAs that published their h rows
+  unsigned hamax[kMaxK];  // fused kernel: max |h_k| as float bits
+  unsigned pad[44];
 };
-static_assert(sizeof(WsControl) == 128, "control block");
+static_assert(sizeof(WsControl) == 256, "control block");
 
 // Offsets (bytes) of the workspace regions for T tokens.
 struct WsLayout {
@@ -56,11 +56,11 @@ WsLayout ws_layout(int H, int E, int K, int I, int T);
 
 // Geometry of the fused single-token kernel.
 struct FusedGeometry {
-  int RB, RC;            // rows of a gate/up item, rows of a down item
+  int RB, RC;            // rows of a gate/up item, rows of a down block
   int nIB, nB, nCB;      // gate/up items per expert, gate/up items, output blocks
   int max_own;           // most output blocks one CTA owns
-  int slot;              // bytes of one warp ring slot (largest item)
-  int nslot;             // slots per warp (1 or 2)
+  int slot;              // bytes of one group ring slot
+  int nslot;             // slots per 4-warp group
   int off_ring, off_xp4, off_xp2, off_xs, off_hp, off_hs, off_ycomb, off_misc;
   int smem_bytes;
   int grid;

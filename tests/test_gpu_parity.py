@@ -103,18 +103,20 @@ def test_fused_tiny_layer(q, bits, residual):
     assert max(e for e in errs if e is not None) < 1e-5
 
 
-def test_fused_ragged_mixed_bits_gamma_offset(q):
-    """Odd sizes (hidden 320, intermediate 192, 37 experts, top-3): items do
-    not divide evenly over the CTAs; half the experts are 2-bit; random gamma
-    and a Zipf logit offset."""
-    cfg = q.Cfg(320, 37, 3, 192)
-    gamma = np.random.default_rng(1).uniform(0.5, 1.5, 320).astype(np.float32)
+@pytest.mark.parametrize("H", [768, 320])
+def test_ragged_mixed_bits_gamma_offset(q, H):
+    """Odd sizes (intermediate 192, 37 experts, top-3): items do not divide
+    evenly over the CTAs; half the experts are 2-bit; random gamma and a Zipf
+    logit offset.  Hidden 768 runs the fused kernel; hidden 320 (not a
+    multiple of 256) takes the multi-kernel path for a single token."""
+    cfg = q.Cfg(H, 37, 3, 192)
+    gamma = np.random.default_rng(1).uniform(0.5, 1.5, H).astype(np.float32)
     off = synth.zipf_logit_offset(5, 1, 37)
     dl = DevLayer(q, cfg, seed=5, layer=1, bits_of=lambda e: 4 if e % 2 == 0 else 2, offset=off, gamma=gamma)
-    x = dev_tokens(5, 100, 12, 320)
+    x = dev_tokens(5, 100, 12, H)
     out, idx, w = run_fused(q, dl, x, residual=True)
     for t in range(12):
-        ref = dl.oracle(host_x_f64(5, 100 + t, 320), residual=True)
+        ref = dl.oracle(host_x_f64(5, 100 + t, H), residual=True)
         check(dl, out[t], idx[t], w[t], ref)
 
 
@@ -330,3 +332,46 @@ def test_bounded_wait_times_out_and_recovers(q):
     q.qe_workspace_init(ws)
     o, i, w = run_fused(q, dl, x, ws=ws)
     check(dl, o[0], i[0], w[0], dl.oracle(host_x_f64(0, 0, 256)))
+
+
+def test_c1_fused_matches_multikernel_path_on_many_tokens(q, c1_layer):
+    """256 tokens through the fused kernel (a CUDA graph of single-token
+    steps) against the separate route / expert-FFN / combine kernels on the
+    same tokens.  Both are fp32 GPU paths, so they agree far inside the oracle
+    tolerance; a missed barrier inside the fused kernel would read
+    unfinished partial sums and show up here."""
+    import torch
+    dl = c1_layer
+    cfg = dl.cfg
+    n = 256
+    x = dev_tokens(0, 20000, n, 4096)
+    out = torch.zeros((n, 4096), dtype=torch.float32, device="cuda")
+    idx = torch.zeros((n, 4), dtype=torch.int32, device="cuda")
+    ws = q.workspace(cfg, 1)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        q.moe_layer_step(cfg, dl.layer_struct, x[0:1], out[0:1], True, idx[0:1], None, ws, stream=s)
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for t in range(n):
+                q.moe_layer_step(cfg, dl.layer_struct, x[t:t + 1], out[t:t + 1], True, idx[t:t + 1], None, ws,
+                                 stream=s)
+        g.replay()
+        s.synchronize()
+    assert q.qe_workspace_status(ws, s) == q.QE_OK
+    xn = torch.empty((n, 4096), dtype=torch.float32, device="cuda")
+    idx2 = torch.empty((n, 4), dtype=torch.int32, device="cuda")
+    w2 = torch.empty((n, 4), dtype=torch.float32, device="cuda")
+    y2 = torch.empty((n, 4, 4096), dtype=torch.float32, device="cuda")
+    out2 = torch.empty((n, 4096), dtype=torch.float32, device="cuda")
+    ws2 = q.workspace(cfg, n)
+    q.moe_route(cfg, x, None, dl.W, None, xn, idx2, w2, ws2)
+    q.moe_expert_ffn_q4(cfg, dl.table, xn, idx2, y2, ws2)
+    q.moe_combine(y2, w2, x, out2)
+    assert q.qe_workspace_status(ws2) == q.QE_OK
+    same = (idx == idx2).all(dim=1)
+    assert int(same.sum()) >= n - 2
+    a, b = out[same].double(), out2[same].double()
+    err = ((a - b).abs().amax(dim=1) / b.abs().amax(dim=1)).max().item()
+    assert err < 2e-5, err
