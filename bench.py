@@ -1,16 +1,18 @@
 #!/usr/bin/env python
 """Benchmark of the quantized MoE expert step on B200.
 
-Default workload (one decode MoE layer shaped like the Flash-MoE pages'
-model): hidden 4096, 512 experts, top-4 renormalised, expert intermediate
-1024, 4-bit affine group-64 experts (bf16 scale/bias), SwiGLU, batch 1 token
-fp32, all experts resident in HBM.  One step = one token through the whole
-layer (RMSNorm, router, top-K, 4 expert FFNs, combine) = one launch of the
-fused kernel.  Tokens are distinct (a stream of seeded N(0,1) vectors), so the
-routing scatters over the 3.6 GB expert pool, far larger than L2.
+Default workload (the configuration the headline metric is quoted on): one
+decode MoE layer shaped like the Flash-MoE pages' model, hidden 4096, 512
+experts, top-4 renormalised, expert intermediate 1024, 4-bit affine group-64
+experts (bf16 scale/bias), SwiGLU, batch 1 token fp32, all experts resident
+in HBM.  One step = one token through the whole layer (RMSNorm, router,
+top-K, 4 expert FFNs, combine) = one launch of the fused kernel.  Tokens are
+distinct seeded N(0,1) vectors, so routing scatters over the 3.6 GB expert
+pool, far larger than L2.
 
-Prints one JSON line (see the design doc for every key).  ``--impl reference``
-times the fp64 CPU oracle on the host cores instead.
+Other workloads (--workload): c0 tiny layer, c4 batched decode (256 tokens
+per step, grouped experts).  Prints one JSON line; ``--impl reference`` times
+the fp64 CPU oracle on the host cores instead.
 """
 from __future__ import annotations
 
@@ -30,33 +32,28 @@ sys.path.insert(0, os.path.join(ROOT, "tests"))
 
 import numpy as np  # noqa: E402
 
+EPS32 = float(np.float32(1e-6))
+
 WORKLOADS = {
-    "c1": dict(H=4096, E=512, K=4, I=1024, bits=4,
+    "c1": dict(H=4096, E=512, K=4, I=1024, bits=4, T=1,
                name="one decode MoE layer: hidden 4096, 512 experts, top-4 renormalised, intermediate 1024, "
-                    "4-bit affine g64 bf16 scale/bias, SwiGLU, batch 1 token fp32, all experts in HBM"),
-    "c0": dict(H=256, E=16, K=2, I=64, bits=4,
-               name="tiny MoE FFN: hidden 256, 16 experts, top-2, intermediate 64, 4-bit g64, 1 token"),
+                    "4-bit affine g64 bf16 scale/bias, SwiGLU, batch 1 token fp32, all experts in HBM",
+               metric="MoE-layer decode tokens/s at 1 B200"),
+    "c0": dict(H=256, E=16, K=2, I=64, bits=4, T=1,
+               name="tiny MoE FFN: hidden 256, 16 experts, top-2, intermediate 64, 4-bit g64, 1 token",
+               metric="MoE-layer decode tokens/s at 1 B200 (tiny layer)"),
+    "c4": dict(H=4096, E=512, K=4, I=1024, bits=4, T=256,
+               name="batched decode of the one-layer workload: 256 bf16 tokens per step, own top-4 of 512 each, "
+                    "grouped per expert, 4-bit g64 experts in HBM, uniform routing",
+               metric="MoE-layer batched decode tokens/s at 1 B200"),
 }
 
-METRIC = "MoE-layer decode tokens/s at 1 B200"
 UNIT = "tokens/s"
-EPS32 = float(np.float32(1e-6))
-KERNEL_NAME = "qe_fused_layer_kernel"
 
 
 def expert_bytes(H, I, bits):
     n = 3 * H * I
     return n * bits // 8 + 2 * 2 * n // 64
-
-
-def algorithmic_bytes(wl):
-    """Bytes one fused launch must move: K experts' packed weights and
-    scales/biases, the fp32 router, x in and out."""
-    H, E, K, I, bits = wl["H"], wl["E"], wl["K"], wl["I"], wl["bits"]
-    experts = K * expert_bytes(H, I, bits)
-    router = E * H * 4
-    act = 2 * H * 4
-    return experts, router, act
 
 
 def kernel_source_hash():
@@ -71,7 +68,7 @@ def kernel_source_hash():
 def load_traffic(workload):
     """Per-launch DRAM bytes from the committed ncu summary, if it was taken
     on the current kernel sources."""
-    path = os.path.join(ROOT, "profiles", f"fused_layer_{workload}_traffic.json")
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
     try:
         d = json.load(open(path))
     except (OSError, ValueError):
@@ -143,17 +140,24 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 
 def oracle_token_time(wl, seed, tokens, row_fraction=1.0, nthreads=None):
-    """Time the fp64 oracle on `tokens` tokens of the workload: routing in
-    full, expert matvecs on a leading fraction of the rows.  Expert weights
-    are regenerated before the timed calls.  Returns (seconds per token
-    extrapolated to all rows, threads, seconds measured)."""
+    """Time the fp64 oracle on whole tokens of the workload's layer: routing
+    in full, expert matvecs on a leading fraction of the rows (extrapolated).
+    Expert weights are regenerated before the timed calls.  Returns (seconds
+    per token, threads, seconds measured)."""
     import oracle
     import synth
     H, E, K, I, bits = wl["H"], wl["E"], wl["K"], wl["I"], wl["bits"]
+    bf16 = wl["T"] > 1
     nthreads = nthreads or os.cpu_count() or 1
     W = synth.host_router(seed, 0, E, H)
-    xs = [synth.host_tokens(seed, t, 1, H)[0].astype(np.float64) for t in tokens]
-    # untimed: find the experts, regenerate them
+
+    def tok(t):
+        x = synth.host_tokens(seed, t, 1, H, bf16=bf16)[0]
+        if bf16:
+            return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        return x.astype(np.float64)
+
+    xs = [tok(t) for t in tokens]
     cache = {}
     for x in xs:
         idx, _ = oracle.topk(oracle.router(W, oracle.rmsnorm(x, None, EPS32), None, nthreads), K)
@@ -193,12 +197,12 @@ def oracle_token_time(wl, seed, tokens, row_fraction=1.0, nthreads=None):
 
 def cpu_baseline(wl, seed, budget_s=15.0):
     """The oracle on a bounded sample of the workload (whole tokens)."""
-    per1, nth, spent = oracle_token_time(wl, seed, [1_000_000])
+    per1, nth, _ = oracle_token_time(wl, seed, [1_000_000])
     n = max(1, min(64, int(budget_s / max(per1, 1e-9))))
-    per, nth, spent2 = oracle_token_time(wl, seed, list(range(1_000_001, 1_000_001 + n)))
+    per, nth, spent = oracle_token_time(wl, seed, list(range(1_000_001, 1_000_001 + n)))
     return {"value": 1.0 / per, "unit": UNIT, "cores": nth, "kind": "oracle",
             "sample": f"{n} whole tokens of the workload (fp64 oracle, OpenMP over rows, {nth} threads), "
-                      f"{spent2:.1f} s of CPU time"}
+                      f"{spent:.1f} s of CPU time"}
 
 
 def run_reference(args, wl, rank, world):
@@ -207,7 +211,7 @@ def run_reference(args, wl, rank, world):
     K, W = args.steps, args.warmup
     per_full, nth, _ = oracle_token_time(wl, args.seed, [2_000_000])
     budget = 150.0  # seconds for all K + W steps
-    frac = min(1.0, max(1.0 / 256, (budget / (K + W)) / max(per_full, 1e-9)))
+    frac = min(1.0, max(1.0 / 512, (budget / (K + W)) / max(per_full * wl["T"], 1e-9)))
     for t in range(W):
         oracle_token_time(wl, args.seed, [3_000_000 + t], frac, nth)
     t0 = time.perf_counter()
@@ -217,8 +221,8 @@ def run_reference(args, wl, rank, world):
         per.append(p)
     wall = time.perf_counter() - t0
     value = K / sum(per)
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": W,
-            "ms_per_step": 1000.0 * sum(per) / K, "higher_is_better": True, "scaling": "weak",
+    line = {"metric": wl["metric"], "value": value, "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": W,
+            "ms_per_step": 1000.0 * sum(per) * wl["T"] / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": wl["name"], "tokens": "distinct seeded N(0,1) tokens"},
             "cpu_baseline": {"kind": "oracle", "cores": nth, "value": value, "unit": UNIT,
@@ -232,40 +236,52 @@ def run_reference(args, wl, rank, world):
 # our arm
 # --------------------------------------------------------------------------
 
+class LayerSetup:
+    """One resident layer (pool, router, workspace) and a token stream."""
+
+    def __init__(self, q, wl, seed, dev, n_tok, tok0):
+        import torch
+        from _util import dev_router, dev_tokens, fill_pool
+        H, E, K, I, bits, T = wl["H"], wl["E"], wl["K"], wl["I"], wl["bits"], wl["T"]
+        self.wl = wl
+        self.cfg = q.Cfg(H, E, K, I, 64, EPS32)
+        self.pool = q.ExpertPool(self.cfg, E, bits, device=dev)
+        fill_pool(self.pool, seed, 0)
+        self.W = dev_router(seed, 0, E, H, device=dev)
+        self.layer = q.Layer(self.W.data_ptr(), None, None, self.pool.table.data_ptr())
+        self.ws = q.workspace(self.cfg, T, device=dev)
+        self.x = dev_tokens(seed, tok0, n_tok, H, bf16=T > 1, device=dev)
+        self.out = torch.empty((n_tok, H), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((n_tok, K), dtype=torch.int32, device=dev)
+        self.w = torch.empty((n_tok, K), dtype=torch.float32, device=dev)
+        self.n_tok = n_tok
+        self.T = T
+
+
 def run_ours(args, wl, rank, world, local_rank):
     import torch
     import quantized_expert_matvec_b200 as q
-    from _util import dev_router, dev_tokens, fill_pool
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    H, E, K, I, bits = wl["H"], wl["E"], wl["K"], wl["I"], wl["bits"]
-    cfg = q.Cfg(H, E, K, I, 64, EPS32)
+    H, E, K, I, bits, T = wl["H"], wl["E"], wl["K"], wl["I"], wl["bits"], wl["T"]
     seed = args.seed
-    pool = q.ExpertPool(cfg, E, bits, device=dev)
-    fill_pool(pool, seed, 0)
-    Wr = dev_router(seed, 0, E, H, device=dev)
-    layer = q.Layer(Wr.data_ptr(), None, None, pool.table.data_ptr())
-    ws = q.workspace(cfg, 1, device=dev)
-    chunk = 1024
-    n_chunks = 8
-    n_tok = chunk * n_chunks
-    tok0 = 10_000_000 * (rank + 1)
-    x = dev_tokens(seed, tok0, n_tok, H, device=dev)
-    out = torch.empty((n_tok, H), dtype=torch.float32, device=dev)
-    idx = torch.empty((n_tok, K), dtype=torch.int32, device=dev)
-    wts = torch.empty((n_tok, K), dtype=torch.float32, device=dev)
+    chunk = 1024 if T == 1 else 8          # steps per captured graph
+    n_chunks = 8 if T == 1 else 4
+    n_tok = chunk * n_chunks * T
+    ls = LayerSetup(q, wl, seed, dev, n_tok, 10_000_000 * (rank + 1))
     s = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
 
-    def step(t, stream):
-        q.moe_layer_step(cfg, layer, x[t:t + 1], out[t:t + 1], False, idx[t:t + 1], wts[t:t + 1], ws,
-                         stream=stream)
+    def step(i, stream):
+        t0 = (i * T) % n_tok
+        q.moe_layer_step(ls.cfg, ls.layer, ls.x[t0:t0 + T], ls.out[t0:t0 + T], False, ls.idx[t0:t0 + T],
+                         ls.w[t0:t0 + T], ls.ws, stream=stream)
 
     def capture(first, count):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=s):
             for i in range(count):
-                step((first + i) % n_tok, s)
+                step(first + i, s)
         return g
 
     with torch.cuda.stream(s):
@@ -274,9 +290,9 @@ def run_ours(args, wl, rank, world, local_rank):
         graphs = [capture(c * chunk, chunk) for c in range(n_chunks)]
         rem = args.steps % chunk
         rem_graph = capture(0, rem) if rem else None
-        warm_graph = capture(0, args.warmup) if args.warmup else None
+        warm_graph = capture(0, min(args.warmup, chunk * n_chunks))
     torch.cuda.synchronize()
-    if q.qe_workspace_status(ws, s) != q.QE_OK:
+    if q.qe_workspace_status(ls.ws, s) != q.QE_OK:
         raise RuntimeError("device status after capture: " + q.qe_last_error())
 
     def barrier():
@@ -284,10 +300,8 @@ def run_ours(args, wl, rank, world, local_rank):
             import torch.distributed as dist
             dist.barrier()
 
-    # warm-up
     with torch.cuda.stream(s):
-        if warm_graph is not None:
-            warm_graph.replay()
+        warm_graph.replay()
     s.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -310,8 +324,7 @@ def run_ours(args, wl, rank, world, local_rank):
     barrier()
     clocks = sampler.stop() if sampler else None
     ms = ev0.elapsed_time(ev1)
-    status = q.qe_workspace_status(ws, s)
-    if status != q.QE_OK:
+    if q.qe_workspace_status(ls.ws, s) != q.QE_OK:
         raise RuntimeError("device status after timing: " + q.qe_last_error())
     ms_max = ms
     if world > 1:
@@ -319,63 +332,73 @@ def run_ours(args, wl, rank, world, local_rank):
         tt = torch.tensor([ms], dtype=torch.float64, device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         ms_max = float(tt.item())
-    value = world * args.steps / (ms_max / 1000.0)
+    value = world * args.steps * T / (ms_max / 1000.0)
+
+    # distinct experts touched per step (from the routing of the timed steps)
+    idx_h = ls.idx.cpu().numpy().reshape(-1, T * K)
+    distinct = float(np.mean([len(np.unique(r)) for r in idx_h[: max(1, min(len(idx_h), chunk * n_chunks))]]))
 
     # ---------------------------------------------------------------- e2e
-    n_e2e = min(args.steps, 2048)
-    x_host = x[:n_e2e].cpu().pin_memory()
-    out_host = torch.empty((n_e2e, H), dtype=torch.float32).pin_memory()
-    xin = torch.empty((1, H), dtype=torch.float32, device=dev)
-    res = torch.empty((1, H), dtype=torch.float32, device=dev)
+    n_e2e = min(args.steps, 2048 if T == 1 else 64)
+    x_host = ls.x[: max(T, 1) * min(n_e2e, ls.n_tok // T)].cpu().pin_memory()
+    out_host = torch.empty((T, H), dtype=torch.float32).pin_memory()
+    xin = torch.empty((T, H), dtype=ls.x.dtype, device=dev)
+    res = torch.empty((T, H), dtype=torch.float32, device=dev)
+    nb = x_host.shape[0] // T
+
+    def e2e_step(i):
+        b = (i % nb) * T
+        xin.copy_(x_host[b:b + T], non_blocking=True)
+        q.moe_layer_step(ls.cfg, ls.layer, xin, res, False, None, None, ls.ws, stream=s)
+        out_host.copy_(res, non_blocking=True)
+        s.synchronize()
+
     with torch.cuda.stream(s):
-        for t in range(8):
-            xin.copy_(x_host[t:t + 1], non_blocking=True)
-            q.moe_layer_step(cfg, layer, xin, res, False, None, None, ws, stream=s)
-            out_host[t:t + 1].copy_(res, non_blocking=True)
-            s.synchronize()
+        for i in range(4):
+            e2e_step(i)
     barrier()
     t0 = time.perf_counter()
     with torch.cuda.stream(s):
-        for t in range(n_e2e):
-            xin.copy_(x_host[t:t + 1], non_blocking=True)
-            q.moe_layer_step(cfg, layer, xin, res, False, None, None, ws, stream=s)
-            out_host[t:t + 1].copy_(res, non_blocking=True)
-            s.synchronize()
+        for i in range(n_e2e):
+            e2e_step(i)
     e2e_s = time.perf_counter() - t0
     if world > 1:
         import torch.distributed as dist
         tt = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         e2e_s = float(tt.item())
-    e2e_value = world * n_e2e / e2e_s
+    e2e_value = world * n_e2e * T / e2e_s
 
     if rank != 0:
         return
     peaks, peak_kind = measured_peaks()
-    exp_b, rout_b, act_b = algorithmic_bytes(wl)
-    per_launch_s = (ms / 1000.0) / args.steps
-    alg = exp_b + rout_b + act_b
-    achieved = alg / per_launch_s / 1e9
+    per_step_s = (ms / 1000.0) / args.steps
+    exp_b = distinct * expert_bytes(H, I, bits)
+    alg = exp_b + E * H * 4 + T * H * (2 if T > 1 else 4) + T * H * 4
+    achieved = alg / per_step_s / 1e9
     peak = float(peaks["hbm_gbs"])
-    traffic = load_traffic(args.workload)
     cpu = None if args.no_cpu_baseline else cpu_baseline(wl, seed)
+    kern = "qe_fused_layer_kernel" if T == 1 else "grouped_expert_kernel (+ route, group, combine)"
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": wl["metric"], "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": wl["name"], "batch": 1, "tokens_distinct": n_tok,
+        "config": {"workload": wl["name"], "tokens_per_step": T, "tokens_distinct": ls.n_tok,
                    "l2": "inputs larger than L2: 3.6 GB expert pool, routing scatters over all 512 experts",
-                   "launch": "CUDA graphs of 1024 single-token layer steps, one fused persistent kernel each",
+                   "launch": f"CUDA graphs of {chunk} layer steps",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
-                     "kernel": KERNEL_NAME, "algorithmic_bytes_per_launch": alg},
-        "expert_gbs": exp_b / per_launch_s / 1e9,
-        "expert_frac": exp_b / per_launch_s / 1e9 / peak,
+                     "frac": achieved / peak, "traffic": load_traffic(args.workload), "peak_source": peak_kind,
+                     "kernel": kern, "algorithmic_bytes_per_launch": alg,
+                     "duration": "whole step (launch gaps included)"},
+        "expert_gbs": exp_b / per_step_s / 1e9,
+        "expert_frac": exp_b / per_step_s / 1e9 / peak,
+        "distinct_experts_per_step": distinct,
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": H * 4, "d2h_bytes_per_step": H * 4,
-                "steps": n_e2e, "how": "per token: pinned H2D of x, moe_layer_step, D2H of out, stream sync"},
-        "gpu_launches": args.steps,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * H * ls.x.element_size(),
+                "d2h_bytes_per_step": T * H * 4, "steps": n_e2e,
+                "how": "per step: pinned H2D of x, moe_layer_step, D2H of out, stream sync"},
+        "gpu_launches": args.steps * (1 if T == 1 else 6),
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
@@ -384,16 +407,19 @@ def run_ours(args, wl, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=65536)
-    ap.add_argument("--warmup", type=int, default=1024)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="c1", choices=sorted(WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
-    if args.warmup < 3:
-        args.warmup = 3
     wl = WORKLOADS[args.workload]
+    if args.steps is None:
+        args.steps = 32768 if wl["T"] == 1 else 64
+    if args.warmup is None:
+        args.warmup = 256 if wl["T"] == 1 else 8
+    args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -52,10 +52,10 @@ WsLayout ws_layout(int H, int E, int K, int I, int T) {
   L.y = take(4 * t * K * H);
   L.idx = take(4 * t * K);
   L.w = take(4 * t * K);
-  L.grp_count = take(4 * (size_t)E);
+  L.grp_count = take(4 * ((size_t)E + 2));
   L.grp_start = take(4 * ((size_t)E + 1));
   L.grp_list = take(4 * t * K);
-  L.grp_tiles = take(16 * (t * K + E));
+  L.grp_order = take(4 * (size_t)E);
   L.total = off;
   return L;
 }
@@ -324,8 +324,19 @@ int moe_layer_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_
   rc = route_impl(c, x, x_dtype, layer->gamma, layer->router_w, layer->logit_offset, T, nullptr, idx, w, ws, ws_bytes,
                   true, s);
   if (rc) return rc;
-  rc = ffn_impl(c, layer->experts, at<float>(ws, L.xn), idx, T, at<float>(ws, L.y), ws, ws_bytes, 0, true, s);
-  if (rc) return rc;
+  {
+    GroupedParams gp{};
+    gp.H = c->hidden; gp.E = c->n_experts; gp.K = c->top_k; gp.I = c->inter; gp.T = T;
+    gp.experts = layer->experts; gp.idx = idx; gp.w = w;
+    gp.xp4 = at<float>(ws, L.xp4); gp.xp2 = at<float>(ws, L.xp2); gp.xsum = at<float>(ws, L.xsum);
+    gp.xexp = at<int>(ws, L.xexp);
+    gp.y = at<float>(ws, L.y);
+    gp.grp_count = at<int>(ws, L.grp_count); gp.grp_start = at<int>(ws, L.grp_start);
+    gp.grp_list = at<int>(ws, L.grp_list); gp.grp_order = at<int>(ws, L.grp_order);
+    gp.err = &at<WsControl>(ws, L.control)->err;
+    cudaError_t ge = launch_grouped(gp, s);
+    if (ge != cudaSuccess) return cuda_fail(ge, "moe_layer_step grouped experts");
+  }
   cudaError_t e = launch_combine(at<float>(ws, L.y), w, add_residual ? x : nullptr, x_dtype == QE_BF16, T,
                                  c->top_k, c->hidden, out, s);
   if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step combine");

@@ -45,10 +45,10 @@ struct WsLayout {
   size_t y;         // float  [T*K*H] expert outputs
   size_t idx;       // int32  [T*K]
   size_t w;         // float  [T*K]
-  size_t grp_count; // int    [E]    assignments per expert
+  size_t grp_count; // int    [E+2]  assignments per expert, active count, work counter
   size_t grp_start; // int    [E+1]
   size_t grp_list;  // int    [T*K]  assignment ids (t*K+k) sorted by expert
-  size_t grp_tiles; // int4   [T*K + E] work tiles of the grouped kernels
+  size_t grp_order; // int    [E]    active experts, most tokens first
   size_t total;
 };
 
@@ -154,10 +154,10 @@ struct GroupedParams {
   int* hexp;
   unsigned* hamax;
   float* y;
-  int* grp_count;
-  int* grp_start;
-  int* grp_list;
-  int4* grp_tiles;
+  int* grp_count;     // [E + 2]: counts, then active-expert count and work counter
+  int* grp_start;     // [E + 1]
+  int* grp_list;      // [T*K]
+  int* grp_order;     // [E]
   const void* x;     // residual source
   int x_bf16;
   int add_residual;
@@ -165,5 +165,6 @@ struct GroupedParams {
   int* err;
 };
 cudaError_t launch_grouped(const GroupedParams& p, cudaStream_t s);
+int grouped_tile(int H, int I, int smem_optin);
 
 }  // namespace qe

@@ -97,42 +97,45 @@ __global__ void __launch_bounds__(256) route_logits_gemv_kernel(const RouteParam
   }
 }
 
-// Router logits for many tokens: fp64 tiled product, 64 experts x 64 tokens
-// per CTA, 4x4 outputs per thread, 16-column steps through shared memory.
-constexpr int kRT = 64, kRK = 16;
+// Router logits for many tokens: fp64 tiled product, 32 experts x 32
+// tokens per CTA (enough CTAs to cover the SMs), 2x2 outputs per thread,
+// 32-column steps through shared memory with float4 loads of W.
+constexpr int kRT = 32, kRK = 32;
 __global__ void __launch_bounds__(256) route_logits_tiled_kernel(const RouteParams p) {
-  __shared__ __align__(16) double sW[kRK][kRT];
-  __shared__ __align__(16) double sX[kRK][kRT];
+  __shared__ __align__(16) double sW[kRK][kRT + 2];
+  __shared__ __align__(16) double sX[kRK][kRT + 2];
   const int H = p.H, E = p.E, T = p.T;
   const int e0 = blockIdx.x * kRT, t0 = blockIdx.y * kRT;
   const int tid = threadIdx.x;
-  const int te = (tid & 15) * 4, tt = (tid >> 4) * 4;
-  double acc[4][4] = {};
+  const int te = (tid & 15) * 2, tt = (tid >> 4) * 2;
+  double acc[2][2] = {};
   for (int c0 = 0; c0 < H; c0 += kRK) {
-    for (int i = tid; i < kRT * kRK; i += 256) {
-      const int r = i / kRK, c = i % kRK;
+    // 32 rows x 32 columns of W (fp32 -> fp64) and of x*gamma (fp64)
+    {
+      const int r = tid >> 3, c4 = (tid & 7) * 4;
       const int e = e0 + r, t = t0 + r;
-      sW[c][r] = e < E ? (double)p.router_w[(size_t)e * H + c0 + c] : 0.0;
-      sX[c][r] = t < T ? p.xg[(size_t)t * H + c0 + c] : 0.0;
+      if (e < E) {
+        const float4 v = *(const float4*)(p.router_w + (size_t)e * H + c0 + c4);
+        sW[c4][r] = v.x; sW[c4 + 1][r] = v.y; sW[c4 + 2][r] = v.z; sW[c4 + 3][r] = v.w;
+      } else {
+        sW[c4][r] = 0.0; sW[c4 + 1][r] = 0.0; sW[c4 + 2][r] = 0.0; sW[c4 + 3][r] = 0.0;
+      }
+      for (int u = 0; u < 4; ++u) sX[c4 + u][r] = t < T ? p.xg[(size_t)t * H + c0 + c4 + u] : 0.0;
     }
     __syncthreads();
-#pragma unroll
+#pragma unroll 8
     for (int c = 0; c < kRK; ++c) {
-      const double2 w01 = *(const double2*)&sW[c][te];
-      const double2 w23 = *(const double2*)&sW[c][te + 2];
-      const double2 x01 = *(const double2*)&sX[c][tt];
-      const double2 x23 = *(const double2*)&sX[c][tt + 2];
-      const double wv[4] = {w01.x, w01.y, w23.x, w23.y};
-      const double xv[4] = {x01.x, x01.y, x23.x, x23.y};
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fma(wv[a], xv[b], acc[a][b]);
+      const double w0 = sW[c][te], w1 = sW[c][te + 1];
+      const double x0 = sX[c][tt], x1 = sX[c][tt + 1];
+      acc[0][0] = fma(w0, x0, acc[0][0]);
+      acc[0][1] = fma(w0, x1, acc[0][1]);
+      acc[1][0] = fma(w1, x0, acc[1][0]);
+      acc[1][1] = fma(w1, x1, acc[1][1]);
     }
     __syncthreads();
   }
-  for (int a = 0; a < 4; ++a)
-    for (int b = 0; b < 4; ++b) {
+  for (int a = 0; a < 2; ++a)
+    for (int b = 0; b < 2; ++b) {
       const int e = e0 + te + a, t = t0 + tt + b;
       if (e < E && t < T)
         p.logits[(size_t)t * E + e] = acc[a][b] * p.rinv[t] + (p.offset ? (double)p.offset[e] : 0.0);

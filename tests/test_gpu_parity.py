@@ -375,3 +375,45 @@ def test_c1_fused_matches_multikernel_path_on_many_tokens(q, c1_layer):
     a, b = out[same].double(), out2[same].double()
     err = ((a - b).abs().amax(dim=1) / b.abs().amax(dim=1)).max().item()
     assert err < 2e-5, err
+
+
+def test_batched_skewed_routing_many_tokens_per_expert(q):
+    """Every token's top expert is the same (a +8 logit offset), so one
+    expert serves all 40 tokens: several token tiles over its weights."""
+    import torch
+    cfg = q.Cfg(512, 32, 2, 128)
+    off = np.zeros(32, np.float32)
+    off[7] = 8.0
+    dl = DevLayer(q, cfg, seed=12, layer=0, offset=off)
+    T = 40
+    x = dev_tokens(12, 0, T, 512)
+    out = torch.empty((T, 512), dtype=torch.float32, device="cuda")
+    idx = torch.empty((T, 2), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, 2), dtype=torch.float32, device="cuda")
+    ws = q.workspace(cfg, T)
+    q.moe_layer_step(cfg, dl.layer_struct, x, out, True, idx, w, ws)
+    assert q.qe_workspace_status(ws) == q.QE_OK
+    idx_h = idx.cpu().numpy()
+    assert (idx_h[:, 0] == 7).all()
+    out_h, w_h = out.cpu().numpy(), w.cpu().numpy()
+    for t in range(0, T, 3):
+        check(dl, out_h[t], idx_h[t], w_h[t], dl.oracle(host_x_f64(12, t, 512), residual=True))
+
+
+def test_batched_c4_full_step_sampled(q, c1_layer):
+    """The batched workload at full size: 256 bf16 tokens, top-4 of 512,
+    grouped experts; sampled tokens against the oracle."""
+    import torch
+    dl = c1_layer
+    T = 256
+    x = dev_tokens(0, 50000, T, 4096, bf16=True)
+    out = torch.empty((T, 4096), dtype=torch.float32, device="cuda")
+    idx = torch.empty((T, 4), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, 4), dtype=torch.float32, device="cuda")
+    ws = q.workspace(dl.cfg, T)
+    for _ in range(2):  # the second step reuses the workspace
+        q.moe_layer_step(dl.cfg, dl.layer_struct, x, out, False, idx, w, ws)
+    assert q.qe_workspace_status(ws) == q.QE_OK
+    out_h, idx_h, w_h = out.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy()
+    for t in (0, 100, 255):
+        check(dl, out_h[t], idx_h[t], w_h[t], dl.oracle(host_x_f64(0, 50000 + t, 4096, bf16=True)))
