@@ -213,6 +213,38 @@ QE_API int moe_layer_step(const qe_cfg* cfg, const qe_layer* layer, const void* 
                    float* out, int add_residual, int32_t* topk_idx, float* topk_w, void* dev_ws,
                    size_t ws_bytes, qe_stream_t stream);
 
+/* The single-token layer step of moe_layer_step (T == 1, fused kernel) for
+ * callers that cannot allocate device memory: a plugin whose host engine
+ * hands it only input and output buffers, or code running beside an
+ * allocator that has already reserved the GPU's memory for itself.  The
+ * paper has no counterpart of this call; it only changes where the scratch
+ * lives.
+ *
+ * Instead of a workspace it uses a fixed scratch array built into the
+ * library (139,520 bytes, 256-byte aligned), which every GPU that loads the
+ * library holds until the process exits.  It calls no allocation routine.
+ *   x       [1,H] device, fp32 or bf16 bits (x_dtype); out [1,H] fp32
+ *           device (must not alias x); topk_idx/topk_w [1,K] device outputs
+ *           or NULL, as in moe_layer_step.
+ *   dev_status  int32 device output or NULL: after the step it holds the
+ *           device-side status of this call (QE_OK, QE_ERR_TIMEOUT or
+ *           QE_ERR_INVALID_ARG), read by the caller after synchronising.
+ * Limits: top_k * inter <= 32768; hidden a multiple of 256 and <= 4096;
+ * n_experts <= 8 x the SM count.  Larger shapes are rejected with
+ * QE_ERR_INVALID_ARG (top_k * inter) or QE_ERR_UNSUPPORTED (the others)
+ * before anything is launched.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  Every call clears the array's
+ * control block on `stream` before its kernel, so a call that timed out
+ * needs no re-initialisation.  All calls on a device share the array and
+ * its contents outlive the call: two calls whose work overlaps on the GPU
+ * (other streams, other threads) race and give wrong results; order them
+ * on one stream or with events. */
+QE_API int moe_layer_step_noalloc(const qe_cfg* cfg, const qe_layer* layer, const void* x, int x_dtype,
+                                  float* out, int add_residual, int32_t* topk_idx, float* topk_w,
+                                  int32_t* dev_status, qe_stream_t stream);
+
 /* Test hook: make CTA `cta` of the next fused single-token launches skip its
  * arrival at the routing barrier (-1 disables).  The other CTAs' bounded
  * waits then give up and the workspace reports QE_ERR_TIMEOUT. */

@@ -28,7 +28,7 @@ __all__ = [
     "qe_last_error", "qe_version", "qe_expert_bytes", "qe_pool_table", "qe_workspace_bytes",
     "qe_workspace_init", "qe_workspace_status", "qe_set_wait_budget_ns", "qe_test_skip_arrival", "qe_trace_fused",
     "moe_route", "moe_expert_ffn_q4", "moe_expert_ffn_q2", "moe_expert_ffn_mixed", "moe_combine",
-    "moe_layer_step", "workspace",
+    "moe_layer_step", "moe_layer_step_noalloc", "workspace",
 ]
 
 
@@ -87,6 +87,7 @@ def _load():
         "moe_expert_ffn_mixed": (i32, [P(Cfg), vp, vp, vp, i32, vp, vp, sz, vp]),
         "moe_combine": (i32, [vp, vp, vp, i32, i32, i32, vp, vp]),
         "moe_layer_step": (i32, [P(Cfg), P(Layer), vp, i32, i32, vp, i32, vp, vp, vp, sz, vp]),
+        "moe_layer_step_noalloc": (i32, [P(Cfg), P(Layer), vp, i32, vp, i32, vp, vp, vp, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -225,6 +226,20 @@ def moe_layer_step(cfg, layer: Layer, x, out, add_residual=False, topk_idx=None,
     _check(lib.moe_layer_step(ctypes.byref(cfg), ctypes.byref(layer), _ptr(x), dt, T, _ptr(out),
                               1 if add_residual else 0, _ptr(topk_idx), _ptr(topk_w), _ptr(ws), _nbytes(ws),
                               _stream(stream)))
+
+
+def moe_layer_step_noalloc(cfg, layer: Layer, x, out, add_residual=False, topk_idx=None, topk_w=None,
+                           status=None, stream=None):
+    """One token through the layer with the library's built-in scratch
+    (no workspace, no allocation); `status` is an optional int32 device
+    tensor that receives the call's device-side status."""
+    import torch
+    if x.shape[0] != 1:
+        raise ValueError("moe_layer_step_noalloc takes exactly one token")
+    dt = QE_BF16 if x.dtype == torch.bfloat16 else QE_F32
+    _check(lib.moe_layer_step_noalloc(ctypes.byref(cfg), ctypes.byref(layer), _ptr(x), dt, _ptr(out),
+                                      1 if add_residual else 0, _ptr(topk_idx), _ptr(topk_w), _ptr(status),
+                                      _stream(stream)))
 
 
 class ExpertPool:

@@ -344,3 +344,99 @@ int moe_layer_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Single-token layer step whose scratch lives in the library itself.
+//
+// The fused single-token kernel needs three pieces of device scratch besides
+// its inputs and outputs: the control block (grid counters, error word, per
+// expert |h| maxima), the E router logits and the K x I SwiGLU activations.
+// moe_layer_step takes them from a caller-allocated workspace; the entry
+// point below takes them from a fixed array that every GPU loading this
+// library holds until the process exits.
+namespace qe {
+
+constexpr size_t kStaticLogitsOff = sizeof(WsControl);              // 256
+constexpr size_t kStaticHOff = kStaticLogitsOff + 8 * (size_t)kMaxE;  // 8 KiB of fp64 logits
+constexpr size_t kStaticMaxKI = 32768;                               // top_k * inter
+constexpr size_t kStaticBytes = kStaticHOff + 4 * kStaticMaxKI;       // 139,520 bytes
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticBytes];
+
+// Device address of g_static_scratch on the current device.  In host code the
+// name g_static_scratch only stands for the symbol, so the address is asked
+// of the runtime once per device (with that device current) and cached.
+static int static_scratch(unsigned char** out) {
+  static std::mutex mu;
+  static unsigned char* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(QE_ERR_UNSUPPORTED, "moe_layer_step_noalloc: device %d >= 64", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step_noalloc: cudaGetSymbolAddress");
+    if (!p || ((uintptr_t)p & 255) != 0)
+      return fail(QE_ERR_CUDA, "moe_layer_step_noalloc: scratch address %p is not 256-byte aligned", p);
+    addr[dev] = (unsigned char*)p;
+  }
+  *out = addr[dev];
+  return QE_OK;
+}
+
+}  // namespace qe
+
+extern "C" int moe_layer_step_noalloc(const qe_cfg* c, const qe_layer* layer, const void* x, int x_dtype,
+                                      float* out, int add_residual, int32_t* topk_idx, float* topk_w,
+                                      int32_t* dev_status, qe_stream_t stream) {
+  int rc = check_cfg(c);
+  if (rc) return rc;
+  if (!layer) return fail(QE_ERR_INVALID_ARG, "layer is NULL");
+  if (!(x_dtype == QE_F32 || x_dtype == QE_BF16)) return fail(QE_ERR_INVALID_ARG, "x_dtype must be QE_F32 or QE_BF16");
+  if ((size_t)c->top_k * (size_t)c->inter > kStaticMaxKI)
+    return fail(QE_ERR_INVALID_ARG,
+                "moe_layer_step_noalloc: top_k * inter = %d exceeds the built-in scratch limit of %zu "
+                "(use moe_layer_step with a workspace)",
+                c->top_k * c->inter, kStaticMaxKI);
+  if ((rc = check_ptr(x, "x", false, x_dtype == QE_BF16 ? 2 : 4)) || (rc = check_ptr(out, "out")) ||
+      (rc = check_ptr(layer->router_w, "router_w", false, 16)) || (rc = check_ptr(layer->experts, "experts", false, 8)) ||
+      (rc = check_ptr(layer->gamma, "gamma", true)) || (rc = check_ptr(layer->logit_offset, "logit_offset", true)) ||
+      (rc = check_ptr(topk_idx, "topk_idx", true)) || (rc = check_ptr(topk_w, "topk_w", true)) ||
+      (rc = check_ptr(dev_status, "dev_status", true)))
+    return rc;
+  if ((const void*)out == x) return fail(QE_ERR_INVALID_ARG, "out must not alias x");
+  FusedParams p{};
+  const DevInfo d = dev_info();
+  if (fused_geometry(c->hidden, c->n_experts, c->top_k, c->inter, d.sms, d.optin, &p.g) != QE_OK)
+    return fail(QE_ERR_UNSUPPORTED,
+                "moe_layer_step_noalloc: shape not supported by the single-token kernel (hidden %d must be a "
+                "multiple of 256 and <= 4096; n_experts %d must be <= 8 x SMs)",
+                c->hidden, c->n_experts);
+  unsigned char* scratch = nullptr;
+  if ((rc = static_scratch(&scratch))) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  WsControl* ctl = (WsControl*)scratch;
+  // the previous call (possibly one that timed out) left its counters and
+  // error word here: the kernel expects them at zero
+  cudaError_t e = cudaMemsetAsync(ctl, 0, sizeof(WsControl), s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step_noalloc: clear control block");
+  p.H = c->hidden; p.E = c->n_experts; p.K = c->top_k; p.I = c->inter; p.eps = c->eps;
+  p.x = x; p.x_bf16 = x_dtype == QE_BF16; p.add_residual = add_residual != 0;
+  p.gamma = layer->gamma; p.router_w = layer->router_w; p.offset = layer->logit_offset;
+  p.experts = layer->experts; p.out = out; p.topk_idx = topk_idx; p.topk_w = topk_w;
+  p.ctl = ctl;
+  p.logit_part = (double*)(scratch + kStaticLogitsOff);
+  p.hbuf = (float*)(scratch + kStaticHOff);
+  p.budget_ns = g_budget_ns;
+  p.skip_cta = g_skip_cta;
+  p.trace = g_trace;
+  e = launch_fused_layer(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step_noalloc launch");
+  if (dev_status) {
+    e = cudaMemcpyAsync(dev_status, &ctl->err, sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step_noalloc: copy status");
+  }
+  return QE_OK;
+}
