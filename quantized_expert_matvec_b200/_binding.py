@@ -28,7 +28,7 @@ __all__ = [
     "qe_last_error", "qe_version", "qe_expert_bytes", "qe_pool_table", "qe_workspace_bytes",
     "qe_workspace_init", "qe_workspace_status", "qe_set_wait_budget_ns", "qe_test_skip_arrival", "qe_trace_fused",
     "moe_route", "moe_expert_ffn_q4", "moe_expert_ffn_q2", "moe_expert_ffn_mixed", "moe_combine",
-    "moe_layer_step", "moe_layer_step_noalloc", "workspace",
+    "moe_layer_step", "moe_layer_step_noalloc", "workspace", "Tier", "TierDesc",
 ]
 
 
@@ -60,6 +60,15 @@ class Layer(ctypes.Structure):
                 ("experts", ctypes.c_void_p)]
 
 
+class TierDesc(ctypes.Structure):
+    _fields_ = [("cfg", Cfg), ("n_layers", ctypes.c_int32), ("cold_bits", ctypes.c_int32),
+                ("max_tokens", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("cold_host", ctypes.POINTER(ctypes.c_void_p)), ("cache_bytes", ctypes.c_size_t)]
+
+
+assert ctypes.sizeof(TierDesc) == 56
+
+
 assert ctypes.sizeof(Expert) == 96
 
 
@@ -88,6 +97,12 @@ def _load():
         "moe_combine": (i32, [vp, vp, vp, i32, i32, i32, vp, vp]),
         "moe_layer_step": (i32, [P(Cfg), P(Layer), vp, i32, i32, vp, i32, vp, vp, vp, sz, vp]),
         "moe_layer_step_noalloc": (i32, [P(Cfg), P(Layer), vp, i32, vp, i32, vp, vp, vp, vp]),
+        "qe_tier_create": (i32, [P(TierDesc), P(vp)]),
+        "qe_tier_resolve": (i32, [vp, i32, P(ctypes.c_int32), i32, vp, vp]),
+        "qe_tier_layer_step": (i32, [vp, i32, P(Layer), vp, i32, i32, vp, i32, vp, vp, vp, sz, vp]),
+        "qe_tier_stats": (i32, [vp, P(ctypes.c_uint64), P(ctypes.c_uint64), P(ctypes.c_uint64)]),
+        "qe_tier_slots": (i32, [vp]),
+        "qe_tier_destroy": (None, [vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -240,6 +255,62 @@ def moe_layer_step_noalloc(cfg, layer: Layer, x, out, add_residual=False, topk_i
     _check(lib.moe_layer_step_noalloc(ctypes.byref(cfg), ctypes.byref(layer), _ptr(x), dt, _ptr(out),
                                       1 if add_residual else 0, _ptr(topk_idx), _ptr(topk_w), _ptr(status),
                                       _stream(stream)))
+
+
+class Tier:
+    """A two-tier expert store (qe_tier_*): cold_host[l][e] is the host
+    address of cold expert (l, e) in the standard pool layout at cold_bits,
+    or None for a hot expert.  Owns the native tier until close()."""
+
+    def __init__(self, cfg: Cfg, cold_host, cold_bits: int, cache_bytes: int, max_tokens: int = 1):
+        L = len(cold_host)
+        E = cfg.n_experts
+        arr = (ctypes.c_void_p * (L * E))()
+        for l in range(L):
+            for e in range(E):
+                arr[l * E + e] = cold_host[l][e]
+        self._arr = arr
+        d = TierDesc(cfg, L, cold_bits, max_tokens, 0, ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)),
+                     int(cache_bytes))
+        h = ctypes.c_void_p()
+        _check(lib.qe_tier_create(ctypes.byref(d), ctypes.byref(h)))
+        self.handle = h
+        self.cfg = cfg
+
+    @property
+    def slots(self) -> int:
+        return lib.qe_tier_slots(self.handle)
+
+    def stats(self):
+        """(hits, misses, h2d_bytes) since creation."""
+        a, b, c = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
+        _check(lib.qe_tier_stats(self.handle, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+        return a.value, b.value, c.value
+
+    def resolve(self, layer: int, idx, dev_table, stream=None):
+        idx = [int(i) for i in idx]
+        arr = (ctypes.c_int32 * len(idx))(*idx)
+        _check(lib.qe_tier_resolve(self.handle, layer, arr, len(idx), _ptr(dev_table), _stream(stream)))
+
+    def layer_step(self, layer: int, layer_w: Layer, x, out, add_residual=False, topk_idx=None, topk_w=None,
+                   ws=None, stream=None):
+        import torch
+        T = x.shape[0]
+        dt = QE_BF16 if x.dtype == torch.bfloat16 else QE_F32
+        _check(lib.qe_tier_layer_step(self.handle, layer, ctypes.byref(layer_w), _ptr(x), dt, T, _ptr(out),
+                                      1 if add_residual else 0, _ptr(topk_idx), _ptr(topk_w), _ptr(ws),
+                                      _nbytes(ws), _stream(stream)))
+
+    def close(self):
+        if self.handle:
+            lib.qe_tier_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class ExpertPool:

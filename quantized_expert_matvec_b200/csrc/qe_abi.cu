@@ -15,7 +15,7 @@ static unsigned long long g_budget_ns = 200ull * 1000 * 1000;
 static int g_skip_cta = -1;
 static unsigned long long* g_trace = nullptr;
 
-static int fail(int code, const char* fmt, ...) {
+int fail(int code, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
   vsnprintf(g_err, sizeof(g_err), fmt, ap);
@@ -23,11 +23,24 @@ static int fail(int code, const char* fmt, ...) {
   return code;
 }
 
-static int cuda_fail(cudaError_t e, const char* what) {
+int cuda_fail(cudaError_t e, const char* what) {
   return fail(QE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
 static size_t al(size_t v) { return (v + 255) & ~(size_t)255; }
+
+qe_expert pool_descriptor(const qe_cfg* c, void* base, int bits) {
+  const size_t H = c->hidden, I = c->inter;
+  const size_t wq = al(I * H * bits / 8), sb = al(I * H / kGroup * 2);
+  char* b = (char*)base;
+  qe_expert x{};
+  x.gate = {(const uint32_t*)b, (const uint16_t*)(b + 3 * wq), (const uint16_t*)(b + 3 * wq + sb), bits, 0};
+  x.up = {(const uint32_t*)(b + wq), (const uint16_t*)(b + 3 * wq + 2 * sb), (const uint16_t*)(b + 3 * wq + 3 * sb),
+          bits, 0};
+  x.down = {(const uint32_t*)(b + 2 * wq), (const uint16_t*)(b + 3 * wq + 4 * sb),
+            (const uint16_t*)(b + 3 * wq + 5 * sb), bits, 0};
+  return x;
+}
 
 WsLayout ws_layout(int H, int E, int K, int I, int T) {
   WsLayout L{};
@@ -60,7 +73,7 @@ WsLayout ws_layout(int H, int E, int K, int I, int T) {
   return L;
 }
 
-static int check_cfg(const qe_cfg* c) {
+int check_cfg(const qe_cfg* c) {
   if (!c) return fail(QE_ERR_INVALID_ARG, "cfg is NULL");
   if (c->group != kGroup) return fail(QE_ERR_INVALID_ARG, "group must be 64 (got %d)", c->group);
   if (c->hidden <= 0 || c->hidden % kGroup || c->hidden > kMaxDim)
@@ -77,13 +90,13 @@ static int check_cfg(const qe_cfg* c) {
 
 // Pointers must be aligned to `align` bytes: their element size, or 16 where
 // the kernels read them with 128-bit loads (router rows).
-static int check_ptr(const void* p, const char* name, bool may_be_null = false, unsigned align = 4) {
+int check_ptr(const void* p, const char* name, bool may_be_null, unsigned align) {
   if (!p) return may_be_null ? QE_OK : fail(QE_ERR_INVALID_ARG, "%s is NULL", name);
   if (((uintptr_t)p & (align - 1)) != 0) return fail(QE_ERR_INVALID_ARG, "%s is not %u-byte aligned", name, align);
   return QE_OK;
 }
 
-static int check_ws(const qe_cfg* c, int T, void* ws, size_t bytes) {
+int check_ws(const qe_cfg* c, int T, void* ws, size_t bytes) {
   if (!ws) return fail(QE_ERR_INVALID_ARG, "workspace is NULL");
   if (((uintptr_t)ws & 255) != 0) return fail(QE_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   const size_t need = ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, T).total;
@@ -94,11 +107,7 @@ static int check_ws(const qe_cfg* c, int T, void* ws, size_t bytes) {
 template <typename P>
 static P* at(void* base, size_t off) { return (P*)((char*)base + off); }
 
-struct DevInfo {
-  int sms = 0, optin = 0;
-};
-
-static DevInfo dev_info() {
+DevInfo dev_info() {
   static std::mutex mu;
   static DevInfo cache[64];
   int dev = 0;
@@ -112,7 +121,7 @@ static DevInfo dev_info() {
   return d;
 }
 
-static int route_impl(const qe_cfg* c, const void* x, int x_dtype, const float* gamma, const float* router_w,
+int route_impl(const qe_cfg* c, const void* x, int x_dtype, const float* gamma, const float* router_w,
                       const float* offset, int T, float* xn, int32_t* idx, float* w, void* ws, size_t ws_bytes,
                       bool want_xprime, cudaStream_t s) {
   const WsLayout L = ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, T);
@@ -177,14 +186,7 @@ int qe_pool_table(const qe_cfg* c, void* base, int bits, int n, qe_expert* out, 
                           3 * wq + 4 * sb, 3 * wq + 5 * sb};
   if (seg) memcpy(seg, offs, sizeof(offs));
   const size_t stride = 3 * wq + 6 * sb;
-  for (int e = 0; e < n; ++e) {
-    char* b = (char*)base + (size_t)e * stride;
-    qe_expert x{};
-    x.gate = {(const uint32_t*)(b + offs[0]), (const uint16_t*)(b + offs[3]), (const uint16_t*)(b + offs[4]), bits, 0};
-    x.up = {(const uint32_t*)(b + offs[1]), (const uint16_t*)(b + offs[5]), (const uint16_t*)(b + offs[6]), bits, 0};
-    x.down = {(const uint32_t*)(b + offs[2]), (const uint16_t*)(b + offs[7]), (const uint16_t*)(b + offs[8]), bits, 0};
-    out[e] = x;
-  }
+  for (int e = 0; e < n; ++e) out[e] = pool_descriptor(c, (char*)base + (size_t)e * stride, bits);
   return QE_OK;
 }
 
@@ -324,10 +326,22 @@ int moe_layer_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_
   rc = route_impl(c, x, x_dtype, layer->gamma, layer->router_w, layer->logit_offset, T, nullptr, idx, w, ws, ws_bytes,
                   true, s);
   if (rc) return rc;
+  return experts_and_combine(c, layer->experts, idx, w, x, x_dtype, T, out, add_residual, ws, s);
+}
+
+}  // extern "C"
+
+namespace qe {
+
+// Expert FFNs of routed tokens (x' already prepared by route_impl with
+// want_xprime), then the weighted combine: the batched half of the layer step.
+int experts_and_combine(const qe_cfg* c, const qe_expert* experts, const int32_t* idx, const float* w, const void* x,
+                        int x_dtype, int T, float* out, int add_residual, void* ws, cudaStream_t s) {
+  const WsLayout L = ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, T);
   {
     GroupedParams gp{};
     gp.H = c->hidden; gp.E = c->n_experts; gp.K = c->top_k; gp.I = c->inter; gp.T = T;
-    gp.experts = layer->experts; gp.idx = idx; gp.w = w;
+    gp.experts = experts; gp.idx = idx; gp.w = w;
     gp.xp4 = at<float>(ws, L.xp4); gp.xp2 = at<float>(ws, L.xp2); gp.xsum = at<float>(ws, L.xsum);
     gp.xexp = at<int>(ws, L.xexp);
     gp.y = at<float>(ws, L.y);
@@ -343,7 +357,7 @@ int moe_layer_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_
   return QE_OK;
 }
 
-}  // extern "C"
+}  // namespace qe
 
 // ---------------------------------------------------------------------------
 // Single-token layer step whose scratch lives in the library itself.

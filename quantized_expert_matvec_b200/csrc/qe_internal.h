@@ -167,4 +167,22 @@ struct GroupedParams {
 cudaError_t launch_grouped(const GroupedParams& p, cudaStream_t s);
 int grouped_tile(int H, int I, int smem_optin);
 
+
+// ---- shared host helpers (qe_abi.cu)
+struct DevInfo {
+  int sms = 0, optin = 0;
+};
+DevInfo dev_info();
+int fail(int code, const char* fmt, ...);
+int cuda_fail(cudaError_t e, const char* what);
+int check_cfg(const qe_cfg* c);
+int check_ptr(const void* p, const char* name, bool may_be_null = false, unsigned align = 4);
+int check_ws(const qe_cfg* c, int T, void* ws, size_t bytes);
+qe_expert pool_descriptor(const qe_cfg* c, void* base, int bits);
+int route_impl(const qe_cfg* c, const void* x, int x_dtype, const float* gamma, const float* router_w,
+               const float* offset, int T, float* xn, int32_t* idx, float* w, void* ws, size_t ws_bytes,
+               bool want_xprime, cudaStream_t s);
+int experts_and_combine(const qe_cfg* c, const qe_expert* experts, const int32_t* idx, const float* w, const void* x,
+                        int x_dtype, int T, float* out, int add_residual, void* ws, cudaStream_t s);
+
 }  // namespace qe

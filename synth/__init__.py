@@ -127,6 +127,16 @@ def host_fill(n: int, kind: int, seed: int, a: int, b: int, tensor: int,
     return out
 
 
+def host_fill_into(dst_ptr: int, n: int, kind: int, seed: int, a: int, b: int, tensor: int,
+                   p0: float = 0.0, p1: float = 0.0, i0: int = 0) -> None:
+    """Write elements [i0, i0+n) of stream (seed, a, b, tensor) to host memory
+    at dst_ptr (for pinned buffers that numpy does not own)."""
+    rc = _host_lib().sy_host_fill(ctypes.c_void_p(dst_ptr), int(i0), int(n), int(kind), int(seed),
+                                  int(a), int(b), int(tensor), float(p0), float(p1))
+    if rc != 0:
+        raise RuntimeError(f"sy_host_fill failed ({rc})")
+
+
 def dev_fill_family(base_ptr: int, stride_bytes: int, n_per: int, n_members: int, kind: int,
                     seed: int, a: int, b0: int, tensor: int, p0: float = 0.0, p1: float = 0.0,
                     stream: int = 0) -> None:

@@ -91,3 +91,22 @@ def test_empty_batches_are_noops(q):
     assert q.lib.moe_layer_step(ctypes.byref(c), ctypes.byref(layer), 4096, 0, 0, 8192, 0, None, None, None, 0,
                                 None) == q.QE_OK
     assert q.lib.moe_combine(None, None, None, 0, 2, 64, None, None) == q.QE_OK
+
+
+def test_tier_arguments_checked_before_any_cuda_call(q):
+    lib = q.lib
+    h = ctypes.c_void_p()
+    assert lib.qe_tier_create(None, ctypes.byref(h)) == q.QE_ERR_INVALID_ARG
+    cfg = q.Cfg(256, 16, 2, 64)
+    arr = (ctypes.c_void_p * 16)()
+    ptr = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    for bits, layers, toks, cache, msg in [(3, 1, 1, 1 << 20, "cold_bits"), (2, 0, 1, 1 << 20, "n_layers"),
+                                           (2, 1, 0, 1 << 20, "max_tokens"), (2, 1, 1, 100, "cache_bytes")]:
+        d = q.TierDesc(cfg, layers, bits, toks, 0, ptr, cache)
+        assert lib.qe_tier_create(ctypes.byref(d), ctypes.byref(h)) == q.QE_ERR_INVALID_ARG
+        assert msg in q.qe_last_error()
+        assert not h.value
+    assert lib.qe_tier_slots(None) == 0
+    assert lib.qe_tier_stats(None, None, None, None) == q.QE_ERR_INVALID_ARG
+    assert lib.qe_tier_resolve(None, 0, None, 0, None, None) == q.QE_ERR_INVALID_ARG
+    lib.qe_tier_destroy(None)
