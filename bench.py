@@ -42,6 +42,16 @@ WORKLOADS = {
     "c0": dict(H=256, E=16, K=2, I=64, bits=4, T=1,
                name="tiny MoE FFN: hidden 256, 16 experts, top-2, intermediate 64, 4-bit g64, 1 token",
                metric="MoE-layer decode tokens/s at 1 B200 (tiny layer)"),
+    "c2": dict(H=4096, E=512, K=4, I=1024, bits=4, T=1, layers=40, zipf=True,
+               name="40-layer stack of the one-layer workload (no attention), 145 GB of 4-bit experts in HBM, "
+                    "sequential decode tokens with residual add between layers, Zipf(1.1) popularity logit "
+                    "offset per layer (alpha 0.40: about 70% of selections in the hottest 25%)",
+               metric="40-layer MoE stack decode tokens/s at 1 B200"),
+    "c3": dict(H=4096, E=512, K=4, I=1024, bits=4, T=1, layers=60, zipf=True, hot=128, cache_gb=24.0,
+               name="60 tiered layers of the one-layer shape: per layer the 128 most popular experts 4-bit in "
+                    "HBM, the other 384 2-bit in pinned host memory behind a 24 GB HBM LRU expert cache "
+                    "(async H2D on a side stream), Zipf routing, sequential decode tokens with residual",
+               metric="60-layer tiered MoE decode tokens/s at 1 B200"),
     "c4": dict(H=4096, E=512, K=4, I=1024, bits=4, T=256,
                name="batched decode of the one-layer workload: 256 bf16 tokens per step, own top-4 of 512 each, "
                     "grouped per expert, 4-bit g64 experts in HBM, uniform routing",
@@ -139,165 +149,145 @@ class ClockSampler:
 # oracle timing (the CPU baseline and the reference arm)
 # --------------------------------------------------------------------------
 
-def oracle_token_time(wl, seed, tokens, row_fraction=1.0, nthreads=None):
-    """Time the fp64 oracle on whole tokens of the workload's layer: routing
-    in full, expert matvecs on a leading fraction of the rows (extrapolated).
-    Expert weights are regenerated before the timed calls.  Returns (seconds
-    per token, threads, seconds measured)."""
-    import oracle
+def wl_layers(wl):
+    return wl.get("layers", 1)
+
+
+def wl_bits_of(wl, seed, layer):
+    """Bits of each expert of a layer: the tiered workload keeps its hot set
+    (most popular ranks) at 4 bits and the rest at 2."""
     import synth
-    H, E, K, I, bits = wl["H"], wl["E"], wl["K"], wl["I"], wl["bits"]
-    bf16 = wl["T"] > 1
-    nthreads = nthreads or os.cpu_count() or 1
-    W = synth.host_router(seed, 0, E, H)
-
-    def tok(t):
-        x = synth.host_tokens(seed, t, 1, H, bf16=bf16)[0]
-        if bf16:
-            return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-        return x.astype(np.float64)
-
-    xs = [tok(t) for t in tokens]
-    cache = {}
-    for x in xs:
-        idx, _ = oracle.topk(oracle.router(W, oracle.rmsnorm(x, None, EPS32), None, nthreads), K)
-        for e in idx:
-            if int(e) not in cache:
-                cache[int(e)] = synth.host_expert(seed, 0, int(e), H, I, bits)
-    nr_i = max(1, int(round(I * row_fraction)))
-    nr_h = max(1, int(round(H * row_fraction)))
-    t_route = 0.0
-    t_exp = 0.0
-    for x in xs:
-        t0 = time.perf_counter()
-        xn = oracle.rmsnorm(x, None, EPS32)
-        lg = oracle.router(W, xn, None, nthreads)
-        idx, w = oracle.topk(lg, K)
-        t1 = time.perf_counter()
-        ys = []
-        for e in idx:
-            ex = cache[int(e)]
-            g = oracle.qmatvec(ex["gate_wq"][:nr_i], ex["gate_s"][:nr_i], ex["gate_b"][:nr_i], bits, xn, nthreads)
-            u = oracle.qmatvec(ex["up_wq"][:nr_i], ex["up_s"][:nr_i], ex["up_b"][:nr_i], bits, xn, nthreads)
-            h = np.zeros(I)
-            h[:nr_i] = oracle.swiglu(g, u)
-            ys.append(oracle.qmatvec(ex["down_wq"][:nr_h], ex["down_s"][:nr_h], ex["down_b"][:nr_h], bits, h,
-                                     nthreads))
-        yfull = np.zeros((K, H))
-        for k in range(K):
-            yfull[k, :nr_h] = ys[k]
-        oracle.combine(yfull, w, x)
-        t2 = time.perf_counter()
-        t_route += t1 - t0
-        t_exp += t2 - t1
-    n = len(xs)
-    per_token = t_route / n + (t_exp / n) / (nr_h / H if row_fraction < 1.0 else 1.0)
-    return per_token, nthreads, t_route + t_exp
+    if wl.get("hot"):
+        hot = synth.hot_set(seed, layer, wl["E"], wl["hot"])
+        return lambda e: 4 if hot[e] else 2
+    return lambda e: wl["bits"]
 
 
-def cpu_baseline(wl, seed, budget_s=15.0):
-    """The oracle on a bounded sample of the workload (whole tokens)."""
-    per1, nth, _ = oracle_token_time(wl, seed, [1_000_000])
-    n = max(1, min(64, int(budget_s / max(per1, 1e-9))))
-    per, nth, spent = oracle_token_time(wl, seed, list(range(1_000_001, 1_000_001 + n)))
-    return {"value": 1.0 / per, "unit": UNIT, "cores": nth, "kind": "oracle",
-            "sample": f"{n} whole tokens of the workload (fp64 oracle, OpenMP over rows, {nth} threads), "
-                      f"{spent:.1f} s of CPU time"}
+def wl_offset(wl, seed, layer):
+    import synth
+    return synth.zipf_logit_offset(seed, layer, wl["E"]) if wl.get("zipf") else None
 
 
 class OracleSample:
-    """The oracle on a fixed pool of distinct tokens of the workload: routing
-    in full every time, expert matvecs on a leading fraction of the rows
-    (their time extrapolated to the full rows).  Experts are generated once,
-    outside the timed calls, and kept cut to the sampled rows."""
+    """The oracle on a pool of (layer, token) layer steps of the workload:
+    routing in full every time, expert matvecs on a leading fraction of the
+    rows (their time extrapolated to the full rows).  Experts are generated
+    once, outside the timed calls, and kept cut to the sampled rows."""
 
-    def __init__(self, wl, seed, frac, n_pool=32, nthreads=None):
+    def __init__(self, wl, seed, frac, n_pool=32, nthreads=None, max_layers=8):
         import oracle
         import synth
         self.oracle = oracle
-        H, E, K, I, bits = wl["H"], wl["E"], wl["K"], wl["I"], wl["bits"]
-        self.K, self.bits, self.H, self.I = K, bits, H, I
+        H, E, K, I = wl["H"], wl["E"], wl["K"], wl["I"]
+        self.K, self.H, self.I = K, H, I
         self.nthreads = nthreads or os.cpu_count() or 1
         self.frac = frac
         self.nr_i = max(1, int(round(I * frac)))
         self.nr_h = max(1, int(round(H * frac)))
-        self.W = synth.host_router(seed, 0, E, H)
+        self.residual = wl_layers(wl) > 1
+        nl = min(wl_layers(wl), max_layers)
+        self.W = [synth.host_router(seed, l, E, H) for l in range(nl)]
+        self.off = [wl_offset(wl, seed, l) for l in range(nl)]
+        self.bits = [wl_bits_of(wl, seed, l) for l in range(nl)]
         bf16 = wl["T"] > 1
-        self.xs = []
+        self.pool = []
         self.experts = {}
-        for t in range(n_pool):
-            x = synth.host_tokens(seed, 4_000_000 + t, 1, H, bf16=bf16)[0]
+        for j in range(n_pool):
+            l = j % nl
+            x = synth.host_tokens(seed, 4_000_000 + j, 1, H, bf16=bf16)[0]
             x = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64) if bf16 else x.astype(np.float64)
-            self.xs.append(x)
-            idx, _ = oracle.topk(oracle.router(self.W, oracle.rmsnorm(x, None, EPS32), None, self.nthreads), K)
+            self.pool.append((l, x))
+            idx, _ = oracle.topk(oracle.router(self.W[l], oracle.rmsnorm(x, None, EPS32), self.off[l],
+                                               self.nthreads), K)
             for e in idx:
                 e = int(e)
-                if e not in self.experts:
-                    ex = synth.host_expert(seed, 0, e, H, I, bits)
-                    cut = {}
+                if (l, e) not in self.experts:
+                    b = self.bits[l](e)
+                    ex = synth.host_expert(seed, l, e, H, I, b)
+                    cut = {"bits": b}
                     for m, nr in (("gate", self.nr_i), ("up", self.nr_i), ("down", self.nr_h)):
                         for f in ("wq", "s", "b"):
                             cut[f"{m}_{f}"] = np.ascontiguousarray(ex[f"{m}_{f}"][:nr])
-                    self.experts[e] = cut
+                    self.experts[(l, e)] = cut
 
-    def token_seconds(self, t):
-        """Oracle time of pool token t, extrapolated to the full rows."""
-        o, nth, bits = self.oracle, self.nthreads, self.bits
-        x = self.xs[t % len(self.xs)]
+    def step_seconds(self, j):
+        """Oracle time of pool layer step j, extrapolated to the full rows."""
+        o, nth = self.oracle, self.nthreads
+        l, x = self.pool[j % len(self.pool)]
         t0 = time.perf_counter()
         xn = o.rmsnorm(x, None, EPS32)
-        idx, w = o.topk(o.router(self.W, xn, None, nth), self.K)
+        idx, w = o.topk(o.router(self.W[l], xn, self.off[l], nth), self.K)
         t1 = time.perf_counter()
         yfull = np.zeros((self.K, self.H))
         for k, e in enumerate(idx):
-            ex = self.experts[int(e)]
-            g = o.qmatvec(ex["gate_wq"], ex["gate_s"], ex["gate_b"], bits, xn, nth)
-            u = o.qmatvec(ex["up_wq"], ex["up_s"], ex["up_b"], bits, xn, nth)
+            ex = self.experts[(l, int(e))]
+            b = ex["bits"]
+            g = o.qmatvec(ex["gate_wq"], ex["gate_s"], ex["gate_b"], b, xn, nth)
+            u = o.qmatvec(ex["up_wq"], ex["up_s"], ex["up_b"], b, xn, nth)
             h = np.zeros(self.I)
             h[: self.nr_i] = o.swiglu(g, u)
-            yfull[k, : self.nr_h] = o.qmatvec(ex["down_wq"], ex["down_s"], ex["down_b"], bits, h, nth)
-        o.combine(yfull, w, x)
+            yfull[k, : self.nr_h] = o.qmatvec(ex["down_wq"], ex["down_s"], ex["down_b"], b, h, nth)
+        o.combine(yfull, w, x if self.residual else None)
         t2 = time.perf_counter()
         return (t1 - t0) + (t2 - t1) / self.frac
 
 
+def cpu_baseline(wl, seed, budget_s=15.0):
+    """The oracle on a bounded sample of the workload: whole layer steps
+    (routing and all expert rows), scaled to tokens."""
+    probe = OracleSample(wl, seed, 1.0, n_pool=1)
+    per1 = probe.step_seconds(0)
+    n = max(2, min(48, int(budget_s / max(per1, 1e-9))))
+    smp = OracleSample(wl, seed, 1.0, n_pool=n)
+    t0 = time.perf_counter()
+    tot = sum(smp.step_seconds(j) for j in range(n))
+    spent = time.perf_counter() - t0
+    per_token = tot / n * wl_layers(wl)
+    return {"value": 1.0 / per_token, "unit": UNIT, "cores": smp.nthreads, "kind": "oracle",
+            "sample": f"{n} whole layer steps (routing and all expert rows, fp64 oracle, OpenMP over rows, "
+                      f"{smp.nthreads} threads) of {min(wl_layers(wl), 8)} layer(s), scaled to "
+                      f"{wl_layers(wl)} layer(s) per token; {spent:.1f} s of CPU time"}
+
+
 def run_reference(args, wl, rank, world):
     """The reference arm: the fp64 oracle as it stands, on the host cores.
-    Each step is one token (T tokens for a batched workload, of which at
-    most 4 are timed and the rest extrapolated), on a bounded sample sized so
-    that all warm-up and timed steps take about 150 s."""
+    A step is the workload's step (one token through every layer, or T
+    tokens through one layer); at most 4 of its layer steps are timed and the
+    rest extrapolated, on a bounded sample sized so that all warm-up and
+    timed steps take about 150 s."""
     if rank != 0:
         return
     K, W, T = args.steps, args.warmup, wl["T"]
+    per_step_units = T * wl_layers(wl)   # layer steps in one step
     probe = OracleSample(wl, args.seed, 1.0, n_pool=1)
-    per_full = min(probe.token_seconds(0) for _ in range(2))
-    t_timed = min(T, 4)
+    per_full = min(probe.step_seconds(0) for _ in range(2))
+    t_timed = min(per_step_units, 4)
     frac = min(1.0, max(1.0 / 512, (150.0 / (K + W)) / max(per_full * t_timed, 1e-9)))
     smp = OracleSample(wl, args.seed, frac)
     i = 0
     for _ in range(W):
         for _ in range(t_timed):
-            smp.token_seconds(i)
+            smp.step_seconds(i)
             i += 1
     t0 = time.perf_counter()
     total = 0.0
     for _ in range(K):
         st = 0.0
         for _ in range(t_timed):
-            st += smp.token_seconds(i)
+            st += smp.step_seconds(i)
             i += 1
-        total += st * (T / t_timed)
+        total += st * (per_step_units / t_timed)
     wall = time.perf_counter() - t0
     value = K * T / total
     line = {"metric": wl["metric"], "value": value, "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": W,
             "ms_per_step": 1000.0 * total / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": wl["name"], "tokens_per_step": T,
+            "config": {"workload": wl["name"], "tokens_per_step": T, "layers": wl_layers(wl),
                        "tokens": "a pool of 32 distinct seeded N(0,1) tokens, cycled"},
             "cpu_baseline": {"kind": "oracle", "cores": smp.nthreads, "value": value, "unit": UNIT,
-                             "sample": f"each step: {t_timed} of its {T} token(s) timed, routing in full, expert "
-                                       f"rows sampled at fraction {frac:.4f} and extrapolated; "
-                                       f"{wall:.1f} s wall for the timed steps"},
+                             "sample": f"each step: {t_timed} of its {per_step_units} layer step(s) timed, "
+                                       f"routing in full, expert rows sampled at fraction {frac:.4f} and "
+                                       f"extrapolated; {wall:.1f} s wall for the timed steps"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -475,6 +465,350 @@ def run_ours(args, wl, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def sync_max(world, dev, value):
+    """Max of a float over ranks (the slowest rank's time)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def finish_line(args, wl, world, ms_max, ms, n_units, alg_bytes_per_step, exp_bytes_per_step, distinct, extra,
+                e2e, clocks, launches, kernel, duration_note):
+    peaks, peak_kind = measured_peaks()
+    per_step_s = (ms / 1000.0) / args.steps
+    peak = float(peaks["hbm_gbs"])
+    achieved = alg_bytes_per_step / per_step_s / 1e9
+    cpu = None if args.no_cpu_baseline else cpu_baseline(wl, args.seed)
+    line = {
+        "metric": wl["metric"], "value": world * n_units / (ms_max / 1000.0), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl["name"], "parallelism": "replicas" if world > 1 else "single GPU", **extra},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": load_traffic(args.workload), "peak_source": peak_kind, "kernel": kernel,
+                     "algorithmic_bytes_per_launch": alg_bytes_per_step, "duration": duration_note},
+        "expert_gbs": exp_bytes_per_step / per_step_s / 1e9,
+        "expert_frac": exp_bytes_per_step / per_step_s / 1e9 / peak,
+        "distinct_experts_per_step": distinct,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+class StackSetup:
+    """L resident layers (pool, router, Zipf offset each), 4-bit experts."""
+
+    def __init__(self, q, wl, seed, dev, L):
+        import torch
+        from _util import dev_router, fill_pool
+        H, E, K, I = wl["H"], wl["E"], wl["K"], wl["I"]
+        self.cfg = q.Cfg(H, E, K, I, 64, EPS32)
+        self.pools, self.W, self.off, self.layers = [], [], [], []
+        for l in range(L):
+            pool = q.ExpertPool(self.cfg, E, wl["bits"], device=dev)
+            fill_pool(pool, seed, l)
+            W = dev_router(seed, l, E, H, device=dev)
+            o = wl_offset(wl, seed, l)
+            off = torch.tensor(o, device=dev) if o is not None else None
+            self.pools.append(pool)
+            self.W.append(W)
+            self.off.append(off)
+            self.layers.append(q.Layer(W.data_ptr(), off.data_ptr() if off is not None else None, None,
+                                       pool.table.data_ptr()))
+
+
+def run_stack(args, wl, rank, world, local_rank):
+    """One step = one token through all L layers (one fused launch per layer,
+    residual between layers); CUDA graphs of 8 tokens."""
+    import torch
+    import quantized_expert_matvec_b200 as q
+    from _util import dev_tokens
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    H, E, K, I, L = wl["H"], wl["E"], wl["K"], wl["I"], wl["layers"]
+    st = StackSetup(q, wl, args.seed, dev, L)
+    ws = q.workspace(st.cfg, 1, device=dev)
+    n_tok = 256
+    x = dev_tokens(args.seed, 20_000_000 * (rank + 1), n_tok, H, device=dev)
+    act = torch.empty((2, 1, H), dtype=torch.float32, device=dev)
+    out = torch.empty((n_tok, H), dtype=torch.float32, device=dev)
+    idx = torch.empty((n_tok, L, K), dtype=torch.int32, device=dev)
+    s = torch.cuda.Stream(device=dev)
+
+    def token(t, stream, xin=None, dst=None, keep_idx=True):
+        cur = x[t:t + 1] if xin is None else xin
+        for l in range(L):
+            o = (dst if dst is not None else out[t:t + 1]) if l == L - 1 else act[l % 2]
+            q.moe_layer_step(st.cfg, st.layers[l], cur, o, True, idx[t, l:l + 1] if keep_idx else None, None,
+                             ws, stream=stream)
+            cur = o
+
+    chunk = 8
+    n_graphs = n_tok // chunk
+    with torch.cuda.stream(s):
+        token(0, s)
+        s.synchronize()
+        graphs = []
+        for c in range(n_graphs):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for i in range(chunk):
+                    token(c * chunk + i, s)
+            graphs.append(g)
+        rem = args.steps % chunk
+        rem_graph = None
+        if rem:
+            rem_graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(rem_graph, stream=s):
+                for i in range(rem):
+                    token(i, s)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        for i in range(max(1, args.warmup // chunk)):
+            graphs[i % n_graphs].replay()
+    s.synchronize()
+    if q.qe_workspace_status(ws, s) != q.QE_OK:
+        raise RuntimeError("device status after warm-up: " + q.qe_last_error())
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        ev0.record(s)
+        for i in range(args.steps // chunk):
+            graphs[i % n_graphs].replay()
+        if rem_graph is not None:
+            rem_graph.replay()
+        ev1.record(s)
+    s.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    ms = ev0.elapsed_time(ev1)
+    if q.qe_workspace_status(ws, s) != q.QE_OK:
+        raise RuntimeError("device status after timing: " + q.qe_last_error())
+    ms_max = sync_max(world, dev, ms)
+    ih = idx.cpu().numpy()
+    written = min(n_tok, max(args.steps, chunk))
+    distinct = float(np.mean([len(np.unique(ih[t, l])) for t in range(written) for l in range(L)])) * L
+    hot_share = None
+    if wl.get("zipf"):
+        import synth
+        hots = [synth.hot_set(args.seed, l, E, E // 4) for l in range(L)]
+        hot_share = float(np.mean([hots[l][ih[t, l]].mean() for t in range(written) for l in range(L)]))
+
+    # e2e: per token, pinned H2D of x, the L layer steps, D2H of the output
+    n_e2e = min(args.steps, 64)
+    x_host = x[:n_e2e].cpu().pin_memory()
+    out_host = torch.empty((1, H), dtype=torch.float32).pin_memory()
+    xin = torch.empty((1, H), dtype=torch.float32, device=dev)
+    res = torch.empty((1, H), dtype=torch.float32, device=dev)
+
+    def e2e_step(i):
+        xin.copy_(x_host[i % n_e2e:i % n_e2e + 1], non_blocking=True)
+        token(0, s, xin=xin, dst=res, keep_idx=False)
+        out_host.copy_(res, non_blocking=True)
+        s.synchronize()
+
+    with torch.cuda.stream(s):
+        for i in range(2):
+            e2e_step(i)
+    barrier(world)
+    t0 = time.perf_counter()
+    with torch.cuda.stream(s):
+        for i in range(n_e2e):
+            e2e_step(i)
+    e2e_s = sync_max(world, dev, time.perf_counter() - t0)
+    if rank != 0:
+        return
+    eb = expert_bytes(H, I, 4)
+    alg = distinct * eb + L * (E * H * 4 + 2 * H * 4 + E * 4)
+    e2e = {"value": world * n_e2e / e2e_s, "unit": UNIT, "h2d_bytes_per_step": H * 4, "d2h_bytes_per_step": H * 4,
+           "steps": n_e2e, "how": f"per token: pinned H2D of x, {L} moe_layer_step calls, D2H of out, sync"}
+    extra = {"layers": L, "tokens_per_step": 1, "tokens_distinct": n_tok,
+             "l2": f"inputs larger than L2: {L * E * eb / 1e9:.0f} GB of experts and {L * E * H * 4 / 1e6:.0f} MB "
+                   "of routers, read once per token",
+             "launch": f"CUDA graphs of {chunk} tokens x {L} layers", "zipf_alpha": 0.40,
+             "share_of_selections_in_hottest_25pct": hot_share}
+    finish_line(args, wl, world, ms_max, ms, args.steps, alg, distinct * eb, distinct, extra, e2e, clocks,
+                args.steps * L, "qe_fused_layer_kernel (one launch per layer)", "whole step (launch gaps included)")
+
+
+def pinned_host(nbytes):
+    """Page-locked host buffer of exactly nbytes (numpy-owned, registered
+    with the CUDA driver; the caller unregisters)."""
+    import torch
+    buf = np.empty(nbytes + 4096, dtype=np.uint8)
+    base = (buf.ctypes.data + 4095) // 4096 * 4096
+    rc = torch.cuda.cudart().cudaHostRegister(base, nbytes, 0)
+    if int(rc) != 0:
+        raise MemoryError(f"cudaHostRegister of {nbytes} bytes failed ({rc})")
+    return buf, base
+
+
+def mem_available():
+    try:
+        for ln in open("/proc/meminfo"):
+            if ln.startswith("MemAvailable:"):
+                return int(ln.split()[1]) * 1024
+    except OSError:
+        pass
+    return 0
+
+
+def run_tiered(args, wl, rank, world, local_rank):
+    """One step = one token through all tiered layers: per layer routing, one
+    host synchronisation, cache resolve (misses copied host->device on the
+    side stream), grouped expert FFNs and the combine with residual."""
+    import torch
+    import quantized_expert_matvec_b200 as q
+    from _util import dev_router, dev_tokens, fill_pool, fill_pool_slots
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    H, E, K, I, L, n_hot = wl["H"], wl["E"], wl["K"], wl["I"], wl["layers"], wl["hot"]
+    cfg = q.Cfg(H, E, K, I, 64, EPS32)
+    cold_b = q.qe_expert_bytes(cfg, 2)
+    n_cold = E - n_hot
+    need = L * n_cold * cold_b
+    avail = mem_available()
+    label = None
+    if need > 0.6 * avail:
+        L_fit = max(1, int(0.6 * avail // (n_cold * cold_b)))
+        label = (f"scaled down to {L_fit} of {L} layers: the cold pool needs {need / 1e9:.1f} GB of pinned host "
+                 f"memory, {avail / 1e9:.1f} GB available")
+        L = L_fit
+    import synth
+    hot = [synth.hot_set(args.seed, l, E, n_hot) for l in range(L)]
+    # cold pool: generated per layer on the device (2-bit, all experts), the
+    # cold ones copied to pinned host memory
+    stage = q.ExpertPool(cfg, E, 2, device=dev)
+    host_bufs, cold_host = [], []
+    for l in range(L):
+        fill_pool(stage, args.seed, l)
+        buf, base = pinned_host(n_cold * cold_b)
+        host_bufs.append((buf, base))
+        hv = torch.from_numpy(buf[base - buf.ctypes.data: base - buf.ctypes.data + n_cold * cold_b])
+        ptrs = [None] * E
+        cold_ids = [e for e in range(E) if not hot[l][e]]
+        sv = stage.buf[stage.base - stage.buf.data_ptr():]
+        for j, e in enumerate(cold_ids):
+            hv[j * cold_b:(j + 1) * cold_b].copy_(sv[e * stage.stride:e * stage.stride + cold_b])
+            ptrs[e] = base + j * cold_b
+        cold_host.append(ptrs)
+    del stage, sv
+    torch.cuda.synchronize()
+    pools, tables, Ws, offs, layers = [], [], [], [], []
+    for l in range(L):
+        hot_ids = [e for e in range(E) if hot[l][e]]
+        pool = q.ExpertPool(cfg, n_hot, 4, device=dev)
+        fill_pool_slots(pool, args.seed, l, hot_ids)
+        table = (q.Expert * E)()
+        for m, e in enumerate(hot_ids):
+            table[e] = pool.host_table[m]
+        dtab = torch.frombuffer(bytearray(bytes(table)), dtype=torch.uint8).to(dev)
+        W = dev_router(args.seed, l, E, H, device=dev)
+        off = torch.tensor(wl_offset(wl, args.seed, l), device=dev)
+        pools.append(pool)
+        tables.append(dtab)
+        Ws.append(W)
+        offs.append(off)
+        layers.append(q.Layer(W.data_ptr(), off.data_ptr(), None, dtab.data_ptr()))
+    tier = q.Tier(cfg, cold_host, 2, int(wl["cache_gb"] * 1e9), max_tokens=1)
+    ws = q.workspace(cfg, 1, device=dev)
+    n_tok = args.warmup + args.steps
+    x = dev_tokens(args.seed, 30_000_000 * (rank + 1), n_tok, H, device=dev)
+    act = torch.empty((2, 1, H), dtype=torch.float32, device=dev)
+    idx = torch.empty((n_tok, L, K), dtype=torch.int32, device=dev)
+    s = torch.cuda.Stream(device=dev)
+
+    def token(t, xin=None, dst=None):
+        cur = x[t:t + 1] if xin is None else xin
+        for l in range(L):
+            o = dst if (dst is not None and l == L - 1) else act[l % 2]
+            tier.layer_step(l, layers[l], cur, o, True, idx[t, l:l + 1] if xin is None else None, None, ws,
+                            stream=s)
+            cur = o
+
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        for t in range(args.warmup):
+            token(t)
+    s.synchronize()
+    h0, m0, b0 = tier.stats()
+    barrier(world)
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        ev0.record(s)
+        for t in range(args.warmup, n_tok):
+            token(t)
+        ev1.record(s)
+    s.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    ms = ev0.elapsed_time(ev1)
+    if q.qe_workspace_status(ws, s) != q.QE_OK:
+        raise RuntimeError("device status after timing: " + q.qe_last_error())
+    ms_max = sync_max(world, dev, ms)
+    h1, m1, b1 = tier.stats()
+    ih = idx[args.warmup:].cpu().numpy()
+    cold_sel = float(np.mean([[not hot[l][e] for e in ih[t, l]] for t in range(len(ih)) for l in range(L)]))
+    distinct = float(np.mean([len(np.unique(ih[t, l])) for t in range(len(ih)) for l in range(L)])) * L
+
+    n_e2e = min(args.steps, 16)
+    x_host = x[:n_e2e].cpu().pin_memory()
+    out_host = torch.empty((1, H), dtype=torch.float32).pin_memory()
+    xin = torch.empty((1, H), dtype=torch.float32, device=dev)
+    res = torch.empty((1, H), dtype=torch.float32, device=dev)
+    barrier(world)
+    t0 = time.perf_counter()
+    with torch.cuda.stream(s):
+        for i in range(n_e2e):
+            xin.copy_(x_host[i:i + 1], non_blocking=True)
+            token(0, xin=xin, dst=res)
+            out_host.copy_(res, non_blocking=True)
+            s.synchronize()
+    e2e_s = sync_max(world, dev, time.perf_counter() - t0)
+    tier.close()
+    for buf, base in host_bufs:
+        torch.cuda.cudart().cudaHostUnregister(base)
+    if rank != 0:
+        return
+    per_tok_hbm = L * ((1 - cold_sel) * K * expert_bytes(H, I, 4) + cold_sel * K * expert_bytes(H, I, 2)
+                       + E * H * 4 + 2 * H * 4)
+    steps_s = ms / 1000.0
+    e2e = {"value": world * n_e2e / e2e_s, "unit": UNIT, "h2d_bytes_per_step": H * 4, "d2h_bytes_per_step": H * 4,
+           "steps": n_e2e, "how": f"per token: pinned H2D of x, {L} qe_tier_layer_step calls, D2H of out, sync"}
+    extra = {"layers": L, "tokens_per_step": 1, "warmup_tokens_excluded": args.warmup,
+             "hot_per_layer": n_hot, "cold_per_layer": n_cold, "cache_gb": wl["cache_gb"],
+             "cache_slots": int(wl["cache_gb"] * 1e9 // cold_b), "cold_pool_gb": L * n_cold * cold_b / 1e9,
+             "cold_share_of_selections": cold_sel,
+             "cache_hit_rate": (h1 - h0) / max(1, (h1 - h0) + (m1 - m0)),
+             "h2d_gbs": (b1 - b0) / steps_s / 1e9, "misses_per_token": (m1 - m0) / args.steps,
+             "l2": "inputs larger than L2", "launch": "eager (one host synchronisation per layer)"}
+    if label:
+        extra["scaled"] = label
+    finish_line(args, wl, world, ms_max, ms, args.steps, per_tok_hbm, per_tok_hbm - L * (E * H * 4 + 2 * H * 4),
+                distinct, extra, e2e, clocks, args.steps * L * 5,
+                "per layer: route kernels, descriptor scatter, qe_fused_layer_kernel with the given routing",
+                "whole step (host sync per layer included)")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -486,10 +820,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
+    defaults = {"c2": (1024, 32), "c3": (224, 32)}
     if args.steps is None:
-        args.steps = 32768 if wl["T"] == 1 else 64
+        args.steps = defaults.get(args.workload, (32768 if wl["T"] == 1 else 64, 0))[0]
     if args.warmup is None:
-        args.warmup = 256 if wl["T"] == 1 else 8
+        args.warmup = defaults.get(args.workload, (0, 256 if wl["T"] == 1 else 8))[1]
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -504,7 +839,12 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_ours(args, wl, rank, world, local_rank)
+        if args.workload == "c2":
+            run_stack(args, wl, rank, world, local_rank)
+        elif args.workload == "c3":
+            run_tiered(args, wl, rank, world, local_rank)
+        else:
+            run_ours(args, wl, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -157,6 +157,37 @@ static int ffn_impl(const qe_cfg* c, const qe_expert* experts, const float* xn, 
   return QE_OK;
 }
 
+bool fused_fits(const qe_cfg* c) {
+  const DevInfo d = dev_info();
+  FusedGeometry g;
+  return fused_geometry(c->hidden, c->n_experts, c->top_k, c->inter, d.sms, d.optin, &g) == QE_OK;
+}
+
+int fused_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_dtype, float* out, int add_residual,
+               int32_t* topk_idx, float* topk_w, void* ws, const int32_t* given_idx, const float* given_w,
+               cudaStream_t s) {
+  const WsLayout L = ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, 1);
+  FusedParams p{};
+  const DevInfo d = dev_info();
+  if (fused_geometry(c->hidden, c->n_experts, c->top_k, c->inter, d.sms, d.optin, &p.g) != QE_OK)
+    return fail(QE_ERR_UNSUPPORTED, "shape not supported by the single-token kernel");
+  p.H = c->hidden; p.E = c->n_experts; p.K = c->top_k; p.I = c->inter; p.eps = c->eps;
+  p.x = x; p.x_bf16 = x_dtype == QE_BF16; p.add_residual = add_residual != 0;
+  p.gamma = layer->gamma; p.router_w = layer->router_w; p.offset = layer->logit_offset;
+  p.experts = layer->experts; p.out = out; p.topk_idx = topk_idx; p.topk_w = topk_w;
+  p.ctl = at<WsControl>(ws, L.control);
+  p.logit_part = at<double>(ws, L.logits);
+  p.hbuf = at<float>(ws, L.h);
+  p.given_idx = given_idx;
+  p.given_w = given_w;
+  p.budget_ns = g_budget_ns;
+  p.skip_cta = g_skip_cta;
+  p.trace = g_trace;
+  cudaError_t e = launch_fused_layer(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "fused layer launch");
+  return QE_OK;
+}
+
 }  // namespace qe
 
 using namespace qe;
@@ -298,27 +329,8 @@ int moe_layer_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_
   if ((const void*)out == x) return fail(QE_ERR_INVALID_ARG, "out must not alias x");
   cudaStream_t s = (cudaStream_t)stream;
   const WsLayout L = ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, T);
-  FusedParams p{};
-  bool fused = false;
-  if (T == 1) {
-    const DevInfo d = dev_info();
-    fused = fused_geometry(c->hidden, c->n_experts, c->top_k, c->inter, d.sms, d.optin, &p.g) == QE_OK;
-  }
-  if (fused) {
-    p.H = c->hidden; p.E = c->n_experts; p.K = c->top_k; p.I = c->inter; p.eps = c->eps;
-    p.x = x; p.x_bf16 = x_dtype == QE_BF16; p.add_residual = add_residual != 0;
-    p.gamma = layer->gamma; p.router_w = layer->router_w; p.offset = layer->logit_offset;
-    p.experts = layer->experts; p.out = out; p.topk_idx = topk_idx; p.topk_w = topk_w;
-    p.ctl = at<WsControl>(ws, L.control);
-    p.logit_part = at<double>(ws, L.logits);
-    p.hbuf = at<float>(ws, L.h);
-    p.budget_ns = g_budget_ns;
-    p.skip_cta = g_skip_cta;
-    p.trace = g_trace;
-    cudaError_t e = launch_fused_layer(p, s);
-    if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step fused launch");
-    return QE_OK;
-  }
+  if (T == 1 && fused_fits(c)) return fused_step(c, layer, x, x_dtype, out, add_residual, topk_idx, topk_w, ws,
+                                                   nullptr, nullptr, s);
   // batched (or a single token whose shape does not fit the fused kernel):
   // route all tokens, then the expert FFNs, then the combine
   int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.idx);

@@ -292,7 +292,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   // logit is s_e * rinv (+ offset_e), all in fp64.  Warp w covers the column
   // slice [w*S, (w+1)*S), S = H/16, of each router row its CTA owns; the 16
   // slice sums are added in slice order.
-  const int nrows = E > cta ? (E - cta + G - 1) / G : 0;
+  const bool given = p.given_idx != nullptr;
+  const int nrows = (!given && E > cta) ? (E - cta + G - 1) / G : 0;
   {
     const int S = H / kWarps;
     double ss = 0.0;
@@ -380,8 +381,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   __syncthreads();
   if (tid == 0) {
     QE_TRACE(kTrRouterDone);
-    __threadfence();
-    if (cta != p.skip_cta) atomicAdd(&ctl->route_ctr, 1u);
+    if (!given) {
+      __threadfence();
+      if (cta != p.skip_cta) atomicAdd(&ctl->route_ctr, 1u);
+    }
   }
   {
     float m = 0.f;
@@ -401,7 +404,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
     }
   }
   if (tid == 0) {
-    if (!wait_geq(&ctl->route_ctr, (unsigned)G, deadline, abort_flag)) {
+    if (!given && !wait_geq(&ctl->route_ctr, (unsigned)G, deadline, abort_flag)) {
       set_error(&ctl->err, QE_ERR_TIMEOUT);
       misc->abort = 1;
     }
@@ -413,7 +416,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   // Thread t ranks logits t and t+512.  Each warp finds its own top-K by K
   // rounds of warp_argmax_key (a sorted candidate list, keys and values kept
   // in shared memory); warp 0 then merges the 16 lists, one list per lane.
-  if (!*abort_flag) {
+  if (!given && !*abort_flag) {
     const unsigned iA = (unsigned)tid, iB = (unsigned)(tid + kFusedThreads);
     bool hasA = tid < E, hasB = tid + kFusedThreads < E;
     const double vA = hasA ? __ldcg(&p.logit_part[iA]) : 0.0;
@@ -436,7 +439,29 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
     }
   }
   __syncthreads();
-  if (warp == 0 && !*abort_flag) {
+  if (warp == 0 && given && !*abort_flag) {
+    // routing decided beforehand: take its experts and weights as they are
+    if (lane < K) {
+      const int e = p.given_idx[lane];
+      misc->wk[lane] = p.given_w[lane];
+      if (cta == 0 && p.topk_idx) p.topk_idx[lane] = e;
+      if (cta == 0 && p.topk_w) p.topk_w[lane] = p.given_w[lane];
+      bool ok = e >= 0 && e < E;
+      qe_expert ex{};
+      if (ok) {
+        ex = p.experts[e];
+        const int bits = ex.gate.bits;
+        ok = (bits == 4 || bits == 2) && desc_ok(ex.gate, bits) && desc_ok(ex.up, bits) && desc_ok(ex.down, bits);
+      }
+      if (!ok) {
+        set_error(&ctl->err, QE_ERR_INVALID_ARG);
+        misc->abort = 1;
+      }
+      misc->idx[lane] = e;
+      misc->ex[lane] = ex;
+    }
+  }
+  if (warp == 0 && !given && !*abort_flag) {
     int ptr = 0;
     double myval = 0.0;
     for (int k = 0; k < K; ++k) {

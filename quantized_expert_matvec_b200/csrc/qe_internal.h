@@ -82,6 +82,10 @@ struct FusedParams {
   WsControl* ctl;
   double* logit_part;  // [E] routing logits
   float* hbuf;         // [K][I]
+  // routing decided beforehand (device [K] each), or null: the kernel then
+  // skips the router, the routing barrier and the top-K
+  const int32_t* given_idx;
+  const float* given_w;
   FusedGeometry g;
   unsigned long long budget_ns;
   int skip_cta;
@@ -182,6 +186,10 @@ qe_expert pool_descriptor(const qe_cfg* c, void* base, int bits);
 int route_impl(const qe_cfg* c, const void* x, int x_dtype, const float* gamma, const float* router_w,
                const float* offset, int T, float* xn, int32_t* idx, float* w, void* ws, size_t ws_bytes,
                bool want_xprime, cudaStream_t s);
+bool fused_fits(const qe_cfg* c);
+int fused_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_dtype, float* out, int add_residual,
+               int32_t* topk_idx, float* topk_w, void* ws, const int32_t* given_idx, const float* given_w,
+               cudaStream_t s);
 int experts_and_combine(const qe_cfg* c, const qe_expert* experts, const int32_t* idx, const float* w, const void* x,
                         int x_dtype, int T, float* out, int add_residual, void* ws, cudaStream_t s);
 

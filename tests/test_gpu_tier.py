@@ -146,3 +146,35 @@ def test_tiered_batched_call_and_oom(q):
     assert ei.value.code == q.QE_ERR_OOM
     assert small.stats() == (0, 0, 0)
     small.close()
+
+
+def test_tiered_full_layer_shape(q):
+    """The tiered workload's layer shape (hidden 4096, 512 experts: the 128
+    most popular 4-bit in HBM, 384 2-bit in pinned host memory), two layers,
+    a 48-slot cache, six tokens; every layer output against the oracle."""
+    import torch
+    cfg = q.Cfg(4096, 512, 4, 1024)
+    st = TieredStack(q, cfg, n_layers=2, n_hot=128, seed=0, cache_slots=48, max_tokens=1)
+    model = LruModel(48)
+    K, H, E = cfg.top_k, cfg.hidden, cfg.n_experts
+    x = dev_tokens(0, 123_000, 6, H)
+    n_ok = 0
+    for t in range(6):
+        cur = x[t:t + 1].clone()
+        for l in range(2):
+            out = torch.empty((1, H), dtype=torch.float32, device="cuda")
+            idx = torch.empty((1, K), dtype=torch.int32, device="cuda")
+            st.tier.layer_step(l, st.layers[l], cur, out, True, idx, None, st.ws)
+            idx_h = idx.cpu().numpy()[0]
+            model.call([l * E + int(e) for e in idx_h if not st.hot[l][int(e)]])
+            ref = st.oracle(l, cur.cpu().numpy()[0].astype(np.float64))
+            assert routing_matches(idx_h, ref["logits"], ref["idx"], K)
+            if list(idx_h) == list(ref["idx"]):
+                assert normwise_err(out.cpu().numpy()[0], ref["out"]) <= TOL
+                n_ok += 1
+            cur = out
+    assert q.qe_workspace_status(st.ws) == q.QE_OK, q.qe_last_error()
+    hits, misses, _ = st.tier.stats()
+    assert (hits, misses) == (model.hits, model.misses)
+    assert n_ok >= 11
+    st.tier.close()
