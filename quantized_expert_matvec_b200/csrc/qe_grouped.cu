@@ -2,17 +2,20 @@
 // assignments are grouped by expert so each selected expert's weights are
 // streamed from HBM once per step and reused by all of its tokens.
 //
-//   group kernel : counting sort of the T*K assignments by expert (stable:
-//                  ascending assignment id inside an expert)
-//   expert kernel: persistent CTAs take whole experts from a shared counter;
-//                  per expert: stage the x' of its tokens in shared memory,
-//                  gate/up rows (a warp takes blocks of kRowBlk rows and
-//                  runs every token over them; after the first token the
-//                  block's packed words come from L1),
-//                  h = silu(g) u in shared memory, then down rows ->
-//                  y[assignment][H]
-//   combine      : out[t] = sum_k w[t,k] y[t*K+k] (+ x[t])
-// Up to kTokTile tokens of an expert are processed per pass over its weights.
+//   group kernel  : counting sort of the T*K assignments by expert (stable:
+//                   ascending assignment id inside an expert); active experts
+//                   ordered by descending token count
+//   gate/up kernel: persistent CTAs take items (expert, block of kRowsA
+//                   rows) from a shared counter; the CTA stages the x' of the
+//                   expert's tokens in shared memory and each warp takes
+//                   rows: a packed word is masked once and multiplied into
+//                   the accumulators of every token; h = silu(g) u and the
+//                   running max |h| per assignment go to global memory
+//   down kernel   : items (expert, block of kRowsB output rows); the CTA
+//                   stages h of the expert's tokens in x' form, warps take
+//                   pairs of rows -> y[assignment][H]
+//   combine       : out[t] = sum_k w[t,k] y[t*K+k] (+ x[t])
+// Up to kTT tokens of an expert share one pass over its weights.
 #include <math.h>
 
 #include "qe_device.cuh"
@@ -21,21 +24,26 @@ namespace qe {
 
 constexpr int kGWarps = 16;
 constexpr int kGThreads = kGWarps * 32;
-constexpr int kTokTile = 8;  // tokens staged per pass over an expert's weights
-constexpr int kRowBlk = 4;   // rows per warp block
+constexpr int kTT = 8;       // tokens sharing one pass over the weights
+constexpr int kRowsA = 128;  // gate/up rows (of gate and of up) per item
+constexpr int kRowsB = 512;  // down rows per item
 
 // Round a count of 4-byte elements up to a multiple of 4 (16 bytes).
 static __host__ __device__ __forceinline__ int al4(int n) { return (n + 3) & ~3; }
 
 // -------------------------------------------------------------- grouping
+// One CTA of 1024 threads (E <= 1024).  Also zeroes the per-assignment |h|
+// maxima and the two work counters of the expert kernels.
 __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__ idx, int A, int E, int* count,
-                                                     int* start, int* list, int* order, int* n_active,
-                                                     int* err) {
-  extern __shared__ int sh[];
-  int* cnt = sh;          // [E]
-  int* cur = sh + E;      // [E]
-  const int tid = threadIdx.x;
+                                                     int* start, int* list, int* order, int* ctl,
+                                                     unsigned* hamax, int* err) {
+  __shared__ int cnt[kMaxE];
+  __shared__ int cur[kMaxE];
+  __shared__ int wsum[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+  for (int a = tid; a < A; a += blockDim.x) hamax[a] = 0u;
+  if (tid < 4) ctl[tid] = 0;  // [0] active experts, [1] gate/up work, [2] down work
   __syncthreads();
   for (int a = tid; a < A; a += blockDim.x) {
     const int e = idx[a];
@@ -43,18 +51,43 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__
     atomicAdd(&cnt[e], 1);
   }
   __syncthreads();
-  if (tid == 0) {
-    int s = 0, na = 0;
-    for (int e = 0; e < E; ++e) {
-      start[e] = s;
-      cur[e] = s;
-      count[e] = cnt[e];
-      s += cnt[e];
-      if (cnt[e] > 0) order[na++] = e;
-    }
-    start[E] = s;
-    *n_active = na;
+  // exclusive scan of the counts (thread e holds expert e)
+  const int c = tid < E ? cnt[tid] : 0;
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
   }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    wsum[lane] = v;  // inclusive over warps
+  }
+  __syncthreads();
+  const int excl = incl - c + (warp > 0 ? wsum[warp - 1] : 0);
+  if (tid < E) {
+    start[tid] = excl;
+    cur[tid] = excl;
+    count[tid] = c;
+    if (c > 0) {
+      // rank among active experts: more tokens first, then lower index
+      int rank = 0;
+      for (int f = 0; f < E; ++f) {
+        const int cf = cnt[f];
+        rank += (cf > c) || (cf == c && f < tid);
+      }
+      order[rank] = tid;
+      atomicAdd(&ctl[0], 1);
+    }
+  }
+  if (tid == 0) start[E] = wsum[31];
   __syncthreads();
   for (int a = tid; a < A; a += blockDim.x) {
     const int e = idx[a];
@@ -62,56 +95,95 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__
     list[atomicAdd(&cur[e], 1)] = a;
   }
   __syncthreads();
-  // restore ascending assignment order inside each expert (lists are short)
-  for (int e = tid; e < E; e += blockDim.x) {
-    int* l = list + start[e];
-    const int n = cnt[e];
-    for (int i = 1; i < n; ++i) {
+  // ascending assignment order inside each expert (lists are short)
+  if (tid < E) {
+    int* l = list + excl;
+    for (int i = 1; i < c; ++i) {
       const int v = l[i];
       int j = i - 1;
       while (j >= 0 && l[j] > v) { l[j + 1] = l[j]; --j; }
       l[j + 1] = v;
     }
   }
-  __syncthreads();
-  // larger groups first so the persistent CTAs end together: a stable
-  // counting sort of the active experts by descending token count
-  if (tid == 0) {
-    int na = 0, maxc = 0;
-    for (int e = 0; e < E; ++e) maxc = cnt[e] > maxc ? cnt[e] : maxc;
-    for (int c = maxc; c >= 1; --c)
-      for (int e = 0; e < E; ++e)
-        if (cnt[e] == c) order[na++] = e;
-  }
 }
 
-struct ExpertParams {
+struct GroupedKParams {
   int H, I, K, T;
   const qe_expert* experts;
-  const float* xp4;   // [T][H] x' (linear layout, global)
+  const float* xp4;   // [T][H] x' (linear layout)
   const float* xp2;
   const float* xsum;  // [T][H/32]
   const int* xexp;    // [T]
+  const int* count;
   const int* start;
   const int* list;
   const int* order;
-  const int* n_active;
-  int* work;          // shared work counter (reset by the caller)
+  int* ctl;           // [0] active experts, [1] gate/up work, [2] down work
+  float* h;           // [T*K][I]
+  unsigned* hamax;    // [T*K]
   float* y;           // [T*K][H]
   int* err;
-  int tile;           // tokens per pass over an expert's weights
+  int tile;           // tokens per pass (<= kTT)
 };
 
-// Stage the x' (4- or 2-bit form, swizzled) and 32-column sums of `nt`
-// tokens into shared memory.
-static __device__ void stage_tokens(const ExpertParams& p, int bits, const int* toks, int nt, float* xs_sm,
-                                    float* sum_sm, float* xk_sm) {
+static __device__ __forceinline__ bool qmat_ok(const qe_qmat& m, int bits) {
+  return m.bits == bits && m.wq && m.scales && m.biases && ((uintptr_t)m.wq & 15) == 0;
+}
+
+// Masked field pairs of one packed word (4-bit: 4 pairs, 2-bit: 8 pairs),
+// in the pair order of the x' layout (see dot8_q4 / dot16_q2).
+template <int BITS>
+static __device__ __forceinline__ void mask_word(uint32_t v, float2 (&m)[BITS == 4 ? 4 : 8]) {
+  const uint32_t hv = v >> 12;
+  if (BITS == 4) {
+    m[0] = make_float2(f_of(v & 0xFu), f_of(v & 0xF0u));
+    m[1] = make_float2(f_of(v & 0xF00u), f_of(v & 0xF000u));
+    m[2] = make_float2(f_of(v & 0xF0000u), f_of(hv & 0xF00u));
+    m[3] = make_float2(f_of(hv & 0xF000u), f_of(hv & 0xF0000u));
+  } else {
+    m[0] = make_float2(f_of(v & 0x3u), f_of(v & 0xCu));
+    m[1] = make_float2(f_of(v & 0x30u), f_of(v & 0xC0u));
+    m[2] = make_float2(f_of(v & 0x300u), f_of(v & 0xC00u));
+    m[3] = make_float2(f_of(v & 0x3000u), f_of(v & 0xC000u));
+    m[4] = make_float2(f_of(v & 0x30000u), f_of(v & 0xC0000u));
+    m[5] = make_float2(f_of(v & 0x300000u), f_of(hv & 0xC00u));
+    m[6] = make_float2(f_of(hv & 0x3000u), f_of(hv & 0xC000u));
+    m[7] = make_float2(f_of(hv & 0x30000u), f_of(hv & 0xC0000u));
+  }
+}
+
+// x' pairs of word j of lane chunk lc (32 columns) from a swizzled buffer.
+template <int BITS>
+static __device__ __forceinline__ void xs_word(const float* xp, int lc, int j, float2 (&x)[BITS == 4 ? 4 : 8]) {
+  if (BITS == 4) {
+    const float4* src = (const float4*)(xp + lc * 32);
+    const int sw = lc & 7;
+    const float4 a = src[(2 * j) ^ sw], b = src[(2 * j + 1) ^ sw];
+    x[0] = make_float2(a.x, a.y); x[1] = make_float2(a.z, a.w);
+    x[2] = make_float2(b.x, b.y); x[3] = make_float2(b.z, b.w);
+  } else {
+    const int ch = lc >> 1, hf = lc & 1;
+    const float4* src = (const float4*)(xp + ch * 64);
+    const int sw = ch & 7;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 a = src[(8 * hf + 4 * j + i) ^ sw];
+      x[2 * i] = make_float2(a.x, a.y);
+      x[2 * i + 1] = make_float2(a.z, a.w);
+    }
+  }
+}
+
+// Stage x' (swizzled), 32-column sums and scale of nt tokens.
+static __device__ void stage_x(const GroupedKParams& p, int bits, const int* toks, int nt, float* xs_sm,
+                               float* sum_sm, float* xk_sm) {
   const int H = p.H;
   const float* src = bits == 4 ? p.xp4 : p.xp2;
-  for (int i = threadIdx.x; i < nt * H; i += kGThreads) {
-    const int t = i / H, c = i - t * H;
-    const float v = src[(size_t)toks[t] * H + c];
-    xs_sm[t * H + (bits == 4 ? swz_q4(c) : swz_q2(c))] = v;
+  for (int i = threadIdx.x; i < nt * (H / 4); i += kGThreads) {
+    const int t = i / (H / 4), c = (i - t * (H / 4)) * 4;
+    const float4 v = *(const float4*)(src + (size_t)toks[t] * H + c);
+    const int d = bits == 4 ? swz_q4(c) : swz_q2(c);  // 4 consecutive columns stay together
+    *(float4*)(xs_sm + t * H + d) = v;
   }
   for (int i = threadIdx.x; i < nt * (H / 32); i += kGThreads) {
     const int t = i / (H / 32), c = i - t * (H / 32);
@@ -120,203 +192,318 @@ static __device__ void stage_tokens(const ExpertParams& p, int bits, const int* 
   if (threadIdx.x < nt) xk_sm[threadIdx.x] = acc_scale(p.xexp[toks[threadIdx.x]]);
 }
 
-// kRowBlk rows (r0 .. r0+nv-1) of a packed matrix with `cols` columns
-// against one token's x' (shared memory): acc[i] collects this lane's partial
-// sum of row r0+i.  The block's packed rows are small (kRowBlk * cols/2
-// bytes), so the tokens after the first read them from L1.
+// One gate row and one up row (row r) against the nt staged tokens: v[t]
+// (gate) and v[kTT + t] (up) get this lane's partial sums.
 template <int BITS>
-static __device__ __forceinline__ void block_rows(const qe_qmat& m, int r0, int nv, int cols, const float* xs_t,
-                                                  const float* sum_t, float xk, float (&acc)[kRowBlk], int lane) {
-  const int gpr = cols / kGroup;
-  const size_t rowb = (size_t)cols * BITS / 8;
-  const unsigned char* base = (const unsigned char*)m.wq + (size_t)r0 * rowb;
-  for (int lc = lane; lc < cols / 32; lc += 32) {
-    uint4 w[kRowBlk];
-    uint32_t sb[kRowBlk];
-    const int g = lc >> 1;
+static __device__ __forceinline__ void gateup_row(const qe_expert& ex, int r, int H, int nt, const float* xs_sm,
+                                                  const float* sum_sm, const float* xk_sm, float (&v)[2 * kTT],
+                                                  int lane) {
+  constexpr int NP = BITS == 4 ? 4 : 8;
+  constexpr int WPC = BITS == 4 ? 4 : 2;  // words per 32-column chunk
+  const int gpr = H / kGroup;
+  const size_t rowb = (size_t)H * BITS / 8;
+  const unsigned char* gp = (const unsigned char*)ex.gate.wq + (size_t)r * rowb;
+  const unsigned char* up = (const unsigned char*)ex.up.wq + (size_t)r * rowb;
+  for (int lc = lane; lc < H / 32; lc += 32) {
+    uint32_t wg[WPC], wu[WPC];
+    if (BITS == 4) {
+      const uint4 a = __ldcs((const uint4*)gp + lc), b = __ldcs((const uint4*)up + lc);
+      wg[0] = a.x; wg[1] = a.y; wg[2 % WPC] = a.z; wg[3 % WPC] = a.w;
+      wu[0] = b.x; wu[1] = b.y; wu[2 % WPC] = b.z; wu[3 % WPC] = b.w;
+    } else {
+      const uint2 a = __ldcs((const uint2*)gp + lc), b = __ldcs((const uint2*)up + lc);
+      wg[0] = a.x; wg[1 % WPC] = a.y;
+      wu[0] = b.x; wu[1 % WPC] = b.y;
+    }
+    const size_t gi = (size_t)r * gpr + (lc >> 1);
+    const float sg = bf16f(__ldg(ex.gate.scales + gi)), bg = bf16f(__ldg(ex.gate.biases + gi));
+    const float su = bf16f(__ldg(ex.up.scales + gi)), bu = bf16f(__ldg(ex.up.biases + gi));
+    float2 ga[kTT], ua[kTT];
 #pragma unroll
-    for (int i = 0; i < kRowBlk; ++i) {
-      if (i < nv) {
-        const unsigned char* rp = base + (size_t)i * rowb;
-        if (BITS == 4) {
-          w[i] = __ldg((const uint4*)rp + lc);
-        } else {
-          const uint2 v = __ldg((const uint2*)rp + lc);
-          w[i] = make_uint4(v.x, v.y, 0u, 0u);
+    for (int t = 0; t < kTT; ++t) { ga[t] = make_float2(0.f, 0.f); ua[t] = make_float2(0.f, 0.f); }
+#pragma unroll
+    for (int j = 0; j < WPC; ++j) {
+      float2 mg[NP], mu[NP];
+      mask_word<BITS>(wg[j], mg);
+      mask_word<BITS>(wu[j], mu);
+#pragma unroll
+      for (int t = 0; t < kTT; ++t) {
+        if (t < nt) {
+          float2 xw[NP];
+          xs_word<BITS>(xs_sm + t * H, lc, j, xw);
+#pragma unroll
+          for (int i = 0; i < NP; ++i) {
+            ga[t] = __ffma2_rn(mg[i], xw[i], ga[t]);
+            ua[t] = __ffma2_rn(mu[i], xw[i], ua[t]);
+          }
         }
-        const size_t gi = (size_t)(r0 + i) * gpr + g;
-        sb[i] = (uint32_t)__ldg(m.scales + gi) | ((uint32_t)__ldg(m.biases + gi) << 16);
       }
     }
-    float2 xs[16];
-    if (BITS == 4) load_xs32_q4(xs_t, lc, xs);
-    else load_xs32_q2(xs_t, lc, xs);
-    const float xsum = sum_t[lc];
 #pragma unroll
-    for (int i = 0; i < kRowBlk; ++i) {
-      if (i < nv) {
-        const float2 a = BITS == 4 ? dot32_q4(w[i], xs, make_float2(0.f, 0.f))
-                                   : dot32_q2(make_uint2(w[i].x, w[i].y), xs, make_float2(0.f, 0.f));
-        acc[i] += bf16f(sb[i] & 0xFFFFu) * xk * (a.x + a.y) + bf16f(sb[i] >> 16) * xsum;
+    for (int t = 0; t < kTT; ++t) {
+      if (t < nt) {
+        const float xk = xk_sm[t], xsum = sum_sm[t * (H / 32) + lc];
+        v[t] += sg * xk * (ga[t].x + ga[t].y) + bg * xsum;
+        v[kTT + t] += su * xk * (ua[t].x + ua[t].y) + bu * xsum;
       }
     }
   }
 }
 
-__global__ void __launch_bounds__(kGThreads, 1) grouped_expert_kernel(const ExpertParams p) {
+template <int BITS>
+static __device__ void gateup_item(const GroupedKParams& p, const qe_expert& ex, int r0, int r1, int nt,
+                                   const int* asg, const float* xs_sm, const float* sum_sm, const float* xk_sm,
+                                   int warp, int lane) {
+  const int H = p.H, I = p.I;
+  for (int r = r0 + warp; r < r1; r += kGWarps) {
+    float v[2 * kTT];  // gate sums of the tokens, then up sums
+#pragma unroll
+    for (int t = 0; t < 2 * kTT; ++t) v[t] = 0.f;
+    gateup_row<BITS>(ex, r, H, nt, xs_sm, sum_sm, xk_sm, v, lane);
+    const float s = warp_reduce_rows<2 * kTT>(v, lane);
+    const int row = reduced_row_of_lane<2 * kTT>(lane);
+    // lanes holding g of token t fetch u of token t
+    const int src = lane_of_reduced_row<2 * kTT>(row < kTT ? row + kTT : row);
+    const float uv = __shfl_sync(0xffffffffu, s, src);
+    if (row < nt && lane == lane_of_reduced_row<2 * kTT>(row)) {
+      const float hv = s / (1.0f + expf(-s)) * uv;
+      const int a = asg[row];
+      p.h[(size_t)a * I + r] = hv;
+      atomicMax(&p.hamax[a], __float_as_uint(fabsf(hv)));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kGThreads, 1) grouped_gateup_kernel(const GroupedKParams p) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int H = p.H, I = p.I, tile = p.tile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // every region starts on a 16-byte boundary (float4 reads of x' and h')
-  float* xs_sm = (float*)smem;                            // [tile][H]
-  float* xsum_sm = xs_sm + al4(tile * H);                 // [tile][H/32]
-  float* xk_sm = xsum_sm + al4(tile * (H / 32));          // [tile]
-  float* h_sm = xk_sm + al4(tile);                        // [tile][I] raw h
-  float* hp_sm = h_sm + al4(tile * I);                    // [tile][I] x' of h
-  float* hsum_sm = hp_sm + al4(tile * I);                 // [tile][I/32]
-  float* hk_sm = hsum_sm + al4(tile * (I / 32));          // [tile]
-  int* toks = (int*)(hk_sm + al4(tile));                  // [tile]
-  int* asg = toks + al4(tile);                            // [tile]
-  unsigned* hmax = (unsigned*)(asg + al4(tile));          // [tile]
+  float* xs_sm = (float*)smem;                    // [tile][H]
+  float* sum_sm = xs_sm + al4(tile * H);          // [tile][H/32]
+  float* xk_sm = sum_sm + al4(tile * (H / 32));   // [tile]
+  int* toks = (int*)(xk_sm + al4(tile));          // [tile]
+  int* asg = toks + al4(tile);                    // [tile]
   __shared__ int s_item;
   __shared__ qe_expert s_ex;
-  const int na = *p.n_active;
+  const int ipe = (I + kRowsA - 1) / kRowsA;
+  const int n_items = p.ctl[0] * ipe;
   for (;;) {
-    if (threadIdx.x == 0) s_item = atomicAdd(p.work, 1);
+    if (threadIdx.x == 0) s_item = atomicAdd(&p.ctl[1], 1);
     __syncthreads();
     const int item = s_item;
-    __syncthreads();
-    if (item >= na) break;
-    const int e = p.order[item];
-    // the descriptor lives in shared memory, not in 24 registers
+    if (item >= n_items) break;
+    const int e = p.order[item / ipe];
+    const int r0 = (item % ipe) * kRowsA, r1 = min(I, r0 + kRowsA);
     if (threadIdx.x == 0) s_ex = p.experts[e];
     __syncthreads();
-    const qe_expert& ex = s_ex;
-    const int bits = ex.gate.bits;
-    if (!(bits == 4 || bits == 2) || ex.up.bits != bits || ex.down.bits != bits || !ex.gate.wq || !ex.up.wq ||
-        !ex.down.wq || ((uintptr_t)ex.gate.wq & 15) || ((uintptr_t)ex.up.wq & 15) || ((uintptr_t)ex.down.wq & 15)) {
+    const int bits = s_ex.gate.bits;
+    const bool ok = (bits == 4 || bits == 2) && qmat_ok(s_ex.gate, bits) && qmat_ok(s_ex.up, bits) &&
+                    qmat_ok(s_ex.down, bits);
+    if (!ok) {
       if (threadIdx.x == 0) set_error(p.err, QE_ERR_INVALID_ARG);
+      __syncthreads();
       continue;
     }
-    const int n = p.start[e + 1] - p.start[e];
+    const int n = p.count[e], s0 = p.start[e];
     for (int t0 = 0; t0 < n; t0 += tile) {
-      const int nt = n - t0 < tile ? n - t0 : tile;
+      const int nt = min(tile, n - t0);
       if (threadIdx.x < nt) {
-        const int a = p.list[p.start[e] + t0 + threadIdx.x];
+        const int a = p.list[s0 + t0 + threadIdx.x];
         asg[threadIdx.x] = a;
         toks[threadIdx.x] = a / p.K;
-        hmax[threadIdx.x] = 0u;
       }
       __syncthreads();
-      stage_tokens(p, bits, toks, nt, xs_sm, xsum_sm, xk_sm);
+      stage_x(p, bits, toks, nt, xs_sm, sum_sm, xk_sm);
       __syncthreads();
-      // -------------------------------- gate/up: kRowBlk-row blocks per warp
-      for (int r0 = warp * kRowBlk; r0 < I; r0 += kGWarps * kRowBlk) {
-        const int nv = I - r0 < kRowBlk ? I - r0 : kRowBlk;
-        for (int t = 0; t < nt; ++t) {
-          float ga[kRowBlk], ua[kRowBlk];
+      if (bits == 4) gateup_item<4>(p, s_ex, r0, r1, nt, asg, xs_sm, sum_sm, xk_sm, warp, lane);
+      else gateup_item<2>(p, s_ex, r0, r1, nt, asg, xs_sm, sum_sm, xk_sm, warp, lane);
+      __syncthreads();
+    }
+  }
+}
+
+// Two down rows (r and, if two == 2, r + 1) against the nt staged h'
+// vectors: v[t] and v[kTT + t] get this lane's partial sums.
+template <int BITS>
+static __device__ __forceinline__ void down_rows(const qe_qmat& d, int r, int two, int I, int nt, const float* hs_sm,
+                                                 const float* hsum_sm, const float* hk_sm, float (&v)[2 * kTT],
+                                                 int lane) {
+  constexpr int NP = BITS == 4 ? 4 : 8;
+  constexpr int WPC = BITS == 4 ? 4 : 2;
+  const int gpr = I / kGroup;
+  const size_t rowb = (size_t)I * BITS / 8;
+  for (int lc = lane; lc < I / 32; lc += 32) {
+    uint32_t w[2][WPC];
+    float sc[2], bi[2];
 #pragma unroll
-          for (int i = 0; i < kRowBlk; ++i) { ga[i] = 0.f; ua[i] = 0.f; }
-          const float* xst = xs_sm + t * H;
-          const float* sst = xsum_sm + t * (H / 32);
-          if (bits == 4) {
-            block_rows<4>(ex.gate, r0, nv, H, xst, sst, xk_sm[t], ga, lane);
-            block_rows<4>(ex.up, r0, nv, H, xst, sst, xk_sm[t], ua, lane);
-          } else {
-            block_rows<2>(ex.gate, r0, nv, H, xst, sst, xk_sm[t], ga, lane);
-            block_rows<2>(ex.up, r0, nv, H, xst, sst, xk_sm[t], ua, lane);
-          }
-          const float gv = warp_reduce_rows<kRowBlk>(ga, lane);
-          const float uv = warp_reduce_rows<kRowBlk>(ua, lane);
-          const int i = reduced_row_of_lane<kRowBlk>(lane);
-          if (lane == lane_of_reduced_row<kRowBlk>(i) && i < nv) {
-            const float hv = gv / (1.0f + expf(-gv)) * uv;
-            h_sm[t * I + r0 + i] = hv;
-            atomicMax(&hmax[t], __float_as_uint(fabsf(hv)));
+    for (int q = 0; q < 2; ++q) {
+      const int rr = r + (q < two ? q : 0);
+      const unsigned char* rp = (const unsigned char*)d.wq + (size_t)rr * rowb;
+      if (BITS == 4) {
+        const uint4 a = __ldcs((const uint4*)rp + lc);
+        w[q][0] = a.x; w[q][1] = a.y; w[q][2 % WPC] = a.z; w[q][3 % WPC] = a.w;
+      } else {
+        const uint2 a = __ldcs((const uint2*)rp + lc);
+        w[q][0] = a.x; w[q][1 % WPC] = a.y;
+      }
+      const size_t gi = (size_t)rr * gpr + (lc >> 1);
+      sc[q] = bf16f(__ldg(d.scales + gi));
+      bi[q] = bf16f(__ldg(d.biases + gi));
+    }
+    float2 acc[2][kTT];
+#pragma unroll
+    for (int t = 0; t < kTT; ++t) { acc[0][t] = make_float2(0.f, 0.f); acc[1][t] = make_float2(0.f, 0.f); }
+#pragma unroll
+    for (int j = 0; j < WPC; ++j) {
+      float2 m0[NP], m1[NP];
+      mask_word<BITS>(w[0][j], m0);
+      mask_word<BITS>(w[1][j], m1);
+#pragma unroll
+      for (int t = 0; t < kTT; ++t) {
+        if (t < nt) {
+          float2 xw[NP];
+          xs_word<BITS>(hs_sm + t * I, lc, j, xw);
+#pragma unroll
+          for (int i = 0; i < NP; ++i) {
+            acc[0][t] = __ffma2_rn(m0[i], xw[i], acc[0][t]);
+            acc[1][t] = __ffma2_rn(m1[i], xw[i], acc[1][t]);
           }
         }
       }
+    }
+#pragma unroll
+    for (int t = 0; t < kTT; ++t) {
+      if (t < nt) {
+        const float hk = hk_sm[t], hsum = hsum_sm[t * (I / 32) + lc];
+        v[t] += sc[0] * hk * (acc[0][t].x + acc[0][t].y) + bi[0] * hsum;
+        v[kTT + t] += sc[1] * hk * (acc[1][t].x + acc[1][t].y) + bi[1] * hsum;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kGThreads, 1) grouped_down_kernel(const GroupedKParams p) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int H = p.H, I = p.I, tile = p.tile;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* hs_sm = (float*)smem;                     // [tile][I] x' of h
+  float* hsum_sm = hs_sm + al4(tile * I);          // [tile][I/32]
+  float* hk_sm = hsum_sm + al4(tile * (I / 32));   // [tile]
+  int* asg = (int*)(hk_sm + al4(tile));            // [tile]
+  int* hexp = asg + al4(tile);                     // [tile]
+  __shared__ int s_item;
+  __shared__ qe_qmat s_d;
+  const int ipe = (H + kRowsB - 1) / kRowsB;
+  const int n_items = p.ctl[0] * ipe;
+  for (;;) {
+    if (threadIdx.x == 0) s_item = atomicAdd(&p.ctl[2], 1);
+    __syncthreads();
+    const int item = s_item;
+    if (item >= n_items) break;
+    const int e = p.order[item / ipe];
+    const int r0 = (item % ipe) * kRowsB, r1 = min(H, r0 + kRowsB);
+    if (threadIdx.x == 0) s_d = p.experts[e].down;
+    __syncthreads();
+    const int bits = s_d.bits;
+    if (!((bits == 4 || bits == 2) && qmat_ok(s_d, bits))) {
+      if (threadIdx.x == 0) set_error(p.err, QE_ERR_INVALID_ARG);
       __syncthreads();
-      // -------------------------------------------------- x' of h, per token
+      continue;
+    }
+    const int n = p.count[e], s0 = p.start[e];
+    for (int t0 = 0; t0 < n; t0 += tile) {
+      const int nt = min(tile, n - t0);
+      if (threadIdx.x < nt) {
+        const int a = p.list[s0 + t0 + threadIdx.x];
+        asg[threadIdx.x] = a;
+        const int Eh = xscale_exponent(__uint_as_float(__ldcg(&p.hamax[a])));
+        hexp[threadIdx.x] = Eh;
+        hk_sm[threadIdx.x] = acc_scale(Eh);
+      }
+      __syncthreads();
       for (int i = threadIdx.x; i < nt * I; i += kGThreads) {
         const int t = i / I, c = i - t * I;
-        const int Eh = xscale_exponent(__uint_as_float(hmax[t]));
-        hp_sm[t * I + (bits == 4 ? swz_q4(c) : swz_q2(c))] =
-            bits == 4 ? xprime_q4(h_sm[i], c, Eh) : xprime_q2(h_sm[i], c, Eh);
+        const float hv = __ldcg(p.h + (size_t)asg[t] * I + c);
+        hs_sm[t * I + (bits == 4 ? swz_q4(c) : swz_q2(c))] =
+            bits == 4 ? xprime_q4(hv, c, hexp[t]) : xprime_q2(hv, c, hexp[t]);
       }
       for (int i = warp; i < nt * (I / 32); i += kGWarps) {
         const int t = i / (I / 32), ch = i - t * (I / 32);
-        const float sm = warp_sum(h_sm[t * I + ch * 32 + lane]);
+        const float sm = warp_sum(__ldcg(p.h + (size_t)asg[t] * I + ch * 32 + lane));
         if (lane == 0) hsum_sm[i] = sm;
       }
-      if (threadIdx.x < nt) hk_sm[threadIdx.x] = acc_scale(xscale_exponent(__uint_as_float(hmax[threadIdx.x])));
       __syncthreads();
-      // ----------------------------------- down: kRowBlk-row blocks per warp
-      for (int r0 = warp * kRowBlk; r0 < H; r0 += kGWarps * kRowBlk) {
-        const int nv = H - r0 < kRowBlk ? H - r0 : kRowBlk;
-        for (int t = 0; t < nt; ++t) {
-          float ya[kRowBlk];
+      for (int r = r0 + 2 * warp; r < r1; r += 2 * kGWarps) {
+        const int two = r + 1 < r1 ? 2 : 1;
+        float v[2 * kTT];
 #pragma unroll
-          for (int i = 0; i < kRowBlk; ++i) ya[i] = 0.f;
-          if (bits == 4) block_rows<4>(ex.down, r0, nv, I, hp_sm + t * I, hsum_sm + t * (I / 32), hk_sm[t], ya, lane);
-          else block_rows<2>(ex.down, r0, nv, I, hp_sm + t * I, hsum_sm + t * (I / 32), hk_sm[t], ya, lane);
-          const float yv = warp_reduce_rows<kRowBlk>(ya, lane);
-          const int i = reduced_row_of_lane<kRowBlk>(lane);
-          if (lane == lane_of_reduced_row<kRowBlk>(i) && i < nv) p.y[(size_t)asg[t] * H + r0 + i] = yv;
-        }
+        for (int t = 0; t < 2 * kTT; ++t) v[t] = 0.f;
+        if (bits == 4) down_rows<4>(s_d, r, two, I, nt, hs_sm, hsum_sm, hk_sm, v, lane);
+        else down_rows<2>(s_d, r, two, I, nt, hs_sm, hsum_sm, hk_sm, v, lane);
+        const float sv = warp_reduce_rows<2 * kTT>(v, lane);
+        const int row = reduced_row_of_lane<2 * kTT>(lane);
+        const int q = row / kTT, t = row - q * kTT;
+        if (t < nt && q < two && lane == lane_of_reduced_row<2 * kTT>(row))
+          p.y[(size_t)asg[t] * H + r + q] = sv;
       }
       __syncthreads();
     }
   }
 }
 
-// Shared memory of the expert kernel for a token tile of `tile`.
-size_t grouped_smem_bytes(int H, int I, int tile) {
-  const size_t f = (size_t)al4(tile * H) + al4(tile * (H / 32)) + al4(tile) + 2 * (size_t)al4(tile * I) +
-                   al4(tile * (I / 32)) + al4(tile);
-  return 4 * (f + 3 * (size_t)al4(tile)) + 64;
+static size_t gateup_smem(int H, int tile) {
+  return 4 * ((size_t)al4(tile * H) + al4(tile * (H / 32)) + 3 * (size_t)al4(tile));
 }
 
-// Largest token tile (<= kTokTile) whose buffers fit in shared memory.
+static size_t down_smem(int I, int tile) {
+  return 4 * ((size_t)al4(tile * I) + al4(tile * (I / 32)) + 3 * (size_t)al4(tile));
+}
+
+// Largest token tile (<= kTT) whose buffers fit in shared memory.
 int grouped_tile(int H, int I, int smem_optin) {
-  for (int t = kTokTile; t >= 1; --t)
-    if (grouped_smem_bytes(H, I, t) <= (size_t)smem_optin) return t;
+  for (int t = kTT; t >= 1; --t)
+    if (gateup_smem(H, t) <= (size_t)smem_optin && down_smem(I, t) <= (size_t)smem_optin) return t;
   return 0;
 }
 
 cudaError_t launch_grouped(const GroupedParams& gp, cudaStream_t s) {
   const int A = gp.T * gp.K;
   if (A == 0) return cudaSuccess;
-  int* n_active = gp.grp_count + gp.E;  // the workspace reserves E+2 ints
-  int* work = n_active + 1;
-  const size_t gsm = sizeof(int) * 2 * (size_t)gp.E;
-  group_kernel<<<1, 1024, gsm, s>>>(gp.idx, A, gp.E, gp.grp_count, gp.grp_start, gp.grp_list, gp.grp_order,
-                                    n_active, gp.err);
-  cudaError_t e = cudaMemsetAsync(work, 0, sizeof(int), s);
+  int* ctl = gp.grp_count + gp.E;  // the workspace reserves E + 4 ints
+  group_kernel<<<1, 1024, 0, s>>>(gp.idx, A, gp.E, gp.grp_count, gp.grp_start, gp.grp_list, gp.grp_order, ctl,
+                                  gp.hamax, gp.err);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148, optin = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  cudaFuncAttributes fa{};
-  e = cudaFuncGetAttributes(&fa, grouped_expert_kernel);
-  if (e != cudaSuccess) return e;
-  optin -= (int)fa.sharedSizeBytes;  // static shared memory counts against the limit
-  ExpertParams p{};
+  cudaFuncAttributes fa{}, fb{};
+  if ((e = cudaFuncGetAttributes(&fa, grouped_gateup_kernel)) != cudaSuccess) return e;
+  if ((e = cudaFuncGetAttributes(&fb, grouped_down_kernel)) != cudaSuccess) return e;
+  // static shared memory counts against the per-block limit
+  const int avail = optin - (int)(fa.sharedSizeBytes > fb.sharedSizeBytes ? fa.sharedSizeBytes : fb.sharedSizeBytes);
+  GroupedKParams p{};
   p.H = gp.H; p.I = gp.I; p.K = gp.K; p.T = gp.T;
-  p.tile = grouped_tile(gp.H, gp.I, optin);
+  p.tile = grouped_tile(gp.H, gp.I, avail);
   if (p.tile == 0) return cudaErrorInvalidConfiguration;
   p.experts = gp.experts;
   p.xp4 = gp.xp4; p.xp2 = gp.xp2; p.xsum = gp.xsum; p.xexp = gp.xexp;
-  p.start = gp.grp_start; p.list = gp.grp_list; p.order = gp.grp_order; p.n_active = n_active; p.work = work;
-  p.y = gp.y; p.err = gp.err;
-  static int attr_done = 0;
-  if (!attr_done) {
-    e = cudaFuncSetAttribute(grouped_expert_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-    if (e != cudaSuccess) return e;
-    attr_done = 1;
+  p.count = gp.grp_count; p.start = gp.grp_start; p.list = gp.grp_list; p.order = gp.grp_order; p.ctl = ctl;
+  p.h = gp.h; p.hamax = gp.hamax; p.y = gp.y; p.err = gp.err;
+  static int attr_dev = -1;
+  if (attr_dev != dev) {
+    if ((e = cudaFuncSetAttribute(grouped_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, avail)) !=
+        cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(grouped_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, avail)) !=
+        cudaSuccess)
+      return e;
+    attr_dev = dev;
   }
-  grouped_expert_kernel<<<sms, kGThreads, grouped_smem_bytes(gp.H, gp.I, p.tile), s>>>(p);
+  grouped_gateup_kernel<<<sms, kGThreads, gateup_smem(gp.H, p.tile), s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  grouped_down_kernel<<<sms, kGThreads, down_smem(gp.I, p.tile), s>>>(p);
   return cudaGetLastError();
 }
 

@@ -45,7 +45,7 @@ struct WsLayout {
   size_t y;         // float  [T*K*H] expert outputs
   size_t idx;       // int32  [T*K]
   size_t w;         // float  [T*K]
-  size_t grp_count; // int    [E+2]  assignments per expert, active count, work counter
+  size_t grp_count; // int    [E+4]  assignments per expert, active count, two work counters
   size_t grp_start; // int    [E+1]
   size_t grp_list;  // int    [T*K]  assignment ids (t*K+k) sorted by expert
   size_t grp_order; // int    [E]    active experts, most tokens first
@@ -158,7 +158,7 @@ struct GroupedParams {
   int* hexp;
   unsigned* hamax;
   float* y;
-  int* grp_count;     // [E + 2]: counts, then active-expert count and work counter
+  int* grp_count;     // [E + 4]: counts, then active-expert count and two work counters
   int* grp_start;     // [E + 1]
   int* grp_list;      // [T*K]
   int* grp_order;     // [E]
