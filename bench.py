@@ -328,7 +328,7 @@ def run_ours(args, wl, rank, world, local_rank):
     chunk = 1024 if T == 1 else 8          # steps per captured graph
     n_chunks = 8 if T == 1 else 4
     n_tok = chunk * n_chunks * T
-    ls = LayerSetup(q, wl, seed, dev, n_tok, 10_000_000 * (rank + 1))
+    ls = LayerSetup(q, wl, seed, dev, n_tok, rank_token_base(10_000_000, rank))
     s = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
 
@@ -355,15 +355,10 @@ def run_ours(args, wl, rank, world, local_rank):
     if q.qe_workspace_status(ls.ws, s) != q.QE_OK:
         raise RuntimeError("device status after capture: " + q.qe_last_error())
 
-    def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
-
     with torch.cuda.stream(s):
         warm_graph.replay()
     s.synchronize()
-    barrier()
+    barrier(world)
     torch.cuda.synchronize()
     sampler = ClockSampler(local_rank) if rank == 0 else None
     if sampler:
@@ -381,17 +376,12 @@ def run_ours(args, wl, rank, world, local_rank):
         ev1.record(s)
     s.synchronize()
     torch.cuda.synchronize()
-    barrier()
+    barrier(world)
     clocks = sampler.stop() if sampler else None
     ms = ev0.elapsed_time(ev1)
     if q.qe_workspace_status(ls.ws, s) != q.QE_OK:
         raise RuntimeError("device status after timing: " + q.qe_last_error())
-    ms_max = ms
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_max = float(tt.item())
+    ms_max = sync_max(world, dev, ms)
     value = world * args.steps * T / (ms_max / 1000.0)
 
     # distinct experts touched per step (from the routing of the timed steps)
@@ -417,17 +407,12 @@ def run_ours(args, wl, rank, world, local_rank):
     with torch.cuda.stream(s):
         for i in range(4):
             e2e_step(i)
-    barrier()
+    barrier(world)
     t0 = time.perf_counter()
     with torch.cuda.stream(s):
         for i in range(n_e2e):
             e2e_step(i)
-    e2e_s = time.perf_counter() - t0
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_s = float(tt.item())
+    e2e_s = sync_max(world, dev, time.perf_counter() - t0)
     e2e_value = world * n_e2e * T / e2e_s
 
     if rank != 0:
@@ -463,6 +448,12 @@ def run_ours(args, wl, rank, world, local_rank):
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
+
+
+def rank_token_base(base, rank):
+    """First token id of a rank's token stream: replicas draw disjoint
+    token streams (each rank's stream holds fewer than 10^7 tokens)."""
+    return base * (rank + 1)
 
 
 def sync_max(world, dev, value):
@@ -539,7 +530,7 @@ def run_stack(args, wl, rank, world, local_rank):
     st = StackSetup(q, wl, args.seed, dev, L)
     ws = q.workspace(st.cfg, 1, device=dev)
     n_tok = 256
-    x = dev_tokens(args.seed, 20_000_000 * (rank + 1), n_tok, H, device=dev)
+    x = dev_tokens(args.seed, rank_token_base(20_000_000, rank), n_tok, H, device=dev)
     act = torch.empty((2, 1, H), dtype=torch.float32, device=dev)
     out = torch.empty((n_tok, H), dtype=torch.float32, device=dev)
     idx = torch.empty((n_tok, L, K), dtype=torch.int32, device=dev)
@@ -728,7 +719,7 @@ def run_tiered(args, wl, rank, world, local_rank):
     tier = q.Tier(cfg, cold_host, 2, int(wl["cache_gb"] * 1e9), max_tokens=1)
     ws = q.workspace(cfg, 1, device=dev)
     n_tok = args.warmup + args.steps
-    x = dev_tokens(args.seed, 30_000_000 * (rank + 1), n_tok, H, device=dev)
+    x = dev_tokens(args.seed, rank_token_base(30_000_000, rank), n_tok, H, device=dev)
     act = torch.empty((2, 1, H), dtype=torch.float32, device=dev)
     idx = torch.empty((n_tok, L, K), dtype=torch.int32, device=dev)
     s = torch.cuda.Stream(device=dev)
