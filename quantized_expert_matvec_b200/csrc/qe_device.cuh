@@ -123,7 +123,6 @@ QE_DEV void cp_async16(void* dst, const void* src, uint64_t pol) {
 QE_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 QE_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
 QE_DEV void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p)); }
 QE_DEV void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 
@@ -215,70 +214,86 @@ QE_DEV int lane_of_reduced_row(int row) {
 // word read as a float is the subnormal q * 2^(p-149), p = the field's bit
 // offset.  The activation is pre-scaled per column by 2^(89-p-E) (see
 // xprime_q4 / xprime_q2), so every product is exactly q*x*2^(-60-E) before
-// the single fp32 rounding of the fused multiply-add.  Two products go
-// through one packed f32x2 FMA.  Fields above bit 22 are first shifted down
-// by 12.  Per group the dot product is then
+// the single fp32 rounding of the fused multiply-add.  Per group the dot
+// product is then
 //   sum_c (q_c*s + b) x_c = s * 2^(60+E) * acc + b * sum_c x_c.
 // Subnormal operands and results must not be flushed: never build these
 // kernels with -ftz=true or --use_fast_math.
+//
+// Pair form.  Two adjacent packed words are one 64-bit value P (an aligned
+// register pair), and one 64-bit AND with the field mask repeated in both
+// halves yields the same field of both words: a ready operand pair of one
+// packed f32x2 FMA, with no register moves.  Fields that reach bit 23 or
+// above are taken from P >> 12, where they sit at bits 8..19 (a 64-bit
+// shift: the bits the high word pushes into the low half land at bit 20 and
+// above, where no mask of the shifted value looks).  The x'
+// of a 32-column chunk is therefore stored in pair order: pair k holds the
+// columns of field k of both words of a word pair (see xperm_q4 / xperm_q2).
 
-// Field offset p of column j (0..7) of a 4-bit word after the mapping above.
+// Field offset p of field j (0..7) of a 4-bit word after the mapping above.
 QE_DEV int q4_field_pos(int j) { return j < 5 ? 4 * j : 4 * j - 12; }
-// Field offset p of column j (0..15) of a 2-bit word.
+// Field offset p of field j (0..15) of a 2-bit word.
 QE_DEV int q2_field_pos(int j) { return j < 11 ? 2 * j : 2 * j - 12; }
 
 QE_DEV float f_of(uint32_t u) { return __uint_as_float(u); }
 
-// Eight 4-bit columns of one word against their x' (4 float2).
-QE_DEV float2 dot8_q4(const uint32_t v, const float2* x, float2 acc) {
-  const uint32_t hv = v >> 12;
-  acc = __ffma2_rn(make_float2(f_of(v & 0xFu), f_of(v & 0xF0u)), x[0], acc);
-  acc = __ffma2_rn(make_float2(f_of(v & 0xF00u), f_of(v & 0xF000u)), x[1], acc);
-  acc = __ffma2_rn(make_float2(f_of(v & 0xF0000u), f_of(hv & 0xF00u)), x[2], acc);
-  acc = __ffma2_rn(make_float2(f_of(hv & 0xF000u), f_of(hv & 0xF0000u)), x[3], acc);
-  return acc;
+QE_DEV float2 f2_of(unsigned long long v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
 }
 
-// Sixteen 2-bit columns of one word against their x' (8 float2).
-QE_DEV float2 dot16_q2(const uint32_t v, const float2* x, float2 acc) {
-  const uint32_t hv = v >> 12;
-  acc = __ffma2_rn(make_float2(f_of(v & 0x3u), f_of(v & 0xCu)), x[0], acc);
-  acc = __ffma2_rn(make_float2(f_of(v & 0x30u), f_of(v & 0xC0u)), x[1], acc);
-  acc = __ffma2_rn(make_float2(f_of(v & 0x300u), f_of(v & 0xC00u)), x[2], acc);
-  acc = __ffma2_rn(make_float2(f_of(v & 0x3000u), f_of(v & 0xC000u)), x[3], acc);
-  acc = __ffma2_rn(make_float2(f_of(v & 0x30000u), f_of(v & 0xC0000u)), x[4], acc);
-  acc = __ffma2_rn(make_float2(f_of(v & 0x300000u), f_of(hv & 0xC00u)), x[5], acc);
-  acc = __ffma2_rn(make_float2(f_of(hv & 0x3000u), f_of(hv & 0xC000u)), x[6], acc);
-  acc = __ffma2_rn(make_float2(f_of(hv & 0x30000u), f_of(hv & 0xC0000u)), x[7], acc);
-  return acc;
-}
+// acc += (P & M) * x as one packed FMA (P: two words, M: the mask in both halves).
+#define QE_QFMA2(acc, P, M, x) (acc) = __ffma2_rn(f2_of((P) & (M)), (x), (acc))
 
-// Two words of 2-bit weights (32 columns) against x' (16 float2).
-QE_DEV float2 dot32_q2(const uint2 w, const float2* xs, float2 acc) {
+QE_DEV constexpr unsigned long long rep2(unsigned m) { return ((unsigned long long)m << 32) | m; }
+
+// One 32-column chunk of 4-bit weights (words 0..3 as two 64-bit pairs)
+// against its 16 x' pairs; pair 8h + j holds columns 16h + j and 16h + 8 + j.
+// Two accumulators so consecutive FMAs do not wait on each other.
+QE_DEV float2 dot32_q4(const ulonglong2 w, const float2* xs, float2 acc) {
   float2 a2 = make_float2(0.f, 0.f);
-  acc = dot16_q2(w.x, xs, acc);
-  a2 = dot16_q2(w.y, xs + 8, a2);
+  const unsigned long long s0 = w.x >> 12, s1 = w.y >> 12;
+  QE_QFMA2(acc, w.x, rep2(0xFu), xs[0]);
+  QE_QFMA2(a2, w.y, rep2(0xFu), xs[8]);
+  QE_QFMA2(acc, w.x, rep2(0xF0u), xs[1]);
+  QE_QFMA2(a2, w.y, rep2(0xF0u), xs[9]);
+  QE_QFMA2(acc, w.x, rep2(0xF00u), xs[2]);
+  QE_QFMA2(a2, w.y, rep2(0xF00u), xs[10]);
+  QE_QFMA2(acc, w.x, rep2(0xF000u), xs[3]);
+  QE_QFMA2(a2, w.y, rep2(0xF000u), xs[11]);
+  QE_QFMA2(acc, w.x, rep2(0xF0000u), xs[4]);
+  QE_QFMA2(a2, w.y, rep2(0xF0000u), xs[12]);
+  QE_QFMA2(acc, s0, rep2(0xF00u), xs[5]);
+  QE_QFMA2(a2, s1, rep2(0xF00u), xs[13]);
+  QE_QFMA2(acc, s0, rep2(0xF000u), xs[6]);
+  QE_QFMA2(a2, s1, rep2(0xF000u), xs[14]);
+  QE_QFMA2(acc, s0, rep2(0xF0000u), xs[7]);
+  QE_QFMA2(a2, s1, rep2(0xF0000u), xs[15]);
   return make_float2(acc.x + a2.x, acc.y + a2.y);
 }
 
-// One uint4 of 4-bit weights (32 columns) against x' (16 float2); two
-// accumulators so consecutive FMAs do not wait on each other.
-QE_DEV float2 dot32_q4(const uint4 w, const float2* xs, float2 acc) {
+// One 32-column chunk of 2-bit weights (two words as one 64-bit pair)
+// against its 16 x' pairs; pair j holds columns j and 16 + j.
+QE_DEV float2 dot32_q2(const unsigned long long w, const float2* xs, float2 acc) {
   float2 a2 = make_float2(0.f, 0.f);
-  acc = dot8_q4(w.x, xs, acc);
-  a2 = dot8_q4(w.y, xs + 4, a2);
-  acc = dot8_q4(w.z, xs + 8, acc);
-  a2 = dot8_q4(w.w, xs + 12, a2);
-  return make_float2(acc.x + a2.x, acc.y + a2.y);
-}
-
-// One uint4 of 2-bit weights (64 columns, one group) against x' (32 float2).
-QE_DEV float2 dot64_q2(const uint4 w, const float2* xs, float2 acc) {
-  float2 a2 = make_float2(0.f, 0.f);
-  acc = dot16_q2(w.x, xs, acc);
-  a2 = dot16_q2(w.y, xs + 8, a2);
-  acc = dot16_q2(w.z, xs + 16, acc);
-  a2 = dot16_q2(w.w, xs + 24, a2);
+  const unsigned long long s = w >> 12;
+  QE_QFMA2(acc, w, rep2(0x3u), xs[0]);
+  QE_QFMA2(a2, w, rep2(0xCu), xs[1]);
+  QE_QFMA2(acc, w, rep2(0x30u), xs[2]);
+  QE_QFMA2(a2, w, rep2(0xC0u), xs[3]);
+  QE_QFMA2(acc, w, rep2(0x300u), xs[4]);
+  QE_QFMA2(a2, w, rep2(0xC00u), xs[5]);
+  QE_QFMA2(acc, w, rep2(0x3000u), xs[6]);
+  QE_QFMA2(a2, w, rep2(0xC000u), xs[7]);
+  QE_QFMA2(acc, w, rep2(0x30000u), xs[8]);
+  QE_QFMA2(a2, w, rep2(0xC0000u), xs[9]);
+  QE_QFMA2(acc, w, rep2(0x300000u), xs[10]);
+  QE_QFMA2(a2, s, rep2(0xC00u), xs[11]);
+  QE_QFMA2(acc, s, rep2(0x3000u), xs[12]);
+  QE_QFMA2(a2, s, rep2(0xC000u), xs[13]);
+  QE_QFMA2(acc, s, rep2(0x30000u), xs[14]);
+  QE_QFMA2(a2, s, rep2(0xC0000u), xs[15]);
   return make_float2(acc.x + a2.x, acc.y + a2.y);
 }
 
@@ -292,31 +307,38 @@ QE_DEV int xscale_exponent(float amax) {
   return E < -38 ? -38 : (E > 60 ? 60 : E);
 }
 
-// x' of column c for 4-bit / 2-bit matrices.
+// x' of column c for 4-bit / 2-bit matrices (c's field is c mod 8 / 16).
 QE_DEV float xprime_q4(float x, int c, int E) {
   return x * __int_as_float((127 + 89 - q4_field_pos(c & 7) - E) << 23);
 }
 QE_DEV float xprime_q2(float x, int c, int E) {
   return x * __int_as_float((127 + 89 - q2_field_pos(c & 15) - E) << 23);
 }
-// Shared-memory layout of x' in the fused kernel.  A lane reads the whole
-// uint4 chunk of columns it works on (32 columns for 4-bit, 64 for 2-bit) as
-// float4 pieces; stored linearly, the 32 lanes of a warp would hit the same
-// banks (chunks are 128 or 256 bytes apart).  Piece i of chunk ch is stored
-// at position i ^ (ch & 7), so lanes ch..ch+7 reading piece i touch eight
-// different 16-byte bank groups.
-QE_DEV int swz_q4(int c) {
-  const int ch = c >> 5;
-  return (ch << 5) | ((((c >> 2) & 7) ^ (ch & 7)) << 2) | (c & 3);
+
+// Position of column c in the pair order of its 32-column chunk.
+// 4-bit: column 16h + 8e + j -> 2(8h + j) + e; 2-bit: column 16e + j -> 2j + e.
+QE_DEV int xperm_q4(int c) {
+  const int m = c & 31;
+  return (c & ~31) | ((m >> 4) << 4) | ((m & 7) << 1) | ((m >> 3) & 1);
 }
-QE_DEV int swz_q2(int c) {
-  const int ch = c >> 6;
-  return (ch << 6) | ((((c >> 2) & 15) ^ (ch & 7)) << 2) | (c & 3);
+QE_DEV int xperm_q2(int c) {
+  const int m = c & 31;
+  return (c & ~31) | ((m & 15) << 1) | (m >> 4);
 }
 
-// The 32 x' values of columns [32*lc, 32*lc+32) from a swizzled buffer, as
-// 16 float2 (4-bit form: whole chunk lc; 2-bit form: half lc&1 of chunk lc/2).
-QE_DEV void load_xs32_q4(const float* xp, int lc, float2 (&xs)[16]) {
+// Shared-memory copies of x' also swizzle the eight 16-byte pieces of a
+// chunk: piece i of chunk ch sits at i ^ (ch & 7), so lanes reading piece i
+// of consecutive chunks touch eight different bank groups.  Global copies
+// keep the pair order unswizzled; a float4 piece moves as a whole.
+QE_DEV int xswz(int pos) {
+  const int ch = pos >> 5;
+  return (ch << 5) | ((((pos >> 2) & 7) ^ (ch & 7)) << 2) | (pos & 3);
+}
+QE_DEV int swz_q4(int c) { return xswz(xperm_q4(c)); }
+QE_DEV int swz_q2(int c) { return xswz(xperm_q2(c)); }
+
+// The 16 x' pairs of 32-column chunk lc from a swizzled buffer (either form).
+QE_DEV void load_xs32(const float* xp, int lc, float2 (&xs)[16]) {
   const float4* src = (const float4*)(xp + lc * 32);
   const int sw = lc & 7;
 #pragma unroll
@@ -326,17 +348,8 @@ QE_DEV void load_xs32_q4(const float* xp, int lc, float2 (&xs)[16]) {
     xs[2 * i + 1] = make_float2(v.z, v.w);
   }
 }
-QE_DEV void load_xs32_q2(const float* xp, int lc, float2 (&xs)[16]) {
-  const int ch = lc >> 1, half = lc & 1;
-  const float4* src = (const float4*)(xp + ch * 64);
-  const int sw = ch & 7;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 v = src[(half * 8 + i) ^ sw];
-    xs[2 * i] = make_float2(v.x, v.y);
-    xs[2 * i + 1] = make_float2(v.z, v.w);
-  }
-}
+QE_DEV void load_xs32_q4(const float* xp, int lc, float2 (&xs)[16]) { load_xs32(xp, lc, xs); }
+QE_DEV void load_xs32_q2(const float* xp, int lc, float2 (&xs)[16]) { load_xs32(xp, lc, xs); }
 
 // 2^(60+E): turns acc back into sum q*x.
 QE_DEV float acc_scale(int E) { return __int_as_float((127 + 60 + E) << 23); }

@@ -52,8 +52,8 @@ __global__ void __launch_bounds__(256) xprep_kernel(const float* __restrict__ sr
     const float val = x[c];
     const float s = warp_sum(val);
     if (lane == 0) xsum[(size_t)v * (n / 32) + ch] = s;
-    if (xp4) xp4[(size_t)v * n + c] = xprime_q4(val, c, E);
-    if (xp2) xp2[(size_t)v * n + c] = xprime_q2(val, c, E);
+    if (xp4) xp4[(size_t)v * n + xperm_q4(c)] = xprime_q4(val, c, E);
+    if (xp2) xp2[(size_t)v * n + xperm_q2(c)] = xprime_q2(val, c, E);
   }
 }
 
@@ -72,7 +72,8 @@ __global__ void __launch_bounds__(256) hprep_kernel(const FfnParams p) {
     const float v = h[c];
     const float s = warp_sum(v);
     if (lane == 0) p.hsum[(size_t)a * (I / 32) + ch] = s;
-    p.hp[(size_t)a * I + c] = bits == 4 ? xprime_q4(v, c, E) : xprime_q2(v, c, E);
+    if (bits == 4) p.hp[(size_t)a * I + xperm_q4(c)] = xprime_q4(v, c, E);
+    else p.hp[(size_t)a * I + xperm_q2(c)] = xprime_q2(v, c, E);
   }
 }
 
@@ -83,31 +84,31 @@ static __device__ __forceinline__ float rows_dot_global(const qe_qmat* mats, int
                                                         const float* __restrict__ xp,
                                                         const float* __restrict__ xs_sum, float xK,
                                                         int lane) {
-  constexpr int COLS = BITS == 4 ? 32 : 64;
-  const int nch = cols / COLS;
+  const int nch = cols / 32;  // 32-column chunks (4-bit: 4 words, 2-bit: 2 words)
   const int wpr = cols * BITS / 32;
   const int gpr = cols / kGroup;
   float yv[NM * R];
 #pragma unroll
   for (int i = 0; i < NM * R; ++i) yv[i] = 0.f;
   for (int ch = lane; ch < nch; ch += 32) {
-    float2 xs[COLS / 2];
-    const float4* src = (const float4*)(xp + ch * COLS);
+    float2 xs[16];
+    const float4* src = (const float4*)(xp + ch * 32);  // global x' in pair order
 #pragma unroll
-    for (int i = 0; i < COLS / 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
       const float4 v = __ldg(src + i);
       xs[2 * i] = make_float2(v.x, v.y);
       xs[2 * i + 1] = make_float2(v.z, v.w);
     }
-    const int g = BITS == 4 ? (ch >> 1) : ch;
-    const float xsum = BITS == 4 ? xs_sum[ch] : xs_sum[2 * ch] + xs_sum[2 * ch + 1];
+    const int g = ch >> 1;
+    const float xsum = xs_sum[ch];
 #pragma unroll
     for (int m = 0; m < NM; ++m) {
 #pragma unroll
       for (int rr = 0; rr < R; ++rr) {
         const size_t row = (size_t)(r0 + rr);
-        const uint4 w = __ldcs((const uint4*)(mats[m].wq + row * wpr) + ch);
-        const float2 a = BITS == 4 ? dot32_q4(w, xs, make_float2(0.f, 0.f)) : dot64_q2(w, xs, make_float2(0.f, 0.f));
+        float2 a;
+        if (BITS == 4) a = dot32_q4(__ldcs((const ulonglong2*)(mats[m].wq + row * wpr) + ch), xs, make_float2(0.f, 0.f));
+        else a = dot32_q2(__ldcs((const unsigned long long*)(mats[m].wq + row * wpr) + ch), xs, make_float2(0.f, 0.f));
         const float s = bf16f(__ldg(mats[m].scales + row * gpr + g));
         const float b = bf16f(__ldg(mats[m].biases + row * gpr + g));
         yv[m * R + rr] += s * xK * (a.x + a.y) + b * xsum;

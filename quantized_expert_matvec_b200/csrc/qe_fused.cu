@@ -179,10 +179,7 @@ static __device__ __forceinline__ float gateup_partial(const unsigned char* slot
   const int goff = c.qsc ? qd * (c.H / 256) : 0;
   for (int l = lane; l < c.nlc; l += 32) {
     const int lc = qd * c.nlc + l;  // 32-column chunk of the full row
-    if (!xs_cached) {
-      if (BITS == 4) load_xs32_q4(xp, lc, xs);
-      else load_xs32_q2(xp, lc, xs);
-    }
+    if (!xs_cached) load_xs32(xp, lc, xs);
     const int gi = (lc >> 1) - goff;
     const float xsum = xs_sum[lc];
 #pragma unroll
@@ -191,8 +188,8 @@ static __device__ __forceinline__ float gateup_partial(const unsigned char* slot
       for (int rr = 0; rr < kRB; ++rr) {
         const unsigned char* wp = slot + ((qd * 2 + m) * kRB + rr) * (c.H / 8);
         float2 a;
-        if (BITS == 4) a = dot32_q4(*(const uint4*)(wp + l * 16), xs, make_float2(0.f, 0.f));
-        else a = dot32_q2(*(const uint2*)(wp + l * 8), xs, make_float2(0.f, 0.f));
+        if (BITS == 4) a = dot32_q4(*(const ulonglong2*)(wp + l * 16), xs, make_float2(0.f, 0.f));
+        else a = dot32_q2(*(const unsigned long long*)(wp + l * 8), xs, make_float2(0.f, 0.f));
         const float sv = bf16f(sc[(2 * m) * segs + rr * c.srow + gi]);
         const float bv = bf16f(sc[(2 * m + 1) * segs + rr * c.srow + gi]);
         yv[m * kRB + rr] += sv * xK * (a.x + a.y) + bv * xsum;
@@ -209,8 +206,10 @@ static __device__ __forceinline__ float gateup_partial(const unsigned char* slot
 // of every row; the packed words and the scale/bias pair of that chunk are
 // loaded into registers (before h is ready, for the first chunk).
 struct DownRows {
-  uint4 w[8];       // 4-bit: one uint4; 2-bit: .x, .y
-  uint32_t sb[8];   // bf16 scale (low half) and bias (high half)
+  ulonglong2 w[8];  // 4-bit: words 0..3; 2-bit: words 0..1 in .x
+  // bf16 scale and bias, kept as loaded: combining them would make the warp
+  // wait for the loads here instead of at their first use after the h barrier
+  unsigned short sc[8], bi[8];
 };
 
 static __device__ __forceinline__ int down_row(int cta, int G, int RC, int wi, int nwk, int ri) {
@@ -228,14 +227,10 @@ static __device__ __forceinline__ void down_load(const qe_qmat& d, int cta, int 
     if (i < nr) {
       const int row = down_row(cta, G, RC, wi, nwk, b0 + i);
       const unsigned char* rp = (const unsigned char*)d.wq + (size_t)row * rowb;
-      if (d.bits == 4) {
-        R.w[i] = __ldcs((const uint4*)rp + lc);
-      } else {
-        const uint2 v = __ldcs((const uint2*)rp + lc);
-        R.w[i] = make_uint4(v.x, v.y, 0u, 0u);
-      }
-      R.sb[i] = (uint32_t)__ldg(d.scales + (size_t)row * gpr + g) |
-                ((uint32_t)__ldg(d.biases + (size_t)row * gpr + g) << 16);
+      if (d.bits == 4) R.w[i] = __ldcs((const ulonglong2*)rp + lc);
+      else R.w[i].x = __ldcs((const unsigned long long*)rp + lc);
+      R.sc[i] = __ldg(d.scales + (size_t)row * gpr + g);
+      R.bi[i] = __ldg(d.biases + (size_t)row * gpr + g);
     }
   }
 }
@@ -251,8 +246,8 @@ static __device__ __forceinline__ void down_accum(const DownRows& R, int nr, int
   for (int i = 0; i < 8; ++i) {
     if (i < nr) {
       const float2 a = BITS == 4 ? dot32_q4(R.w[i], xs, make_float2(0.f, 0.f))
-                                 : dot32_q2(make_uint2(R.w[i].x, R.w[i].y), xs, make_float2(0.f, 0.f));
-      yv[i] += bf16f(R.sb[i] & 0xFFFFu) * hK * (a.x + a.y) + bf16f(R.sb[i] >> 16) * xsum;
+                                 : dot32_q2(R.w[i].x, xs, make_float2(0.f, 0.f));
+      yv[i] += bf16f(R.sc[i]) * hK * (a.x + a.y) + bf16f(R.bi[i]) * xsum;
     }
   }
 }
@@ -540,16 +535,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
     float2 xs[16];
     int xs_bits = 0;  // bits of the x' form cached in xs (0: none)
     const bool cache = cx.nlc <= 32;  // one lane chunk of the quarter per lane
+    int slot_i = 0;
     for (int t = 0; t < ng; ++t) {
       int r0;
       const int k = item_k(t, &r0);
-      unsigned char* sl = gring + (size_t)(t % g.nslot) * g.slot;
+      unsigned char* sl = gring + (size_t)slot_i * g.slot;
       // copy groups committed after this item's: the items already issued ahead
       const int later = (t + g.nslot <= ng ? g.nslot : ng - t) - 1;
       if (later >= 2) cp_async_wait<2>();
       else if (later == 1) cp_async_wait<1>();
       else cp_async_wait<0>();
       __syncwarp();
+      if (threadIdx.x == 0 && t < 2) QE_TRACE(59 + 3 * t);  // item t landed (warp 0)
       const int bits = misc->ex[k].gate.bits;
       if (cache && xs_bits != bits && lane < cx.nlc) {
         if (bits == 4) load_xs32_q4(xp4, qd * cx.nlc + lane, xs);
@@ -562,7 +559,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
 #pragma unroll
       for (int i = 0; i < 2 * kRB; ++i)
         if (lane == lane_of_reduced_row<2 * kRB>(i)) red[i] = s;
+      if (threadIdx.x == 0 && t < 2) QE_TRACE(60 + 3 * t);  // item t computed (warp 0)
       named_barrier(1 + gr, 128);
+      if (threadIdx.x == 0 && t == 0) QE_TRACE(61);  // group 0 past item 0
       if (qd == 0 && lane < kRB) {
         // lane rr: h of row r0 + rr = silu(g) * u from the four quarter sums
         float gv = 0.f, uv = 0.f;
@@ -581,6 +580,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
         const int k1 = item_k(t + g.nslot, &r1);
         issue_gateup(misc->ex[k1], r1, sl, qd, cx, lane, pol);
       }
+      if (++slot_i == g.nslot) slot_i = 0;
       if (*abort_flag) break;
     }
     cp_async_wait<0>();  // nothing may still be landing when the CTA exits
@@ -601,12 +601,17 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
         set_error(&ctl->err, QE_ERR_TIMEOUT);
         misc->abort = 1;
       }
-      for (int k = 0; k < K; ++k) {
-        unsigned v;
-        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&ctl->hamax[k]) : "memory");
-        const int Eh = xscale_exponent(__uint_as_float(v));
-        misc->hK[k] = acc_scale(Eh);
-        misc->hamax[k] = (unsigned)Eh;  // reused: vector exponent of h_k
+      unsigned v[kMaxK];  // unrolled: registers, all loads in flight before the first use
+#pragma unroll
+      for (int k = 0; k < kMaxK; ++k)
+        if (k < K) asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v[k]) : "l"(&ctl->hamax[k]) : "memory");
+#pragma unroll
+      for (int k = 0; k < kMaxK; ++k) {
+        if (k < K) {
+          const int Eh = xscale_exponent(__uint_as_float(v[k]));
+          misc->hK[k] = acc_scale(Eh);
+          misc->hamax[k] = (unsigned)Eh;  // reused: vector exponent of h_k
+        }
       }
     }
     QE_TRACE(kTrHFirst);
@@ -615,23 +620,35 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
 
   // stage h in x' form, all warps: chunk ch of the K*I/32 chunks
   if (!*abort_flag) {
-    const int per = I / 32;
+    const int per = I / 32, nch = K * per;
+    // every CTA reads all of h at once: start each CTA at another chunk so
+    // the requests spread over the L2 slices instead of queueing on one
+    const int rot = (int)(((unsigned)cta * 37u) % (unsigned)nch);
     // 8 chunks per pass, loads issued before any of them is used
-    for (int ch0 = warp; ch0 < K * per; ch0 += 8 * kWarps) {
+    for (int ch0 = warp; ch0 < nch; ch0 += 8 * kWarps) {
       float v[8];
+      int kk[8], ll[8];  // chunk ch = k * per + lc, without a division per chunk
+      {
+        int ch = ch0 + rot < nch ? ch0 + rot : ch0 + rot - nch;
+        int k = 0;
+        while (ch >= per) { ch -= per; ++k; }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int ch = ch0 + i * kWarps;
-        if (ch < K * per) {
-          const int k = ch / per, lc = ch - k * per;
-          v[i] = __ldcg(p.hbuf + (size_t)k * I + lc * 32 + lane);
+        for (int i = 0; i < 8; ++i) {
+          kk[i] = k;
+          ll[i] = ch;
+          ch += kWarps;
+          while (ch >= per) { ch -= per; ++k; }
+          while (k >= K) k -= K;  // wrapped past the last expert (rotation)
         }
       }
 #pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (ch0 + i * kWarps < nch) v[i] = __ldcg(p.hbuf + (size_t)kk[i] * I + ll[i] * 32 + lane);
+#pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int ch = ch0 + i * kWarps;
-        if (ch < K * per) {
-          const int k = ch / per, lc = ch - k * per;
+        const int cr = ch0 + i * kWarps;
+        if (cr < nch) {
+          const int k = kk[i], lc = ll[i];
           const int c = lc * 32 + lane;
           const int Eh = (int)misc->hamax[k];
           const float sm = warp_sum(v[i]);

@@ -130,48 +130,59 @@ static __device__ __forceinline__ bool qmat_ok(const qe_qmat& m, int bits) {
   return m.bits == bits && m.wq && m.scales && m.biases && ((uintptr_t)m.wq & 15) == 0;
 }
 
-// Masked field pairs of one packed word (4-bit: 4 pairs, 2-bit: 8 pairs),
-// in the pair order of the x' layout (see dot8_q4 / dot16_q2).
+// Field pairs of sub-block b (0 or 1) of a 32-column chunk: 8 pairs, each
+// the same field of two packed words.  4-bit: b picks the word pair (words
+// 2b, 2b+1), fields 0..7; 2-bit: fields 8b..8b+7 of the chunk's one word
+// pair (in w.x).  Pair k of sub-block b multiplies x' pair 8b + k.
 template <int BITS>
-static __device__ __forceinline__ void mask_word(uint32_t v, float2 (&m)[BITS == 4 ? 4 : 8]) {
-  const uint32_t hv = v >> 12;
+static __device__ __forceinline__ void mask_sub(const ulonglong2 w, int b, float2 (&m)[8]) {
   if (BITS == 4) {
-    m[0] = make_float2(f_of(v & 0xFu), f_of(v & 0xF0u));
-    m[1] = make_float2(f_of(v & 0xF00u), f_of(v & 0xF000u));
-    m[2] = make_float2(f_of(v & 0xF0000u), f_of(hv & 0xF00u));
-    m[3] = make_float2(f_of(hv & 0xF000u), f_of(hv & 0xF0000u));
+    const unsigned long long P = b ? w.y : w.x, S = P >> 12;
+    m[0] = f2_of(P & rep2(0xFu));
+    m[1] = f2_of(P & rep2(0xF0u));
+    m[2] = f2_of(P & rep2(0xF00u));
+    m[3] = f2_of(P & rep2(0xF000u));
+    m[4] = f2_of(P & rep2(0xF0000u));
+    m[5] = f2_of(S & rep2(0xF00u));
+    m[6] = f2_of(S & rep2(0xF000u));
+    m[7] = f2_of(S & rep2(0xF0000u));
+  } else if (b == 0) {
+    const unsigned long long P = w.x;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m[j] = f2_of(P & rep2(3u << (2 * j)));
   } else {
-    m[0] = make_float2(f_of(v & 0x3u), f_of(v & 0xCu));
-    m[1] = make_float2(f_of(v & 0x30u), f_of(v & 0xC0u));
-    m[2] = make_float2(f_of(v & 0x300u), f_of(v & 0xC00u));
-    m[3] = make_float2(f_of(v & 0x3000u), f_of(v & 0xC000u));
-    m[4] = make_float2(f_of(v & 0x30000u), f_of(v & 0xC0000u));
-    m[5] = make_float2(f_of(v & 0x300000u), f_of(hv & 0xC00u));
-    m[6] = make_float2(f_of(hv & 0x3000u), f_of(hv & 0xC000u));
-    m[7] = make_float2(f_of(hv & 0x30000u), f_of(hv & 0xC0000u));
+    const unsigned long long P = w.x, S = P >> 12;
+    m[0] = f2_of(P & rep2(0x30000u));
+    m[1] = f2_of(P & rep2(0xC0000u));
+    m[2] = f2_of(P & rep2(0x300000u));
+    m[3] = f2_of(S & rep2(0xC00u));
+    m[4] = f2_of(S & rep2(0x3000u));
+    m[5] = f2_of(S & rep2(0xC000u));
+    m[6] = f2_of(S & rep2(0x30000u));
+    m[7] = f2_of(S & rep2(0xC0000u));
   }
 }
 
-// x' pairs of word j of lane chunk lc (32 columns) from a swizzled buffer.
-template <int BITS>
-static __device__ __forceinline__ void xs_word(const float* xp, int lc, int j, float2 (&x)[BITS == 4 ? 4 : 8]) {
-  if (BITS == 4) {
-    const float4* src = (const float4*)(xp + lc * 32);
-    const int sw = lc & 7;
-    const float4 a = src[(2 * j) ^ sw], b = src[(2 * j + 1) ^ sw];
-    x[0] = make_float2(a.x, a.y); x[1] = make_float2(a.z, a.w);
-    x[2] = make_float2(b.x, b.y); x[3] = make_float2(b.z, b.w);
-  } else {
-    const int ch = lc >> 1, hf = lc & 1;
-    const float4* src = (const float4*)(xp + ch * 64);
-    const int sw = ch & 7;
+// x' pairs 8b..8b+7 of 32-column chunk lc from a swizzled buffer.
+static __device__ __forceinline__ void xs_sub(const float* xp, int lc, int b, float2 (&x)[8]) {
+  const float4* src = (const float4*)(xp + lc * 32);
+  const int sw = lc & 7;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 a = src[(8 * hf + 4 * j + i) ^ sw];
-      x[2 * i] = make_float2(a.x, a.y);
-      x[2 * i + 1] = make_float2(a.z, a.w);
-    }
+  for (int i = 0; i < 4; ++i) {
+    const float4 a = src[(4 * b + i) ^ sw];
+    x[2 * i] = make_float2(a.x, a.y);
+    x[2 * i + 1] = make_float2(a.z, a.w);
   }
+}
+
+// Packed words of 32-column chunk lc of a row (4-bit: 4 words; 2-bit: 2 in .x).
+template <int BITS>
+static __device__ __forceinline__ ulonglong2 load_chunk(const unsigned char* row, int lc) {
+  if (BITS == 4) return __ldcs((const ulonglong2*)row + lc);
+  ulonglong2 w;
+  w.x = __ldcs((const unsigned long long*)row + lc);
+  w.y = 0ull;
+  return w;
 }
 
 // Stage x' (swizzled), 32-column sums and scale of nt tokens.
@@ -182,8 +193,7 @@ static __device__ void stage_x(const GroupedKParams& p, int bits, const int* tok
   for (int i = threadIdx.x; i < nt * (H / 4); i += kGThreads) {
     const int t = i / (H / 4), c = (i - t * (H / 4)) * 4;
     const float4 v = *(const float4*)(src + (size_t)toks[t] * H + c);
-    const int d = bits == 4 ? swz_q4(c) : swz_q2(c);  // 4 consecutive columns stay together
-    *(float4*)(xs_sm + t * H + d) = v;
+    *(float4*)(xs_sm + t * H + xswz(c)) = v;  // global x' is in pair order; pieces move whole
   }
   for (int i = threadIdx.x; i < nt * (H / 32); i += kGThreads) {
     const int t = i / (H / 32), c = i - t * (H / 32);
@@ -198,23 +208,12 @@ template <int BITS>
 static __device__ __forceinline__ void gateup_row(const qe_expert& ex, int r, int H, int nt, const float* xs_sm,
                                                   const float* sum_sm, const float* xk_sm, float (&v)[2 * kTT],
                                                   int lane) {
-  constexpr int NP = BITS == 4 ? 4 : 8;
-  constexpr int WPC = BITS == 4 ? 4 : 2;  // words per 32-column chunk
   const int gpr = H / kGroup;
   const size_t rowb = (size_t)H * BITS / 8;
   const unsigned char* gp = (const unsigned char*)ex.gate.wq + (size_t)r * rowb;
   const unsigned char* up = (const unsigned char*)ex.up.wq + (size_t)r * rowb;
   for (int lc = lane; lc < H / 32; lc += 32) {
-    uint32_t wg[WPC], wu[WPC];
-    if (BITS == 4) {
-      const uint4 a = __ldcs((const uint4*)gp + lc), b = __ldcs((const uint4*)up + lc);
-      wg[0] = a.x; wg[1] = a.y; wg[2 % WPC] = a.z; wg[3 % WPC] = a.w;
-      wu[0] = b.x; wu[1] = b.y; wu[2 % WPC] = b.z; wu[3 % WPC] = b.w;
-    } else {
-      const uint2 a = __ldcs((const uint2*)gp + lc), b = __ldcs((const uint2*)up + lc);
-      wg[0] = a.x; wg[1 % WPC] = a.y;
-      wu[0] = b.x; wu[1 % WPC] = b.y;
-    }
+    const ulonglong2 wg = load_chunk<BITS>(gp, lc), wu = load_chunk<BITS>(up, lc);
     const size_t gi = (size_t)r * gpr + (lc >> 1);
     const float sg = bf16f(__ldg(ex.gate.scales + gi)), bg = bf16f(__ldg(ex.gate.biases + gi));
     const float su = bf16f(__ldg(ex.up.scales + gi)), bu = bf16f(__ldg(ex.up.biases + gi));
@@ -222,17 +221,17 @@ static __device__ __forceinline__ void gateup_row(const qe_expert& ex, int r, in
 #pragma unroll
     for (int t = 0; t < kTT; ++t) { ga[t] = make_float2(0.f, 0.f); ua[t] = make_float2(0.f, 0.f); }
 #pragma unroll
-    for (int j = 0; j < WPC; ++j) {
-      float2 mg[NP], mu[NP];
-      mask_word<BITS>(wg[j], mg);
-      mask_word<BITS>(wu[j], mu);
+    for (int b = 0; b < 2; ++b) {
+      float2 mg[8], mu[8];
+      mask_sub<BITS>(wg, b, mg);
+      mask_sub<BITS>(wu, b, mu);
 #pragma unroll
       for (int t = 0; t < kTT; ++t) {
         if (t < nt) {
-          float2 xw[NP];
-          xs_word<BITS>(xs_sm + t * H, lc, j, xw);
+          float2 xw[8];
+          xs_sub(xs_sm + t * H, lc, b, xw);
 #pragma unroll
-          for (int i = 0; i < NP; ++i) {
+          for (int i = 0; i < 8; ++i) {
             ga[t] = __ffma2_rn(mg[i], xw[i], ga[t]);
             ua[t] = __ffma2_rn(mu[i], xw[i], ua[t]);
           }
@@ -328,24 +327,15 @@ template <int BITS>
 static __device__ __forceinline__ void down_rows(const qe_qmat& d, int r, int two, int I, int nt, const float* hs_sm,
                                                  const float* hsum_sm, const float* hk_sm, float (&v)[2 * kTT],
                                                  int lane) {
-  constexpr int NP = BITS == 4 ? 4 : 8;
-  constexpr int WPC = BITS == 4 ? 4 : 2;
   const int gpr = I / kGroup;
   const size_t rowb = (size_t)I * BITS / 8;
   for (int lc = lane; lc < I / 32; lc += 32) {
-    uint32_t w[2][WPC];
+    ulonglong2 w[2];
     float sc[2], bi[2];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int rr = r + (q < two ? q : 0);
-      const unsigned char* rp = (const unsigned char*)d.wq + (size_t)rr * rowb;
-      if (BITS == 4) {
-        const uint4 a = __ldcs((const uint4*)rp + lc);
-        w[q][0] = a.x; w[q][1] = a.y; w[q][2 % WPC] = a.z; w[q][3 % WPC] = a.w;
-      } else {
-        const uint2 a = __ldcs((const uint2*)rp + lc);
-        w[q][0] = a.x; w[q][1 % WPC] = a.y;
-      }
+      w[q] = load_chunk<BITS>((const unsigned char*)d.wq + (size_t)rr * rowb, lc);
       const size_t gi = (size_t)rr * gpr + (lc >> 1);
       sc[q] = bf16f(__ldg(d.scales + gi));
       bi[q] = bf16f(__ldg(d.biases + gi));
@@ -354,17 +344,17 @@ static __device__ __forceinline__ void down_rows(const qe_qmat& d, int r, int tw
 #pragma unroll
     for (int t = 0; t < kTT; ++t) { acc[0][t] = make_float2(0.f, 0.f); acc[1][t] = make_float2(0.f, 0.f); }
 #pragma unroll
-    for (int j = 0; j < WPC; ++j) {
-      float2 m0[NP], m1[NP];
-      mask_word<BITS>(w[0][j], m0);
-      mask_word<BITS>(w[1][j], m1);
+    for (int b = 0; b < 2; ++b) {
+      float2 m0[8], m1[8];
+      mask_sub<BITS>(w[0], b, m0);
+      mask_sub<BITS>(w[1], b, m1);
 #pragma unroll
       for (int t = 0; t < kTT; ++t) {
         if (t < nt) {
-          float2 xw[NP];
-          xs_word<BITS>(hs_sm + t * I, lc, j, xw);
+          float2 xw[8];
+          xs_sub(hs_sm + t * I, lc, b, xw);
 #pragma unroll
-          for (int i = 0; i < NP; ++i) {
+          for (int i = 0; i < 8; ++i) {
             acc[0][t] = __ffma2_rn(m0[i], xw[i], acc[0][t]);
             acc[1][t] = __ffma2_rn(m1[i], xw[i], acc[1][t]);
           }

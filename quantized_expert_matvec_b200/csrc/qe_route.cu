@@ -60,8 +60,8 @@ __global__ void __launch_bounds__(256) route_norm_kernel(const RouteParams p) {
     const float v = (float)(ldx(c) * rinv * (p.gamma ? (double)p.gamma[c] : 1.0));
     const float s = warp_sum(v);
     if (lane == 0) p.xsum[(size_t)t * (H / 32) + ch] = s;
-    p.xp4[(size_t)t * H + c] = xprime_q4(v, c, Ex);
-    p.xp2[(size_t)t * H + c] = xprime_q2(v, c, Ex);
+    p.xp4[(size_t)t * H + xperm_q4(c)] = xprime_q4(v, c, Ex);
+    p.xp2[(size_t)t * H + xperm_q2(c)] = xprime_q2(v, c, Ex);
   }
 }
 
