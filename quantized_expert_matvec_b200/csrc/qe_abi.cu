@@ -65,10 +65,11 @@ WsLayout ws_layout(int H, int E, int K, int I, int T) {
   L.y = take(4 * t * K * H);
   L.idx = take(4 * t * K);
   L.w = take(4 * t * K);
-  L.grp_count = take(4 * ((size_t)E + 4));
+  L.grp_count = take(4 * ((size_t)E + 8));
   L.grp_start = take(4 * ((size_t)E + 1));
   L.grp_list = take(4 * t * K);
   L.grp_order = take(4 * (size_t)E);
+  L.xh = take(2 * t * H);
   L.total = off;
   return L;
 }
@@ -134,6 +135,7 @@ int route_impl(const qe_cfg* c, const void* x, int x_dtype, const float* gamma, 
   if (want_xprime) {
     p.xp4 = at<float>(ws, L.xp4); p.xp2 = at<float>(ws, L.xp2); p.xsum = at<float>(ws, L.xsum);
     p.xexp = at<int>(ws, L.xexp);
+    p.xh = at<uint16_t>(ws, L.xh);
   }
   p.err = &at<WsControl>(ws, L.control)->err;
   cudaError_t e = launch_route(p, s);
@@ -357,6 +359,8 @@ int experts_and_combine(const qe_cfg* c, const qe_expert* experts, const int32_t
     gp.xp4 = at<float>(ws, L.xp4); gp.xp2 = at<float>(ws, L.xp2); gp.xsum = at<float>(ws, L.xsum);
     gp.xexp = at<int>(ws, L.xexp);
     gp.h = at<float>(ws, L.h); gp.hamax = at<unsigned>(ws, L.hamax);
+    gp.xh = at<uint16_t>(ws, L.xh);
+    gp.budget_ns = g_budget_ns;
     gp.y = at<float>(ws, L.y);
     gp.grp_count = at<int>(ws, L.grp_count); gp.grp_start = at<int>(ws, L.grp_start);
     gp.grp_list = at<int>(ws, L.grp_list); gp.grp_order = at<int>(ws, L.grp_order);

@@ -27,6 +27,7 @@ constexpr int kGThreads = kGWarps * 32;
 constexpr int kTT = 8;       // tokens sharing one pass over the weights
 constexpr int kRowsA = 128;  // gate/up rows (of gate and of up) per item
 constexpr int kRowsB = 512;  // down rows per item
+constexpr bool kTcEnabled = false;  // see launch_grouped
 
 // Round a count of 4-byte elements up to a multiple of 4 (16 bytes).
 static __host__ __device__ __forceinline__ int al4(int n) { return (n + 3) & ~3; }
@@ -36,14 +37,16 @@ static __host__ __device__ __forceinline__ int al4(int n) { return (n + 3) & ~3;
 // maxima and the two work counters of the expert kernels.
 __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__ idx, int A, int E, int* count,
                                                      int* start, int* list, int* order, int* ctl,
-                                                     unsigned* hamax, int* err) {
+                                                     unsigned* hamax, int tc_min, int* err) {
   __shared__ int cnt[kMaxE];
   __shared__ int cur[kMaxE];
   __shared__ int wsum[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
   for (int a = tid; a < A; a += blockDim.x) hamax[a] = 0u;
-  if (tid < 4) ctl[tid] = 0;  // [0] active experts, [1] gate/up work, [2] down work
+  // [0] active experts, [1] gate/up work, [2] down work, [3] experts with at
+  // least tc_min tokens (tensor-core gate/up; they lead `order`), [4] its work
+  if (tid < 8) ctl[tid] = 0;
   __syncthreads();
   for (int a = tid; a < A; a += blockDim.x) {
     const int e = idx[a];
@@ -85,6 +88,7 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__
       }
       order[rank] = tid;
       atomicAdd(&ctl[0], 1);
+      if (tc_min > 0 && c >= tc_min) atomicAdd(&ctl[3], 1);
     }
   }
   if (tid == 0) start[E] = wsum[31];
@@ -285,13 +289,14 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_gateup_kernel(const Grou
   __shared__ int s_item;
   __shared__ qe_expert s_ex;
   const int ipe = (I + kRowsA - 1) / kRowsA;
-  const int n_items = p.ctl[0] * ipe;
+  const int n_tc = p.ctl[3];  // experts done by the tensor-core kernel
+  const int n_items = (p.ctl[0] - n_tc) * ipe;
   for (;;) {
     if (threadIdx.x == 0) s_item = atomicAdd(&p.ctl[1], 1);
     __syncthreads();
     const int item = s_item;
     if (item >= n_items) break;
-    const int e = p.order[item / ipe];
+    const int e = p.order[n_tc + item / ipe];
     const int r0 = (item % ipe) * kRowsA, r1 = min(I, r0 + kRowsA);
     if (threadIdx.x == 0) s_ex = p.experts[e];
     __syncthreads();
@@ -459,11 +464,16 @@ int grouped_tile(int H, int I, int smem_optin) {
 cudaError_t launch_grouped(const GroupedParams& gp, cudaStream_t s) {
   const int A = gp.T * gp.K;
   if (A == 0) return cudaSuccess;
-  int* ctl = gp.grp_count + gp.E;  // the workspace reserves E + 4 ints
+  int* ctl = gp.grp_count + gp.E;  // the workspace reserves E + 8 ints
+  // The tensor-core gate/up kernel (qe_tc.cu) is not launched: at hidden 4096
+  // with 2-bit experts it stopped with an illegal instruction whose cause is
+  // not found yet, so groups of every size take the CUDA-core path.
+  const bool tc = kTcEnabled && tc_eligible(gp.H, gp.I) && gp.xh != nullptr;
   group_kernel<<<1, 1024, 0, s>>>(gp.idx, A, gp.E, gp.grp_count, gp.grp_start, gp.grp_list, gp.grp_order, ctl,
-                                  gp.hamax, gp.err);
+                                  gp.hamax, tc ? tc_min_tokens() : 0, gp.err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (tc && (e = launch_tc_gateup(gp, ctl, gp.budget_ns, s)) != cudaSuccess) return e;
   int dev = 0, sms = 148, optin = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

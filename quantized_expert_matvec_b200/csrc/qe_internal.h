@@ -45,10 +45,11 @@ struct WsLayout {
   size_t y;         // float  [T*K*H] expert outputs
   size_t idx;       // int32  [T*K]
   size_t w;         // float  [T*K]
-  size_t grp_count; // int    [E+4]  assignments per expert, active count, two work counters
+  size_t grp_count; // int    [E+8]  assignments per expert, then the grouping control words
   size_t grp_start; // int    [E+1]
   size_t grp_list;  // int    [T*K]  assignment ids (t*K+k) sorted by expert
   size_t grp_order; // int    [E]    active experts, most tokens first
+  size_t xh;        // fp16   [T*H]  xn for the tensor-core gate/up
   size_t total;
 };
 
@@ -111,6 +112,7 @@ struct RouteParams {
   double* xg;
   double* logits;
   float* xn_ws;     // normalised activations kept for the expert path (may be null)
+  uint16_t* xh;     // xn as fp16 bits [T][H] for the tensor-core path (may be null)
   float* xp4;       // may be null
   float* xp2;
   float* xsum;
@@ -158,17 +160,23 @@ struct GroupedParams {
   int* hexp;
   unsigned* hamax;
   float* y;
-  int* grp_count;     // [E + 4]: counts, then active-expert count and two work counters
+  int* grp_count;     // [E + 8]: counts, then the grouping control words
   int* grp_start;     // [E + 1]
   int* grp_list;      // [T*K]
   int* grp_order;     // [E]
+  const uint16_t* xh; // [T][H] fp16 bits of xn (tensor-core gate/up)
   const void* x;     // residual source
   int x_bf16;
   int add_residual;
   float* out;
   int* err;
+  unsigned long long budget_ns;  // bounded waits of the tensor-core kernel
 };
 cudaError_t launch_grouped(const GroupedParams& p, cudaStream_t s);
+// Tensor-core gate/up for experts with at least tc_min_tokens() tokens.
+bool tc_eligible(int H, int I);
+int tc_min_tokens();
+cudaError_t launch_tc_gateup(const GroupedParams& gp, int* ctl, unsigned long long budget_ns, cudaStream_t s);
 int grouped_tile(int H, int I, int smem_optin);
 
 

@@ -1,6 +1,7 @@
 // qe_route.cu -- RMSNorm + router + top-K for T tokens (moe_route and the
 // batched layer step).  Norm and router logits are evaluated in double
 // precision so the expert choice is an fp64 decision.
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "qe_device.cuh"
@@ -41,6 +42,7 @@ __global__ void __launch_bounds__(256) route_norm_kernel(const RouteParams p) {
     const float xn = (float)(xv * rinv * gm);
     if (p.xn_out) p.xn_out[(size_t)t * H + c] = xn;
     if (p.xn_ws) p.xn_ws[(size_t)t * H + c] = xn;
+    if (p.xh) p.xh[(size_t)t * H + c] = __half_as_ushort(__float2half_rn(xn));
     amax = fmaxf(amax, fabsf(xn));
   }
   if (!p.xp4) return;

@@ -417,3 +417,33 @@ def test_batched_c4_full_step_sampled(q, c1_layer):
     out_h, idx_h, w_h = out.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy()
     for t in (0, 100, 255):
         check(dl, out_h[t], idx_h[t], w_h[t], dl.oracle(host_x_f64(0, 50000 + t, 4096, bf16=True)))
+
+
+def test_batched_tensor_core_groups_full_shape(q):
+    """Hidden 4096, intermediate 1024: a +8 logit offset on four experts (two
+    4-bit, two 2-bit) sends all 150 tokens to them: groups far above the
+    8-token pass of the grouped kernels; sampled tokens against the oracle."""
+    import torch
+    cfg = q.Cfg(4096, 64, 4, 1024)
+    off = np.zeros(64, np.float32)
+    hot = [3, 10, 21, 40]
+    off[hot] = 8.0
+    dl = DevLayer(q, cfg, seed=31, layer=0, bits_of=lambda e: 2 if e % 2 else 4, offset=off)
+    T = 150
+    x = dev_tokens(31, 7000, T, 4096, bf16=True)
+    ws = q.workspace(cfg, T)
+    out = torch.empty((T, 4096), dtype=torch.float32, device="cuda")
+    idx = torch.empty((T, 4), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, 4), dtype=torch.float32, device="cuda")
+    q.moe_layer_step(cfg, dl.layer_struct, x, out, True, idx, w, ws)
+    assert q.qe_workspace_status(ws) == q.QE_OK, q.qe_last_error()
+    ih = idx.cpu().numpy()
+    assert all(sorted(r) == hot for r in ih.tolist())
+    oh = out.cpu().numpy()
+    xb = x.cpu().view(torch.int16).numpy().astype(np.uint16)
+    for t in (0, 77, 128, 149):
+        x64 = (xb[t].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        ref = dl.oracle(x64, residual=True)
+        assert list(ih[t]) == list(ref["idx"])
+        err = normwise_err(oh[t], ref["out"])
+        assert err <= TOL, (t, err)
