@@ -47,7 +47,6 @@ QE_DEV bool wait_geq(const unsigned* ctr, unsigned target, uint64_t deadline,
   while (ld_acquire(ctr) < target) {
     if (*abort_flag) return false;
     if ((++spins & 15u) == 0 && gtimer() > deadline) return false;
-    __nanosleep(32);
   }
   return true;
 }
@@ -184,6 +183,30 @@ QE_DEV float warp_reduce_rows(float (&v)[R], int lane) {
   }
   float s = v[0];
   for (; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
+// Same as warp_reduce_rows with max instead of sum.
+template <int R>
+QE_DEV float warp_reduce_rows_max(float (&v)[R], int lane) {
+  int live = R;
+  int o = 16;
+#pragma unroll
+  for (; live > 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+    const int half = live / 2;
+#pragma unroll
+    for (int i = 0; i < R / 2; ++i) {
+      if (i < half) {
+        float keep = up ? v[i + half] : v[i];
+        float send = up ? v[i] : v[i + half];
+        v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+      }
+    }
+    live = half;
+  }
+  float s = v[0];
+  for (; o > 0; o >>= 1) s = fmaxf(s, __shfl_xor_sync(0xffffffffu, s, o));
   return s;
 }
 

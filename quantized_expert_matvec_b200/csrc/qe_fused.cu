@@ -47,8 +47,7 @@ struct FusedMisc {
   float wk[kMaxK];
   qe_expert ex[kMaxK];
   float hK[kMaxK];
-  unsigned claim[kMaxK];
-  int hflag[kMaxK];
+  int hexp[kMaxK];  // vector exponent of h_k (x' form of the down input)
   unsigned cand_idx[kWarps][kMaxK];
   unsigned long long cand_key[kWarps][kMaxK];
   double cand_val[kWarps][kMaxK];
@@ -277,8 +276,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
     if (p.trace) p.trace[(size_t)cta * 64 + 12] = clock64();
   }
   if (tid < kMaxK) {
-    misc->claim[tid] = 0;
-    misc->hflag[tid] = 0;
+    misc->hexp[tid] = 0;
   }
 
   // ------------------------------------------------------------- routing
@@ -376,23 +374,29 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   __syncthreads();
   if (tid == 0) {
     QE_TRACE(kTrRouterDone);
-    if (!given) {
-      __threadfence();
-      if (cta != p.skip_cta) atomicAdd(&ctl->route_ctr, 1u);
-    }
+    if (!given && cta != p.skip_cta) red_release_add(&ctl->route_ctr, 1u);  // publishes this CTA's logits
   }
   {
     float m = 0.f;
     for (int w = 0; w < kWarps; ++w) m = fmaxf(m, misc->redf[w]);
     const int Ex = xscale_exponent(m);
     if (tid == 0) misc->xK = acc_scale(Ex);
+    {
+      // the chunk sums of this warp's kChunkMax chunks in one transposed
+      // reduction (chunks past the end hold 0)
+      float sv[kChunkMax];
+#pragma unroll
+      for (int q = 0; q < kChunkMax; ++q) sv[q] = xnv[q];
+      const float sm = warp_reduce_rows<kChunkMax>(sv, lane);
+      const int row = reduced_row_of_lane<kChunkMax>(lane);
+      const int ch = warp + kWarps * row;
+      if (lane == lane_of_reduced_row<kChunkMax>(row) && ch < H / 32) xsum[ch] = sm;
+    }
 #pragma unroll
     for (int q = 0; q < kChunkMax; ++q) {
       const int ch = warp + kWarps * q;
       if (ch < H / 32) {
         const int c = ch * 32 + lane;
-        const float sm = warp_sum(xnv[q]);
-        if (lane == 0) xsum[ch] = sm;
         xp4[swz_q4(c)] = xprime_q4(xnv[q], c, Ex);
         xp2[swz_q2(c)] = xprime_q2(xnv[q], c, Ex);
       }
@@ -572,7 +576,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
         }
         const float hv = gv / (1.0f + expf(-gv)) * uv;
         p.hbuf[(size_t)k * I + r0 + lane] = hv;  // published once per CTA below
-        atomicMax(&misc->hamax[k], __float_as_uint(fabsf(hv)));
       }
       __syncwarp();
       if (t + g.nslot < ng) {
@@ -594,69 +597,106 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   if (tid == 0) {
     QE_TRACE(kTrLastB);
     if (!*abort_flag) {
-      for (int k = 0; k < K; ++k) atomicMax(&ctl->hamax[k], misc->hamax[k]);
-      __threadfence();
-      atomicAdd(&ctl->h_ctr, 1u);
+      // the release publishes the h rows every thread of this CTA stored
+      // before the barrier above
+      red_release_add(&ctl->h_ctr, 1u);
       if (!wait_geq(&ctl->h_ctr, (unsigned)G, deadline, abort_flag)) {
         set_error(&ctl->err, QE_ERR_TIMEOUT);
         misc->abort = 1;
-      }
-      unsigned v[kMaxK];  // unrolled: registers, all loads in flight before the first use
-#pragma unroll
-      for (int k = 0; k < kMaxK; ++k)
-        if (k < K) asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v[k]) : "l"(&ctl->hamax[k]) : "memory");
-#pragma unroll
-      for (int k = 0; k < kMaxK; ++k) {
-        if (k < K) {
-          const int Eh = xscale_exponent(__uint_as_float(v[k]));
-          misc->hK[k] = acc_scale(Eh);
-          misc->hamax[k] = (unsigned)Eh;  // reused: vector exponent of h_k
-        }
       }
     }
     QE_TRACE(kTrHFirst);
   }
   __syncthreads();
 
-  // stage h in x' form, all warps: chunk ch of the K*I/32 chunks
-  if (!*abort_flag) {
-    const int per = I / 32, nch = K * per;
-    // every CTA reads all of h at once: start each CTA at another chunk so
-    // the requests spread over the L2 slices instead of queueing on one
-    const int rot = (int)(((unsigned)cta * 37u) % (unsigned)nch);
-    // 8 chunks per pass, loads issued before any of them is used
-    for (int ch0 = warp; ch0 < nch; ch0 += 8 * kWarps) {
-      float v[8];
-      int kk[8], ll[8];  // chunk ch = k * per + lc, without a division per chunk
-      {
-        int ch = ch0 + rot < nch ? ch0 + rot : ch0 + rot - nch;
-        int k = 0;
-        while (ch >= per) { ch -= per; ++k; }
+  // stage h in x' form, all warps: chunk ch of the K*I/32 chunks.  Every CTA
+  // loads all of h, so it finds max |h_k| itself (per-warp maxima, then one
+  // pass over the warps).  When the chunks fit in one round of 8 per warp the
+  // values stay in registers until their exponent is known; otherwise the raw
+  // values go through shared memory and are rewritten in x' form in place
+  // (the x' layout only permutes values inside a chunk).
+  const int per = I / 32, nch = K * per;
+  // every CTA reads all of h at once: start each CTA at another chunk so the
+  // requests spread over the L2 slices instead of queueing on one
+  const int rot = (int)(((unsigned)cta * 37u) % (unsigned)nch);
+  // (k, lc) of the 8 chunks of the round of this warp that starts at ch0
+  auto round_chunks = [&](int ch0, int (&kk)[8], int (&ll)[8]) {
+    int ch = ch0 + rot < nch ? ch0 + rot : ch0 + rot - nch;
+    int k = 0;
+    while (ch >= per) { ch -= per; ++k; }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          kk[i] = k;
-          ll[i] = ch;
-          ch += kWarps;
-          while (ch >= per) { ch -= per; ++k; }
-          while (k >= K) k -= K;  // wrapped past the last expert (rotation)
-        }
-      }
+    for (int i = 0; i < 8; ++i) {
+      kk[i] = k;
+      ll[i] = ch;
+      ch += kWarps;
+      while (ch >= per) { ch -= per; ++k; }
+      while (k >= K) k -= K;  // wrapped past the last expert (rotation)
+    }
+  };
+  const bool one_round = nch <= 8 * kWarps;
+  float v[8];  // one round: the values stay here until their exponent is known
+  if (!*abort_flag) {
+    for (int ch0 = warp; ch0 < nch; ch0 += 8 * kWarps) {
+      int kk[8], ll[8];
+      round_chunks(ch0, kk, ll);
+      // loads issued before any of them is used
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         if (ch0 + i * kWarps < nch) v[i] = __ldcg(p.hbuf + (size_t)kk[i] * I + ll[i] * 32 + lane);
+      // the 8 chunks' sums and maxima in one transposed reduction each
+      // (chunks past the end hold 0, which changes neither)
+      float sv[8], mv[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int cr = ch0 + i * kWarps;
-        if (cr < nch) {
-          const int k = kk[i], lc = ll[i];
-          const int c = lc * 32 + lane;
-          const int Eh = (int)misc->hamax[k];
-          const float sm = warp_sum(v[i]);
-          if (lane == 0) hsum[(size_t)k * per + lc] = sm;
+        if (ch0 + i * kWarps >= nch) v[i] = 0.f;
+        sv[i] = v[i];
+        mv[i] = fabsf(v[i]);
+        if (!one_round && ch0 + i * kWarps < nch) hp[(size_t)kk[i] * I + ll[i] * 32 + lane] = v[i];
+      }
+      const float sm = warp_reduce_rows<8>(sv, lane);
+      const float am = warp_reduce_rows_max<8>(mv, lane);
+      const int row = reduced_row_of_lane<8>(lane);
+      if (lane == lane_of_reduced_row<8>(row) && ch0 + row * kWarps < nch) {
+        int k = 0, lc = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (i == row) { k = kk[i]; lc = ll[i]; }
+        hsum[(size_t)k * per + lc] = sm;
+        atomicMax(&misc->hamax[k], __float_as_uint(am));
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < K) {
+    const int Eh = xscale_exponent(__uint_as_float(misc->hamax[tid]));
+    misc->hexp[tid] = Eh;
+    misc->hK[tid] = acc_scale(Eh);
+  }
+  __syncthreads();
+  if (!*abort_flag) {
+    if (one_round) {
+      int kk[8], ll[8];
+      round_chunks(warp, kk, ll);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (warp + i * kWarps < nch) {
+          const int k = kk[i], c = ll[i] * 32 + lane;
           float* hpk = hp + (size_t)k * I;
-          if (misc->ex[k].down.bits == 4) hpk[swz_q4(c)] = xprime_q4(v[i], c, Eh);
-          else hpk[swz_q2(c)] = xprime_q2(v[i], c, Eh);
+          if (misc->ex[k].down.bits == 4) hpk[swz_q4(c)] = xprime_q4(v[i], c, misc->hexp[k]);
+          else hpk[swz_q2(c)] = xprime_q2(v[i], c, misc->hexp[k]);
         }
+      }
+    } else {
+      // raw values went through shared memory: rewrite each chunk in place
+      for (int ch = warp; ch < nch; ch += kWarps) {
+        int k = 0, lc = ch;
+        while (lc >= per) { lc -= per; ++k; }
+        float* hpk = hp + (size_t)k * I;
+        const int c = lc * 32 + lane;
+        const float x = hpk[c];
+        __syncwarp();
+        if (misc->ex[k].down.bits == 4) hpk[swz_q4(c)] = xprime_q4(x, c, misc->hexp[k]);
+        else hpk[swz_q2(c)] = xprime_q2(x, c, misc->hexp[k]);
       }
     }
   }
