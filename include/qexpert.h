@@ -213,6 +213,15 @@ QE_API int moe_layer_step(const qe_cfg* cfg, const qe_layer* layer, const void* 
                    float* out, int add_residual, int32_t* topk_idx, float* topk_w, void* dev_ws,
                    size_t ws_bytes, qe_stream_t stream);
 
+/* moe_layer_step on host buffers: x_host [T,H] (fp32 or bf16 bits, page-
+ * locked for the copy to run asynchronously) is copied into the workspace,
+ * the layer step runs on `stream` (the fused kernel for T == 1, the batched
+ * path otherwise), the result is copied to out_host [T,H] fp32, and the call
+ * returns after synchronising `stream`.  Routing is not returned.  The
+ * workspace is the one qe_workspace_bytes(cfg, T) sizes. */
+QE_API int moe_layer_step_host(const qe_cfg* cfg, const qe_layer* layer, const void* x_host, int x_dtype, int T,
+                               float* out_host, int add_residual, void* dev_ws, size_t ws_bytes, qe_stream_t stream);
+
 /* The single-token layer step of moe_layer_step (T == 1, fused kernel) for
  * callers that cannot allocate device memory: a plugin whose host engine
  * hands it only input and output buffers, or code running beside an

@@ -28,7 +28,7 @@ __all__ = [
     "qe_last_error", "qe_version", "qe_expert_bytes", "qe_pool_table", "qe_workspace_bytes",
     "qe_workspace_init", "qe_workspace_status", "qe_set_wait_budget_ns", "qe_test_skip_arrival", "qe_trace_fused",
     "moe_route", "moe_expert_ffn_q4", "moe_expert_ffn_q2", "moe_expert_ffn_mixed", "moe_combine",
-    "moe_layer_step", "moe_layer_step_noalloc", "workspace", "Tier", "TierDesc",
+    "moe_layer_step", "moe_layer_step_noalloc", "moe_layer_step_host", "workspace", "Tier", "TierDesc",
 ]
 
 
@@ -97,6 +97,7 @@ def _load():
         "moe_combine": (i32, [vp, vp, vp, i32, i32, i32, vp, vp]),
         "moe_layer_step": (i32, [P(Cfg), P(Layer), vp, i32, i32, vp, i32, vp, vp, vp, sz, vp]),
         "moe_layer_step_noalloc": (i32, [P(Cfg), P(Layer), vp, i32, vp, i32, vp, vp, vp, vp]),
+        "moe_layer_step_host": (i32, [P(Cfg), P(Layer), vp, i32, i32, vp, i32, vp, sz, vp]),
         "qe_tier_create": (i32, [P(TierDesc), P(vp)]),
         "qe_tier_resolve": (i32, [vp, i32, P(ctypes.c_int32), i32, vp, vp]),
         "qe_tier_layer_step": (i32, [vp, i32, P(Layer), vp, i32, i32, vp, i32, vp, vp, vp, sz, vp]),
@@ -311,6 +312,21 @@ class Tier:
             self.close()
         except Exception:
             pass
+
+
+def moe_layer_step_host(cfg, layer: Layer, x_host, out_host, add_residual=False, ws=None, stream=None):
+    """The layer step on host tensors (pinned for asynchronous copies):
+    copy in, step, copy out, synchronise."""
+    import torch
+    if x_host.is_cuda or out_host.is_cuda:
+        raise ValueError("moe_layer_step_host takes host tensors")
+    if not (x_host.is_contiguous() and out_host.is_contiguous()):
+        raise ValueError("expected contiguous tensors")
+    T = x_host.shape[0]
+    dt = QE_BF16 if x_host.dtype == torch.bfloat16 else QE_F32
+    _check(lib.moe_layer_step_host(ctypes.byref(cfg), ctypes.byref(layer), x_host.data_ptr(), dt, T,
+                                   out_host.data_ptr(), 1 if add_residual else 0, _ptr(ws), _nbytes(ws),
+                                   _stream(stream)))
 
 
 class ExpertPool:

@@ -70,6 +70,8 @@ WsLayout ws_layout(int H, int E, int K, int I, int T) {
   L.grp_list = take(4 * t * K);
   L.grp_order = take(4 * (size_t)E);
   L.xh = take(2 * t * H);
+  L.xin = take(4 * t * H);
+  L.xout = take(4 * t * H);
   L.total = off;
   return L;
 }
@@ -375,6 +377,31 @@ int experts_and_combine(const qe_cfg* c, const qe_expert* experts, const int32_t
 }
 
 }  // namespace qe
+
+extern "C" int moe_layer_step_host(const qe_cfg* c, const qe_layer* layer, const void* x_host, int x_dtype, int T,
+                                   float* out_host, int add_residual, void* ws, size_t ws_bytes, qe_stream_t stream) {
+  int rc = check_cfg(c);
+  if (rc) return rc;
+  if (T < 0) return fail(QE_ERR_INVALID_ARG, "T must be >= 0");
+  if (T == 0) return QE_OK;
+  if (!(x_dtype == QE_F32 || x_dtype == QE_BF16)) return fail(QE_ERR_INVALID_ARG, "x_dtype must be QE_F32 or QE_BF16");
+  if (!x_host || !out_host) return fail(QE_ERR_INVALID_ARG, "x_host and out_host must not be NULL");
+  if ((rc = check_ws(c, T, ws, ws_bytes))) return rc;
+  const WsLayout L = ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, T);
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t xb = (size_t)T * c->hidden * (x_dtype == QE_BF16 ? 2 : 4);
+  const size_t ob = (size_t)T * c->hidden * 4;
+  void* xd = at<unsigned char>(ws, L.xin);
+  float* od = at<float>(ws, L.xout);
+  cudaError_t e = cudaMemcpyAsync(xd, x_host, xb, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step_host: copy x in");
+  rc = moe_layer_step(c, layer, xd, x_dtype, T, od, add_residual, nullptr, nullptr, ws, ws_bytes, stream);
+  if (rc) return rc;
+  e = cudaMemcpyAsync(out_host, od, ob, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step_host: copy out");
+  return QE_OK;
+}
 
 // ---------------------------------------------------------------------------
 // Single-token layer step whose scratch lives in the library itself.

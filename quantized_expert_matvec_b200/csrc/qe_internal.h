@@ -50,6 +50,8 @@ struct WsLayout {
   size_t grp_list;  // int    [T*K]  assignment ids (t*K+k) sorted by expert
   size_t grp_order; // int    [E]    active experts, most tokens first
   size_t xh;        // fp16   [T*H]  xn for the tensor-core gate/up
+  size_t xin;       // float  [T*H]  device copy of a host x (moe_layer_step_host)
+  size_t xout;      // float  [T*H]  device result before its copy to the host
   size_t total;
 };
 

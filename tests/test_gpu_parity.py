@@ -447,3 +447,22 @@ def test_batched_tensor_core_groups_full_shape(q):
         assert list(ih[t]) == list(ref["idx"])
         err = normwise_err(oh[t], ref["out"])
         assert err <= TOL, (t, err)
+
+
+def test_layer_step_on_host_buffers(q, c1_layer):
+    """moe_layer_step_host (host buffers in and out) gives exactly what
+    moe_layer_step gives on device buffers, for one token (fused kernel) and
+    for five (batched path)."""
+    import torch
+    dl = c1_layer
+    for T, bf16 in ((1, False), (5, True)):
+        x = dev_tokens(0, 9100 + T, T, 4096, bf16=bf16)
+        ws = q.workspace(dl.cfg, T)
+        ref = torch.empty((T, 4096), dtype=torch.float32, device="cuda")
+        q.moe_layer_step(dl.cfg, dl.layer_struct, x, ref, True, None, None, ws)
+        assert q.qe_workspace_status(ws) == q.QE_OK, q.qe_last_error()
+        xh = x.cpu().pin_memory()
+        oh = torch.empty((T, 4096), dtype=torch.float32).pin_memory()
+        q.moe_layer_step_host(dl.cfg, dl.layer_struct, xh, oh, True, ws)
+        assert q.qe_workspace_status(ws) == q.QE_OK, q.qe_last_error()
+        assert torch.equal(oh, ref.cpu())
