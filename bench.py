@@ -66,12 +66,19 @@ def expert_bytes(H, I, bits):
     return n * bits // 8 + 2 * 2 * n // 64
 
 
-def kernel_source_hash():
+KERNEL_SOURCES = {  # the sources the dominant kernel of each workload is compiled from
+    "c1": ("qe_fused.cu", "qe_device.cuh"),
+    "c0": ("qe_fused.cu", "qe_device.cuh"),
+    "c2": ("qe_fused.cu", "qe_device.cuh"),
+    "c4": ("qe_grouped.cu", "qe_device.cuh"),
+}
+
+
+def kernel_source_hash(workload="c1"):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "quantized_expert_matvec_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in KERNEL_SOURCES.get(workload, ("qe_fused.cu", "qe_device.cuh")):
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -83,7 +90,7 @@ def load_traffic(workload):
         d = json.load(open(path))
     except (OSError, ValueError):
         return None
-    if d.get("kernel_source_hash") != kernel_source_hash():
+    if d.get("kernel_source_hash") != kernel_source_hash(workload):
         return None
     return d.get("traffic_bytes_per_launch")
 
@@ -420,7 +427,7 @@ def run_ours(args, wl, rank, world, local_rank):
     achieved = alg / per_step_s / 1e9
     peak = float(peaks["hbm_gbs"])
     cpu = None if args.no_cpu_baseline else cpu_baseline(wl, seed)
-    kern = "qe_fused_layer_kernel" if T == 1 else "grouped_expert_kernel (+ route, group, combine)"
+    kern = "qe_fused_layer_kernel" if T == 1 else "grouped_gateup_kernel + grouped_down_kernel (+ route, group, combine)"
     line = {
         "metric": wl["metric"], "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,

@@ -110,3 +110,20 @@ def test_tier_arguments_checked_before_any_cuda_call(q):
     assert lib.qe_tier_stats(None, None, None, None) == q.QE_ERR_INVALID_ARG
     assert lib.qe_tier_resolve(None, 0, None, 0, None, None) == q.QE_ERR_INVALID_ARG
     lib.qe_tier_destroy(None)
+
+
+def test_host_buffer_step_arguments_checked_first(q):
+    """moe_layer_step_host rejects bad arguments before any CUDA call."""
+    lib = q.lib
+    cfg = q.Cfg(256, 16, 2, 64)
+    layer = q.Layer(None, None, None, None)
+    buf = (ctypes.c_float * 256)()
+    assert lib.moe_layer_step_host(ctypes.byref(cfg), ctypes.byref(layer), None, 0, 1, buf, 0, None, 0,
+                                   None) == q.QE_ERR_INVALID_ARG
+    assert lib.moe_layer_step_host(ctypes.byref(cfg), ctypes.byref(layer), buf, 5, 1, buf, 0, None, 0,
+                                   None) == q.QE_ERR_INVALID_ARG
+    assert "x_dtype" in q.qe_last_error()
+    assert lib.moe_layer_step_host(ctypes.byref(cfg), ctypes.byref(layer), buf, 0, 1, buf, 0, None, 0,
+                                   None) == q.QE_ERR_INVALID_ARG
+    assert "workspace" in q.qe_last_error()
+    assert lib.moe_layer_step_host(ctypes.byref(cfg), ctypes.byref(layer), buf, 0, 0, buf, 0, None, 0, None) == q.QE_OK
