@@ -12,17 +12,17 @@
 //
 // Expert phase.  Gate/up: the selected experts' rows are cut into items of
 // RB rows of gate and of up; the four 4-warp groups take items in turn and
-// each warp of a group copies (16-byte cp.async into the group's ring) and
-// dequantises one column quarter of every row, keeping the x' of its columns
-// in registers; the four quarter sums meet in shared memory behind a named
-// barrier, and h = silu(g) * u goes to global memory.  Down: warp w works on
-// expert w % K and computes full rows (RC-row blocks of the output rows this
-// CTA owns) with h_k in registers; its rows are prefetched to L2 when the
-// expert phase starts.  Down rows need h_k in full: every gate/up item of
-// expert k bumps a global counter ready[k]; the first warp of a CTA that needs
-// h_k waits for the count, stages h_k in x' form in shared memory and raises a
-// flag for the others.  All such waits are bounded (QE_ERR_TIMEOUT).
-// The last CTA to finish resets the counters for the next launch.
+// each warp of a group copies (16-byte cp.async into the group's ring, one
+// copy group per item) and dequantises one column quarter of every row,
+// keeping the x' of its columns in registers; the four quarter sums meet in
+// shared memory behind a named barrier, and h = silu(g) * u goes to global
+// memory.  Each warp then loads its first down rows into registers.  A second
+// grid-wide counter waits for every CTA's h rows; every CTA then reads all
+// of h, finds max |h_k| itself and stages h_k in x' form in shared memory.
+// Down: warp w works on expert w % K and computes full rows (RC-row blocks of
+// the output rows this CTA owns); the CTA combines its rows (+ residual).
+// All waits are bounded (QE_ERR_TIMEOUT); the last CTA to finish resets the
+// counters for the next launch.
 #include <math.h>
 
 #include <type_traits>
