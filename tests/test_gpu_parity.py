@@ -466,3 +466,27 @@ def test_layer_step_on_host_buffers(q, c1_layer):
         q.moe_layer_step_host(dl.cfg, dl.layer_struct, xh, oh, True, ws)
         assert q.qe_workspace_status(ws) == q.QE_OK, q.qe_last_error()
         assert torch.equal(oh, ref.cpu())
+
+
+def test_hidden_2048_mixed_bits_single_and_batched(q):
+    """Hidden 2048 (the fused kernel's one-piece scale copies), 64 experts,
+    top-4, intermediate 512, every third expert 2-bit, Zipf offset, residual:
+    one token at a time through the fused kernel and six tokens through the
+    batched path, all against the oracle."""
+    import torch
+    cfg = q.Cfg(2048, 64, 4, 512)
+    off = synth.zipf_logit_offset(8, 2, 64)
+    dl = DevLayer(q, cfg, seed=8, layer=2, bits_of=lambda e: 2 if e % 3 == 0 else 4, offset=off)
+    x = dev_tokens(8, 300, 6, 2048)
+    out, idx, w = run_fused(q, dl, x, residual=True)
+    for t in range(6):
+        check(dl, out[t], idx[t], w[t], dl.oracle(host_x_f64(8, 300 + t, 2048), residual=True))
+    ws = q.workspace(cfg, 6)
+    ob = torch.empty((6, 2048), dtype=torch.float32, device="cuda")
+    ib = torch.empty((6, 4), dtype=torch.int32, device="cuda")
+    wb = torch.empty((6, 4), dtype=torch.float32, device="cuda")
+    q.moe_layer_step(cfg, dl.layer_struct, x, ob, True, ib, wb, ws)
+    assert q.qe_workspace_status(ws) == q.QE_OK, q.qe_last_error()
+    ob, ib, wb = ob.cpu().numpy(), ib.cpu().numpy(), wb.cpu().numpy()
+    for t in range(6):
+        check(dl, ob[t], ib[t], wb[t], dl.oracle(host_x_f64(8, 300 + t, 2048), residual=True))
