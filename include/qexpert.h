@@ -330,7 +330,7 @@ QE_API void qe_test_skip_arrival(int cta);
  * done, 7 gate/up phase done, 8 h barrier passed, 9 h staged, 10 last down
  * row done, 11 end; 12 and 13 the SM cycle counter at start and end; 16+w
  * and 32+w: warp w done with gate/up and with down; 48 CTA joined after the
- * expert phase, 49 combine done, 53 exit counter bumped; 56-58 routing
+ * expert phase, 49 combine done; 56-58 routing
  * sub-steps (router loop, first barrier, RMSNorm pass 2); 59/60 warp 0's
  * first gate/up item landed / computed, 61 its group past that item, 62/63
  * the same for the second item.  Slots a CTA does not reach keep their old

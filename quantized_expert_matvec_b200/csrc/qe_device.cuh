@@ -41,6 +41,30 @@ QE_DEV void set_error(int* err, int code) { atomicCAS(err, 0, code); }
 
 // Spin (bounded) until *ctr >= target.  Returns false on timeout or if the
 // CTA-wide abort flag is raised.
+QE_DEV unsigned long long atom_add_release_u64(unsigned long long* p, unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.release.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+
+QE_DEV unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait until a 64-bit counter reaches target; false if the deadline
+// passed or the CTA's abort flag was raised.
+QE_DEV bool wait_geq64(const unsigned long long* ctr, unsigned long long target, uint64_t deadline,
+                       volatile int* abort_flag) {
+  unsigned spins = 0;
+  while (ld_acquire_u64(ctr) < target) {
+    if (*abort_flag) return false;
+    if ((++spins & 15u) == 0 && gtimer() > deadline) return false;
+  }
+  return true;
+}
+
 QE_DEV bool wait_geq(const unsigned* ctr, unsigned target, uint64_t deadline,
                      volatile int* abort_flag) {
   unsigned spins = 0;

@@ -21,8 +21,9 @@
 // of h, finds max |h_k| itself and stages h_k in x' form in shared memory.
 // Down: warp w works on expert w % K and computes full rows (RC-row blocks of
 // the output rows this CTA owns); the CTA combines its rows (+ residual).
-// All waits are bounded (QE_ERR_TIMEOUT); the last CTA to finish resets the
-// counters for the next launch.
+// All waits are bounded (QE_ERR_TIMEOUT).  The grid counters only grow: each
+// launch adds its grid size, and a CTA's arrival ticket gives the count it
+// waits for, so nothing has to be reset between launches.
 #include <math.h>
 
 #include <type_traits>
@@ -48,6 +49,7 @@ struct FusedMisc {
   qe_expert ex[kMaxK];
   float hK[kMaxK];
   int hexp[kMaxK];  // vector exponent of h_k (x' form of the down input)
+  unsigned long long route_target;  // routing counter value that completes this launch
   unsigned cand_idx[kWarps][kMaxK];
   unsigned long long cand_key[kWarps][kMaxK];
   double cand_val[kWarps][kMaxK];
@@ -374,7 +376,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   __syncthreads();
   if (tid == 0) {
     QE_TRACE(kTrRouterDone);
-    if (!given && cta != p.skip_cta) red_release_add(&ctl->route_ctr, 1u);  // publishes this CTA's logits
+    if (!given) {
+      // the release publishes this CTA's logits; the ticket names the count
+      // that completes this launch's arrivals (a CTA told to skip its
+      // arrival, a test hook, waits for the same count and times out too)
+      const unsigned long long t =
+          cta != p.skip_cta ? atom_add_release_u64(&ctl->route_ctr, 1ull) : ld_acquire_u64(&ctl->route_ctr);
+      misc->route_target = (t / (unsigned)G + 1ull) * (unsigned)G;
+    }
   }
   {
     float m = 0.f;
@@ -403,7 +412,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
     }
   }
   if (tid == 0) {
-    if (!given && !wait_geq(&ctl->route_ctr, (unsigned)G, deadline, abort_flag)) {
+    if (!given && !wait_geq64(&ctl->route_ctr, misc->route_target, deadline, abort_flag)) {
       set_error(&ctl->err, QE_ERR_TIMEOUT);
       misc->abort = 1;
     }
@@ -482,11 +491,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
     // renormalised softmax over the K kept logits (sum in k order); lanes
     // k < K also fetch and check the K expert descriptors
     const double lmax = misc->lsel[0];
-    const double ev = lane < K ? exp(misc->lsel[lane] - lmax) : 0.0;
-    double s = 0.0;
+    const float ev = lane < K ? expf((float)(misc->lsel[lane] - lmax)) : 0.0f;
+    float s = 0.0f;
     for (int k = 0; k < K; ++k) s += __shfl_sync(0xffffffffu, ev, k);
     if (lane < K) {
-      misc->wk[lane] = (float)(ev / s);
+      misc->wk[lane] = ev / s;
       if (cta == 0 && p.topk_idx) p.topk_idx[lane] = misc->idx[lane];
       if (cta == 0 && p.topk_w) p.topk_w[lane] = misc->wk[lane];
       const qe_expert ex = p.experts[misc->idx[lane]];
@@ -599,8 +608,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
     if (!*abort_flag) {
       // the release publishes the h rows every thread of this CTA stored
       // before the barrier above
-      red_release_add(&ctl->h_ctr, 1u);
-      if (!wait_geq(&ctl->h_ctr, (unsigned)G, deadline, abort_flag)) {
+      const unsigned long long t = atom_add_release_u64(&ctl->h_ctr, 1ull);
+      if (!wait_geq64(&ctl->h_ctr, (t / (unsigned)G + 1ull) * (unsigned)G, deadline, abort_flag)) {
         set_error(&ctl->err, QE_ERR_TIMEOUT);
         misc->abort = 1;
       }
@@ -749,17 +758,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   __syncthreads();
   if (tid == 0) {
     QE_TRACE(49);
-    __threadfence();
-    const unsigned prev = atomicAdd(&ctl->exit_ctr, 1u);
-    QE_TRACE(53);
-    if (prev == (unsigned)G - 1) {
-      ctl->route_ctr = 0;
-      ctl->h_ctr = 0;
-      for (int k = 0; k < kMaxK; ++k) ctl->hamax[k] = 0;
-      __threadfence();
-      ctl->exit_ctr = 0;
-      __threadfence();
-    }
     if (p.trace) p.trace[(size_t)cta * 64 + kTrLastC] = misc->t_lastC;
     QE_TRACE(kTrEnd);
     if (p.trace) p.trace[(size_t)cta * 64 + 13] = clock64();

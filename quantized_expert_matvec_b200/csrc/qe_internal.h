@@ -17,12 +17,13 @@ constexpr int kGroup = 64;
 
 // Control words at the start of every workspace.
 struct WsControl {
-  int err;             // first device-side error (QE_ERR_*), 0 if none
-  unsigned route_ctr;  // fused kernel: CTAs past the router
-  unsigned exit_ctr;   // fused kernel: CTAs finished
-  unsigned h_ctr;      // fused kernel: CTAs that published their h rows
-  unsigned hamax[kMaxK];  // fused kernel: max |h_k| as float bits
-  unsigned pad[44];
+  int err;                       // first device-side error (QE_ERR_*), 0 if none
+  unsigned reserved;
+  // fused kernel grid counters: they only grow, every launch adds its grid
+  // size, and a CTA's arrival ticket tells it the count that ends its wait
+  unsigned long long route_ctr;  // CTAs past the router
+  unsigned long long h_ctr;      // CTAs that published their h rows
+  unsigned pad[58];
 };
 static_assert(sizeof(WsControl) == 256, "control block");
 
