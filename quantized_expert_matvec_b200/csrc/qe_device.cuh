@@ -143,6 +143,15 @@ QE_DEV void cp_async16(void* dst, const void* src, uint64_t pol) {
                "l"(pol)
                : "memory");
 }
+// 8- and 4-byte asynchronous copies (cached form; dst and src aligned to the size).
+QE_DEV void cp_async8(void* dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 8, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "l"(pol)
+               : "memory");
+}
+QE_DEV void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
 QE_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 QE_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }

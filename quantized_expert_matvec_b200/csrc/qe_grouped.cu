@@ -1,21 +1,31 @@
 // qe_grouped.cu -- batched layer step (T tokens per step): the (token, k)
 // assignments are grouped by expert so each selected expert's weights are
-// streamed from HBM once per step and reused by all of its tokens.
+// streamed from HBM once per token pass and reused by all of its tokens.
 //
 //   group kernel  : counting sort of the T*K assignments by expert (stable:
 //                   ascending assignment id inside an expert); active experts
 //                   ordered by descending token count
-//   gate/up kernel: persistent CTAs take items (expert, block of kRowsA
-//                   rows) from a shared counter; the CTA stages the x' of the
-//                   expert's tokens in shared memory and each warp takes
-//                   rows: a packed word is masked once and multiplied into
-//                   the accumulators of every token; h = silu(g) u and the
-//                   running max |h| per assignment go to global memory
-//   down kernel   : items (expert, block of kRowsB output rows); the CTA
-//                   stages h of the expert's tokens in x' form, warps take
-//                   pairs of rows -> y[assignment][H]
+//   gate/up kernel: persistent CTAs take items (expert, kRowsA rows of gate
+//                   and of up) from a shared counter; an item is cut into
+//                   segments of at most kTile tokens.  The CTA stages the x'
+//                   of the segment's tokens in shared memory; each warp takes
+//                   units of two output rows (two gate rows and the two up
+//                   rows: four matrix rows) and each lane a 32-column chunk
+//                   of them per step.  A packed word pair is masked once and
+//                   multiplied into the accumulators of every token, and each
+//                   x' piece read from shared memory serves the four rows.
+//                   h = silu(g) u and the running max |h| per assignment go
+//                   to global memory.
+//   down kernel   : the same over items (expert, kRowsB rows of down), units
+//                   of four rows, with h of the segment's tokens staged in
+//                   x' form -> y[assignment][H]
 //   combine       : out[t] = sum_k w[t,k] y[t*K+k] (+ x[t])
-// Up to kTT tokens of an expert share one pass over its weights.
+//
+// The expert kernels are bound by the bytes they stream, so each warp keeps
+// kSlots steps of packed words in flight in registers: the slot of a step is
+// refilled with the step kSlots ahead as soon as it has been used, and at the
+// end of a segment the refills already fetch the next segment's first steps,
+// so the loads run across the staging of the next segment's activations.
 #include <math.h>
 
 #include "qe_device.cuh"
@@ -24,9 +34,10 @@ namespace qe {
 
 constexpr int kGWarps = 16;
 constexpr int kGThreads = kGWarps * 32;
-constexpr int kTT = 8;       // tokens sharing one pass over the weights
+constexpr int kTile = 4;     // tokens sharing one pass over the weights
 constexpr int kRowsA = 128;  // gate/up rows (of gate and of up) per item
 constexpr int kRowsB = 512;  // down rows per item
+constexpr int kSlots = 3;    // steps of packed words in flight per warp
 constexpr bool kTcEnabled = false;  // see launch_grouped
 
 // Round a count of 4-byte elements up to a multiple of 4 (16 bytes).
@@ -113,8 +124,9 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t* __restrict__
 
 struct GroupedKParams {
   int H, I, K, T;
+  int tile;           // tokens per pass of this kernel (1, 2 or 4)
   const qe_expert* experts;
-  const float* xp4;   // [T][H] x' (linear layout)
+  const float* xp4;   // [T][H] x' (pair order, unswizzled)
   const float* xp2;
   const float* xsum;  // [T][H/32]
   const int* xexp;    // [T]
@@ -122,342 +134,430 @@ struct GroupedKParams {
   const int* start;
   const int* list;
   const int* order;
-  int* ctl;           // [0] active experts, [1] gate/up work, [2] down work
+  int* ctl;           // [0] active experts, [1] gate/up work, [2] down work, [3] tensor-core experts
   float* h;           // [T*K][I]
   unsigned* hamax;    // [T*K]
   float* y;           // [T*K][H]
   int* err;
-  int tile;           // tokens per pass (<= kTT)
 };
 
+// Packed words and scales/biases are copied with 16-, 8- and 4-byte
+// asynchronous copies, so every pointer of a descriptor must be 16-byte
+// aligned (the library's documented contract).
 static __device__ __forceinline__ bool qmat_ok(const qe_qmat& m, int bits) {
-  return m.bits == bits && m.wq && m.scales && m.biases && ((uintptr_t)m.wq & 15) == 0;
+  return m.bits == bits && m.wq && m.scales && m.biases && ((uintptr_t)m.wq & 15) == 0 &&
+         ((uintptr_t)m.scales & 15) == 0 && ((uintptr_t)m.biases & 15) == 0;
 }
 
-// Field pairs of sub-block b (0 or 1) of a 32-column chunk: 8 pairs, each
-// the same field of two packed words.  4-bit: b picks the word pair (words
-// 2b, 2b+1), fields 0..7; 2-bit: fields 8b..8b+7 of the chunk's one word
-// pair (in w.x).  Pair k of sub-block b multiplies x' pair 8b + k.
-template <int BITS>
-static __device__ __forceinline__ void mask_sub(const ulonglong2 w, int b, float2 (&m)[8]) {
-  if (BITS == 4) {
-    const unsigned long long P = b ? w.y : w.x, S = P >> 12;
-    m[0] = f2_of(P & rep2(0xFu));
-    m[1] = f2_of(P & rep2(0xF0u));
-    m[2] = f2_of(P & rep2(0xF00u));
-    m[3] = f2_of(P & rep2(0xF000u));
-    m[4] = f2_of(P & rep2(0xF0000u));
-    m[5] = f2_of(S & rep2(0xF00u));
-    m[6] = f2_of(S & rep2(0xF000u));
-    m[7] = f2_of(S & rep2(0xF0000u));
-  } else if (b == 0) {
-    const unsigned long long P = w.x;
+// One segment of an item: rows [r0, r0 + nrows) of expert e against tokens
+// [t0, t0 + nt) of the expert's assignment list.  m0/m1 are gate/up for the
+// gate/up kernel, m0 is down for the down kernel.
+struct GSeg {
+  int valid, e, bits, r0, nrows, t0, nt;
+  qe_qmat m0, m1;
+};
+
+// Per-warp ring of kSlots steps in shared memory.  A step is, for each lane,
+// the packed 32-column chunk of four matrix rows (16 bytes each; 8 at 2-bit)
+// and the 4-byte words holding the chunk's bf16 scale and bias in each row.
+// Layout [slot][row][lane] (words) and [slot][row][scale|bias][lane], so a
+// warp's accesses to one row fall on consecutive addresses.  Each lane reads
+// only what it copied itself.
+constexpr int kRingWords = kSlots * 4 * 32 * 16;
+constexpr int kRingSb = kSlots * 4 * 2 * 32 * 4;
+constexpr int kRingWarp = kRingWords + kRingSb;  // 9 KiB
+
+// Token-pass width for nt live tokens: 1, 2 or 4.
+static __host__ __device__ __forceinline__ int nt_pad(int nt) { return nt <= 1 ? 1 : (nt <= 2 ? 2 : 4); }
+
+// Units of four matrix rows in a segment: gate/up takes output rows in pairs
+// (gate and up of each), down takes four rows.
+template <int MODE>
+static __device__ __forceinline__ int seg_units(const GSeg& s) { return MODE == 0 ? s.nrows / 2 : s.nrows / 4; }
+
+// Steps of warp `warp` in segment s: its units warp, warp + kGWarps, ...
+// times cpl chunks per lane and row.
+template <int MODE>
+static __device__ __forceinline__ int seg_steps(const GSeg& s, int warp, int cpl) {
+  const int u = seg_units<MODE>(s);
+  return u > warp ? ((u - warp + kGWarps - 1) / kGWarps) * cpl : 0;
+}
+
+// Row of matrix row m (0..3) of unit q.
+template <int MODE>
+static __device__ __forceinline__ int unit_row(const GSeg& s, int q, int m) {
+  return MODE == 0 ? s.r0 + 2 * q + (m & 1) : s.r0 + 4 * q + m;
+}
+
+// Issue the copies of step (k, c) of this warp in segment s -- chunk c of
+// the lanes in the warp's k-th unit -- into ring slot (rw, rsb) (C = columns
+// of the matrices; lanes past the last chunk copy nothing).  The caller
+// commits the group.
+template <int MODE>
+static __device__ __forceinline__ void issue_step(const GSeg& s, int C, int k, int c, int warp, int lane,
+                                                  unsigned char* rw, uint32_t* rsb, uint64_t pol) {
+  const int q = warp + kGWarps * k;
+  const int lc = 32 * c + lane;
+  if (lc >= C / 32) return;
+  const int bits = s.bits;
+  const size_t rowb = (size_t)C * bits / 8;
+  const int gpr = C / kGroup;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) m[j] = f2_of(P & rep2(3u << (2 * j)));
-  } else {
-    const unsigned long long P = w.x, S = P >> 12;
-    m[0] = f2_of(P & rep2(0x30000u));
-    m[1] = f2_of(P & rep2(0xC0000u));
-    m[2] = f2_of(P & rep2(0x300000u));
-    m[3] = f2_of(S & rep2(0xC00u));
-    m[4] = f2_of(S & rep2(0x3000u));
-    m[5] = f2_of(S & rep2(0xC000u));
-    m[6] = f2_of(S & rep2(0x30000u));
-    m[7] = f2_of(S & rep2(0xC0000u));
+  for (int m = 0; m < 4; ++m) {
+    const qe_qmat& mat = (MODE == 0 && m >= 2) ? s.m1 : s.m0;
+    const int row = unit_row<MODE>(s, q, m);
+    const unsigned char* rp = (const unsigned char*)mat.wq + (size_t)row * rowb;
+    if (bits == 4) cp_async16(rw + (m * 32 + lane) * 16, rp + (size_t)lc * 16, pol);
+    else cp_async8(rw + (m * 32 + lane) * 16, rp + (size_t)lc * 8, pol);
+    // the 4-byte word holding group gi's entry (gi rounded down to even; the
+    // arrays hold an even number of entries, so the word is in bounds)
+    const size_t gi2 = ((size_t)row * gpr + (lc >> 1)) & ~(size_t)1;
+    cp_async4(rsb + (m * 2 + 0) * 32 + lane, mat.scales + gi2);
+    cp_async4(rsb + (m * 2 + 1) * 32 + lane, mat.biases + gi2);
   }
 }
 
-// x' pairs 8b..8b+7 of 32-column chunk lc from a swizzled buffer.
-static __device__ __forceinline__ void xs_sub(const float* xp, int lc, int b, float2 (&x)[8]) {
-  const float4* src = (const float4*)(xp + lc * 32);
+// Field f of both words of a word pair P (S = P >> 12), as the float pair
+// fed to the multiply-add: fields that reach bit 23 come from S, so no field
+// touches the exponent bits.
+template <int BITS>
+static __device__ __forceinline__ float2 field_pair(unsigned long long P, unsigned long long S, int f) {
+  if (BITS == 4) return f2_of(f < 5 ? (P & rep2(0xFu << (4 * f))) : (S & rep2(0xFu << (4 * f - 12))));
+  return f2_of(f < 11 ? (P & rep2(3u << (2 * f))) : (S & rep2(3u << (2 * f - 12))));
+}
+
+// Piece i (0..7) of a chunk: x' pairs 2i and 2i+1.  4-bit: fields 2(i&3),
+// 2(i&3)+1 of word pair i>>2; 2-bit: fields 2i, 2i+1 of the one word pair.
+template <int BITS>
+static __device__ __forceinline__ void piece_masks(const ulonglong2 w, int i, float2& m0, float2& m1) {
+  const unsigned long long P = (BITS == 4 && i >= 4) ? w.y : w.x, S = P >> 12;
+  const int f = BITS == 4 ? 2 * (i & 3) : 2 * i;
+  m0 = field_pair<BITS>(P, S, f);
+  m1 = field_pair<BITS>(P, S, f + 1);
+}
+
+// One step: chunk lc of the four matrix rows in ring slot (rw, rsb) against
+// the NT staged token vectors (x' swizzled, [NT][C]); v[m*NT + t] gets row m,
+// token t.  par[m] = parity of the chunk's group index in row m (which half
+// of the copied 4-byte scale/bias word is the chunk's).
+template <int BITS, int NT>
+static __device__ __forceinline__ void compute_step(const unsigned char* rw, const uint32_t* rsb, const int (&par)[4],
+                                                    const float* xs, const float* sums, const float* xk, int C,
+                                                    int lc, int lane, float (&v)[4 * NT]) {
+  const int nch = C / 32;
+  if (lc >= nch) return;
+  ulonglong2 w[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    if (BITS == 4) {
+      w[m] = *(const ulonglong2*)(rw + (m * 32 + lane) * 16);
+    } else {
+      w[m].x = *(const unsigned long long*)(rw + (m * 32 + lane) * 16);
+      w[m].y = 0ull;
+    }
+  }
+  float2 acc[4][NT];
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[m][t] = make_float2(0.f, 0.f);
+  const float4* xb = (const float4*)(xs + lc * 32);
   const int sw = lc & 7;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float4 a = src[(4 * b + i) ^ sw];
-    x[2 * i] = make_float2(a.x, a.y);
-    x[2 * i + 1] = make_float2(a.z, a.w);
+  for (int i = 0; i < 8; ++i) {
+    float4 xp[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) xp[t] = xb[t * (C / 4) + (i ^ sw)];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      float2 m0, m1;
+      piece_masks<BITS>(w[m], i, m0, m1);
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        acc[m][t] = __ffma2_rn(m0, make_float2(xp[t].x, xp[t].y), acc[m][t]);
+        acc[m][t] = __ffma2_rn(m1, make_float2(xp[t].z, xp[t].w), acc[m][t]);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const uint32_t sw2 = rsb[(m * 2 + 0) * 32 + lane], bw2 = rsb[(m * 2 + 1) * 32 + lane];
+    const float sc = __uint_as_float(par[m] ? (sw2 & 0xFFFF0000u) : (sw2 << 16));
+    const float bi = __uint_as_float(par[m] ? (bw2 & 0xFFFF0000u) : (bw2 << 16));
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+      v[m * NT + t] += sc * xk[t] * (acc[m][t].x + acc[m][t].y) + bi * sums[t * nch + lc];
   }
 }
 
-// Packed words of 32-column chunk lc of a row (4-bit: 4 words; 2-bit: 2 in .x).
-template <int BITS>
-static __device__ __forceinline__ ulonglong2 load_chunk(const unsigned char* row, int lc) {
-  if (BITS == 4) return __ldcs((const ulonglong2*)row + lc);
-  ulonglong2 w;
-  w.x = __ldcs((const unsigned long long*)row + lc);
-  w.y = 0ull;
-  return w;
+// End of unit q: reduce v over the warp and write the unit's results.
+// Gate/up: h = silu(g) u for output rows 2q, 2q+1, and |h| into the
+// segment's maxima; down: y of rows 4q..4q+3.
+template <int MODE, int NT>
+static __device__ __forceinline__ void unit_epilogue(const GroupedKParams& p, const GSeg& s, const int* asg, int q,
+                                                     float (&v)[4 * NT], unsigned* hmax, int lane) {
+  const float sv = warp_reduce_rows<4 * NT>(v, lane);
+  const int ri = reduced_row_of_lane<4 * NT>(lane);  // m * NT + t
+  const int m = ri / NT, t = ri - m * NT;
+  const bool first = lane == lane_of_reduced_row<4 * NT>(ri);
+  if (MODE == 0) {
+    // lanes holding g of (row, token) fetch u of the same pair
+    const float uv = __shfl_sync(0xffffffffu, sv, lane_of_reduced_row<4 * NT>(m < 2 ? ri + 2 * NT : ri));
+    if (m < 2 && t < s.nt && first) {
+      const float hv = sv / (1.0f + expf(-sv)) * uv;
+      p.h[(size_t)asg[t] * p.I + unit_row<0>(s, q, m)] = hv;
+      atomicMax(&hmax[t], __float_as_uint(fabsf(hv)));
+    }
+  } else {
+    if (t < s.nt && first) p.y[(size_t)asg[t] * p.H + unit_row<1>(s, q, m)] = sv;
+  }
 }
 
-// Stage x' (swizzled), 32-column sums and scale of nt tokens.
-static __device__ void stage_x(const GroupedKParams& p, int bits, const int* toks, int nt, float* xs_sm,
-                               float* sum_sm, float* xk_sm) {
-  const int H = p.H;
-  const float* src = bits == 4 ? p.xp4 : p.xp2;
-  for (int i = threadIdx.x; i < nt * (H / 4); i += kGThreads) {
-    const int t = i / (H / 4), c = (i - t * (H / 4)) * 4;
-    const float4 v = *(const float4*)(src + (size_t)toks[t] * H + c);
-    *(float4*)(xs_sm + t * H + xswz(c)) = v;  // global x' is in pair order; pieces move whole
-  }
-  for (int i = threadIdx.x; i < nt * (H / 32); i += kGThreads) {
-    const int t = i / (H / 32), c = i - t * (H / 32);
-    sum_sm[i] = p.xsum[(size_t)toks[t] * (H / 32) + c];
-  }
-  if (threadIdx.x < nt) xk_sm[threadIdx.x] = acc_scale(p.xexp[toks[threadIdx.x]]);
-}
-
-// One gate row and one up row (row r) against the nt staged tokens: v[t]
-// (gate) and v[kTT + t] (up) get this lane's partial sums.
-template <int BITS>
-static __device__ __forceinline__ void gateup_row(const qe_expert& ex, int r, int H, int nt, const float* xs_sm,
-                                                  const float* sum_sm, const float* xk_sm, float (&v)[2 * kTT],
-                                                  int lane) {
-  const int gpr = H / kGroup;
-  const size_t rowb = (size_t)H * BITS / 8;
-  const unsigned char* gp = (const unsigned char*)ex.gate.wq + (size_t)r * rowb;
-  const unsigned char* up = (const unsigned char*)ex.up.wq + (size_t)r * rowb;
-  for (int lc = lane; lc < H / 32; lc += 32) {
-    const ulonglong2 wg = load_chunk<BITS>(gp, lc), wu = load_chunk<BITS>(up, lc);
-    const size_t gi = (size_t)r * gpr + (lc >> 1);
-    const float sg = bf16f(__ldg(ex.gate.scales + gi)), bg = bf16f(__ldg(ex.gate.biases + gi));
-    const float su = bf16f(__ldg(ex.up.scales + gi)), bu = bf16f(__ldg(ex.up.biases + gi));
-    float2 ga[kTT], ua[kTT];
+// All steps of this warp in segment S.  Before step l the warp waits until
+// at most kSlots-1 copy groups are pending (step l's group is complete);
+// after it the slot is refilled with step l + kSlots and one group is
+// committed (empty if there is nothing to copy), so the groups stay in step
+// order.  Past the end of S the refills fetch the next segment N, whose
+// steps start at the next multiple of kSlots.  Steps run through (unit k,
+// chunk c) with counters, the computed step and the refilled one apart.
+template <int MODE, int BITS, int NT>
+static __device__ __forceinline__ void run_segment(const GroupedKParams& p, const GSeg& Ssm, const GSeg& N,
+                                                   const int* asg, int C, int cpl, const float* xs,
+                                                   const float* sums, const float* xk, unsigned* hmax,
+                                                   unsigned char* ring, int warp, int lane, uint64_t pol) {
+  const GSeg S = Ssm;  // the segment's fields in registers
+  const int nst = seg_steps<MODE>(S, warp, cpl);
+  const int nstp = (nst + kSlots - 1) / kSlots * kSlots;
+  const int nstN = N.valid ? seg_steps<MODE>(N, warp, cpl) : 0;
+  const int gpr = C / kGroup;
+  float v[4 * NT];
 #pragma unroll
-    for (int t = 0; t < kTT; ++t) { ga[t] = make_float2(0.f, 0.f); ua[t] = make_float2(0.f, 0.f); }
+  for (int i = 0; i < 4 * NT; ++i) v[i] = 0.f;
+  int kc = 0, cc = 0;                          // step being computed
+  int ki = kSlots / cpl, ci = kSlots % cpl;    // step being refilled
+  for (int l0 = 0; l0 < nstp; l0 += kSlots) {
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      float2 mg[8], mu[8];
-      mask_sub<BITS>(wg, b, mg);
-      mask_sub<BITS>(wu, b, mu);
+    for (int j = 0; j < kSlots; ++j) {
+      unsigned char* rw = ring + j * (4 * 32 * 16);
+      uint32_t* rsb = (uint32_t*)(ring + kRingWords) + j * (4 * 2 * 32);
+      const int l = l0 + j;
+      cp_async_wait<kSlots - 1>();
+      if (l < nst) {
+        const int q = warp + kGWarps * kc, lc = 32 * cc + lane;
+        int par[4];
 #pragma unroll
-      for (int t = 0; t < kTT; ++t) {
-        if (t < nt) {
-          float2 xw[8];
-          xs_sub(xs_sm + t * H, lc, b, xw);
+        for (int m = 0; m < 4; ++m) par[m] = (unit_row<MODE>(S, q, m) * gpr + (lc >> 1)) & 1;
+        compute_step<BITS, NT>(rw, rsb, par, xs, sums, xk, C, lc, lane, v);
+        if (cc == cpl - 1) {
+          unit_epilogue<MODE, NT>(p, S, asg, q, v, hmax, lane);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            ga[t] = __ffma2_rn(mg[i], xw[i], ga[t]);
-            ua[t] = __ffma2_rn(mu[i], xw[i], ua[t]);
-          }
+          for (int i = 0; i < 4 * NT; ++i) v[i] = 0.f;
+          cc = 0;
+          ++kc;
+        } else {
+          ++cc;
         }
       }
-    }
-#pragma unroll
-    for (int t = 0; t < kTT; ++t) {
-      if (t < nt) {
-        const float xk = xk_sm[t], xsum = sum_sm[t * (H / 32) + lc];
-        v[t] += sg * xk * (ga[t].x + ga[t].y) + bg * xsum;
-        v[kTT + t] += su * xk * (ua[t].x + ua[t].y) + bu * xsum;
-      }
-    }
-  }
-}
-
-template <int BITS>
-static __device__ void gateup_item(const GroupedKParams& p, const qe_expert& ex, int r0, int r1, int nt,
-                                   const int* asg, const float* xs_sm, const float* sum_sm, const float* xk_sm,
-                                   int warp, int lane) {
-  const int H = p.H, I = p.I;
-  for (int r = r0 + warp; r < r1; r += kGWarps) {
-    float v[2 * kTT];  // gate sums of the tokens, then up sums
-#pragma unroll
-    for (int t = 0; t < 2 * kTT; ++t) v[t] = 0.f;
-    gateup_row<BITS>(ex, r, H, nt, xs_sm, sum_sm, xk_sm, v, lane);
-    const float s = warp_reduce_rows<2 * kTT>(v, lane);
-    const int row = reduced_row_of_lane<2 * kTT>(lane);
-    // lanes holding g of token t fetch u of token t
-    const int src = lane_of_reduced_row<2 * kTT>(row < kTT ? row + kTT : row);
-    const float uv = __shfl_sync(0xffffffffu, s, src);
-    if (row < nt && lane == lane_of_reduced_row<2 * kTT>(row)) {
-      const float hv = s / (1.0f + expf(-s)) * uv;
-      const int a = asg[row];
-      p.h[(size_t)a * I + r] = hv;
-      atomicMax(&p.hamax[a], __float_as_uint(fabsf(hv)));
-    }
-  }
-}
-
-__global__ void __launch_bounds__(kGThreads, 1) grouped_gateup_kernel(const GroupedKParams p) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  const int H = p.H, I = p.I, tile = p.tile;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* xs_sm = (float*)smem;                    // [tile][H]
-  float* sum_sm = xs_sm + al4(tile * H);          // [tile][H/32]
-  float* xk_sm = sum_sm + al4(tile * (H / 32));   // [tile]
-  int* toks = (int*)(xk_sm + al4(tile));          // [tile]
-  int* asg = toks + al4(tile);                    // [tile]
-  __shared__ int s_item;
-  __shared__ qe_expert s_ex;
-  const int ipe = (I + kRowsA - 1) / kRowsA;
-  const int n_tc = p.ctl[3];  // experts done by the tensor-core kernel
-  const int n_items = (p.ctl[0] - n_tc) * ipe;
-  for (;;) {
-    if (threadIdx.x == 0) s_item = atomicAdd(&p.ctl[1], 1);
-    __syncthreads();
-    const int item = s_item;
-    if (item >= n_items) break;
-    const int e = p.order[n_tc + item / ipe];
-    const int r0 = (item % ipe) * kRowsA, r1 = min(I, r0 + kRowsA);
-    if (threadIdx.x == 0) s_ex = p.experts[e];
-    __syncthreads();
-    const int bits = s_ex.gate.bits;
-    const bool ok = (bits == 4 || bits == 2) && qmat_ok(s_ex.gate, bits) && qmat_ok(s_ex.up, bits) &&
-                    qmat_ok(s_ex.down, bits);
-    if (!ok) {
-      if (threadIdx.x == 0) set_error(p.err, QE_ERR_INVALID_ARG);
-      __syncthreads();
-      continue;
-    }
-    const int n = p.count[e], s0 = p.start[e];
-    for (int t0 = 0; t0 < n; t0 += tile) {
-      const int nt = min(tile, n - t0);
-      if (threadIdx.x < nt) {
-        const int a = p.list[s0 + t0 + threadIdx.x];
-        asg[threadIdx.x] = a;
-        toks[threadIdx.x] = a / p.K;
-      }
-      __syncthreads();
-      stage_x(p, bits, toks, nt, xs_sm, sum_sm, xk_sm);
-      __syncthreads();
-      if (bits == 4) gateup_item<4>(p, s_ex, r0, r1, nt, asg, xs_sm, sum_sm, xk_sm, warp, lane);
-      else gateup_item<2>(p, s_ex, r0, r1, nt, asg, xs_sm, sum_sm, xk_sm, warp, lane);
-      __syncthreads();
-    }
-  }
-}
-
-// Two down rows (r and, if two == 2, r + 1) against the nt staged h'
-// vectors: v[t] and v[kTT + t] get this lane's partial sums.
-template <int BITS>
-static __device__ __forceinline__ void down_rows(const qe_qmat& d, int r, int two, int I, int nt, const float* hs_sm,
-                                                 const float* hsum_sm, const float* hk_sm, float (&v)[2 * kTT],
-                                                 int lane) {
-  const int gpr = I / kGroup;
-  const size_t rowb = (size_t)I * BITS / 8;
-  for (int lc = lane; lc < I / 32; lc += 32) {
-    ulonglong2 w[2];
-    float sc[2], bi[2];
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int rr = r + (q < two ? q : 0);
-      w[q] = load_chunk<BITS>((const unsigned char*)d.wq + (size_t)rr * rowb, lc);
-      const size_t gi = (size_t)rr * gpr + (lc >> 1);
-      sc[q] = bf16f(__ldg(d.scales + gi));
-      bi[q] = bf16f(__ldg(d.biases + gi));
-    }
-    float2 acc[2][kTT];
-#pragma unroll
-    for (int t = 0; t < kTT; ++t) { acc[0][t] = make_float2(0.f, 0.f); acc[1][t] = make_float2(0.f, 0.f); }
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      float2 m0[8], m1[8];
-      mask_sub<BITS>(w[0], b, m0);
-      mask_sub<BITS>(w[1], b, m1);
-#pragma unroll
-      for (int t = 0; t < kTT; ++t) {
-        if (t < nt) {
-          float2 xw[8];
-          xs_sub(hs_sm + t * I, lc, b, xw);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            acc[0][t] = __ffma2_rn(m0[i], xw[i], acc[0][t]);
-            acc[1][t] = __ffma2_rn(m1[i], xw[i], acc[1][t]);
-          }
+      const int ln = l + kSlots;
+      if (ln < nst) {
+        issue_step<MODE>(S, C, ki, ci, warp, lane, rw, rsb, pol);
+        if (++ci == cpl) {
+          ci = 0;
+          ++ki;
         }
+      } else if (ln >= nstp && ln - nstp < nstN) {
+        const int lN = ln - nstp, kN = lN / cpl;
+        issue_step<MODE>(N, C, kN, lN - kN * cpl, warp, lane, rw, rsb, pol);
       }
+      cp_async_commit();
     }
+  }
+  if (nstp == 0) {
+    // no steps here: the slots take N's first steps (the groups of the
+    // empty steps that were meant for S are complete)
 #pragma unroll
-    for (int t = 0; t < kTT; ++t) {
-      if (t < nt) {
-        const float hk = hk_sm[t], hsum = hsum_sm[t * (I / 32) + lc];
-        v[t] += sc[0] * hk * (acc[0][t].x + acc[0][t].y) + bi[0] * hsum;
-        v[kTT + t] += sc[1] * hk * (acc[1][t].x + acc[1][t].y) + bi[1] * hsum;
-      }
+    for (int j = 0; j < kSlots; ++j) {
+      unsigned char* rw = ring + j * (4 * 32 * 16);
+      uint32_t* rsb = (uint32_t*)(ring + kRingWords) + j * (4 * 2 * 32);
+      if (j < nstN) issue_step<MODE>(N, C, j / cpl, j % cpl, warp, lane, rw, rsb, pol);
+      cp_async_commit();
     }
   }
 }
 
-__global__ void __launch_bounds__(kGThreads, 1) grouped_down_kernel(const GroupedKParams p) {
+// Thread 0: the segment after `prev` (the next token pass of the same item,
+// else the first pass of the next item from the shared counter), with its
+// assignments and tokens.
+template <int MODE>
+static __device__ void next_segment(const GroupedKParams& p, const GSeg& prev, GSeg& out, int* asg, int* toks) {
+  int e = -1, t0 = 0;
+  GSeg s = prev;
+  if (prev.valid && prev.t0 + p.tile < p.count[prev.e]) {
+    e = prev.e;
+    t0 = prev.t0 + p.tile;
+  } else {
+    const int R = MODE == 0 ? p.I : p.H;
+    const int rows = MODE == 0 ? kRowsA : kRowsB;
+    const int ipe = (R + rows - 1) / rows;
+    const int n_tc = MODE == 0 ? p.ctl[3] : 0;  // experts done by the tensor-core kernel
+    const int n_items = (p.ctl[0] - n_tc) * ipe;
+    for (;;) {
+      const int item = atomicAdd(&p.ctl[MODE == 0 ? 1 : 2], 1);
+      if (item >= n_items) {
+        out.valid = 0;
+        return;
+      }
+      e = p.order[n_tc + item / ipe];
+      const qe_expert ex = p.experts[e];
+      const int bits = MODE == 0 ? ex.gate.bits : ex.down.bits;
+      const bool ok = (bits == 4 || bits == 2) &&
+                      (MODE == 0 ? qmat_ok(ex.gate, bits) && qmat_ok(ex.up, bits) && qmat_ok(ex.down, bits)
+                                 : qmat_ok(ex.down, bits));
+      if (!ok) {
+        set_error(p.err, QE_ERR_INVALID_ARG);
+        continue;
+      }
+      s.bits = bits;
+      s.r0 = (item % ipe) * rows;
+      s.nrows = min(rows, R - s.r0);
+      s.m0 = MODE == 0 ? ex.gate : ex.down;
+      s.m1 = ex.up;
+      break;
+    }
+  }
+  s.valid = 1;
+  s.e = e;
+  s.t0 = t0;
+  s.nt = min(p.tile, p.count[e] - t0);
+  const int base = p.start[e] + t0;
+  for (int t = 0; t < s.nt; ++t) {
+    const int a = p.list[base + t];
+    asg[t] = a;
+    toks[t] = a / p.K;
+  }
+  out = s;
+}
+
+// Stage the segment's token vectors in x' form (swizzled), their 32-column
+// sums and accumulator scales; padding tokens up to nt_pad(nt) are zero.
+template <int MODE>
+static __device__ void stage_segment(const GroupedKParams& p, const GSeg& s, const int* asg, const int* toks,
+                                     float* xs, float* sums, float* xk, int* hexp) {
+  const int ntp = nt_pad(s.nt), nt = s.nt;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (MODE == 0) {
+    const int H = p.H;
+    const float* src = s.bits == 4 ? p.xp4 : p.xp2;
+    for (int i = tid; i < ntp * (H / 4); i += kGThreads) {
+      const int t = i / (H / 4), c = (i - t * (H / 4)) * 4;
+      const float4 v = t < nt ? *(const float4*)(src + (size_t)toks[t] * H + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      *(float4*)(xs + t * H + xswz(c)) = v;  // global x' is in pair order; pieces move whole
+    }
+    for (int i = tid; i < ntp * (H / 32); i += kGThreads) {
+      const int t = i / (H / 32), c = i - t * (H / 32);
+      sums[i] = t < nt ? p.xsum[(size_t)toks[t] * (H / 32) + c] : 0.f;
+    }
+    if (tid < ntp) xk[tid] = tid < nt ? acc_scale(p.xexp[toks[tid]]) : 0.f;
+  } else {
+    const int I = p.I;
+    if (tid < ntp) {
+      const int Eh = tid < nt ? xscale_exponent(__uint_as_float(__ldcg(&p.hamax[asg[tid]]))) : 0;
+      hexp[tid] = Eh;
+      xk[tid] = tid < nt ? acc_scale(Eh) : 0.f;
+    }
+    __syncthreads();
+    for (int i = tid; i < ntp * I; i += kGThreads) {
+      const int t = i / I, c = i - t * I;
+      const float hv = t < nt ? __ldcg(p.h + (size_t)asg[t] * I + c) : 0.f;
+      xs[t * I + (s.bits == 4 ? swz_q4(c) : swz_q2(c))] =
+          s.bits == 4 ? xprime_q4(hv, c, hexp[t]) : xprime_q2(hv, c, hexp[t]);
+    }
+    for (int i = warp; i < ntp * (I / 32); i += kGWarps) {
+      const int t = i / (I / 32), ch = i - t * (I / 32);
+      const float sm = t < nt ? warp_sum(__ldcg(p.h + (size_t)asg[t] * I + ch * 32 + lane)) : 0.f;
+      if (lane == 0) sums[i] = sm;
+    }
+  }
+}
+
+template <int MODE, int BITS>
+static __device__ __forceinline__ void run_segment_nt(const GroupedKParams& p, const GSeg& S, const GSeg& N,
+                                                      const int* asg, int C, int cpl, const float* xs,
+                                                      const float* sums, const float* xk, unsigned* hmax,
+                                                      unsigned char* ring, int warp, int lane, uint64_t pol) {
+  const int ntp = nt_pad(S.nt);
+  if (ntp == 1) run_segment<MODE, BITS, 1>(p, S, N, asg, C, cpl, xs, sums, xk, hmax, ring, warp, lane, pol);
+  else if (ntp == 2) run_segment<MODE, BITS, 2>(p, S, N, asg, C, cpl, xs, sums, xk, hmax, ring, warp, lane, pol);
+  else run_segment<MODE, BITS, 4>(p, S, N, asg, C, cpl, xs, sums, xk, hmax, ring, warp, lane, pol);
+}
+
+// Dynamic shared memory: the warps' rings, then x' of `tile` tokens, their
+// 32-column sums and scales.
+static __host__ __device__ __forceinline__ size_t expert_smem(int C, int tile) {
+  return (size_t)kGWarps * kRingWarp + 4 * ((size_t)tile * C + al4(tile * (C / 32)) + al4(tile));
+}
+
+// MODE 0: gate/up (C = H columns); MODE 1: down (C = I columns).
+template <int MODE>
+__global__ void __launch_bounds__(kGThreads, 1) grouped_expert_kernel(const GroupedKParams p) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const int H = p.H, I = p.I, tile = p.tile;
+  const int C = MODE == 0 ? p.H : p.I;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* hs_sm = (float*)smem;                     // [tile][I] x' of h
-  float* hsum_sm = hs_sm + al4(tile * I);          // [tile][I/32]
-  float* hk_sm = hsum_sm + al4(tile * (I / 32));   // [tile]
-  int* asg = (int*)(hk_sm + al4(tile));            // [tile]
-  int* hexp = asg + al4(tile);                     // [tile]
-  __shared__ int s_item;
-  __shared__ qe_qmat s_d;
-  const int ipe = (H + kRowsB - 1) / kRowsB;
-  const int n_items = p.ctl[0] * ipe;
-  for (;;) {
-    if (threadIdx.x == 0) s_item = atomicAdd(&p.ctl[2], 1);
-    __syncthreads();
-    const int item = s_item;
-    if (item >= n_items) break;
-    const int e = p.order[item / ipe];
-    const int r0 = (item % ipe) * kRowsB, r1 = min(H, r0 + kRowsB);
-    if (threadIdx.x == 0) s_d = p.experts[e].down;
-    __syncthreads();
-    const int bits = s_d.bits;
-    if (!((bits == 4 || bits == 2) && qmat_ok(s_d, bits))) {
-      if (threadIdx.x == 0) set_error(p.err, QE_ERR_INVALID_ARG);
-      __syncthreads();
-      continue;
-    }
-    const int n = p.count[e], s0 = p.start[e];
-    for (int t0 = 0; t0 < n; t0 += tile) {
-      const int nt = min(tile, n - t0);
-      if (threadIdx.x < nt) {
-        const int a = p.list[s0 + t0 + threadIdx.x];
-        asg[threadIdx.x] = a;
-        const int Eh = xscale_exponent(__uint_as_float(__ldcg(&p.hamax[a])));
-        hexp[threadIdx.x] = Eh;
-        hk_sm[threadIdx.x] = acc_scale(Eh);
-      }
-      __syncthreads();
-      for (int i = threadIdx.x; i < nt * I; i += kGThreads) {
-        const int t = i / I, c = i - t * I;
-        const float hv = __ldcg(p.h + (size_t)asg[t] * I + c);
-        hs_sm[t * I + (bits == 4 ? swz_q4(c) : swz_q2(c))] =
-            bits == 4 ? xprime_q4(hv, c, hexp[t]) : xprime_q2(hv, c, hexp[t]);
-      }
-      for (int i = warp; i < nt * (I / 32); i += kGWarps) {
-        const int t = i / (I / 32), ch = i - t * (I / 32);
-        const float sm = warp_sum(__ldcg(p.h + (size_t)asg[t] * I + ch * 32 + lane));
-        if (lane == 0) hsum_sm[i] = sm;
-      }
-      __syncthreads();
-      for (int r = r0 + 2 * warp; r < r1; r += 2 * kGWarps) {
-        const int two = r + 1 < r1 ? 2 : 1;
-        float v[2 * kTT];
+  unsigned char* ring = smem + (size_t)warp * kRingWarp;
+  float* xs = (float*)(smem + (size_t)kGWarps * kRingWarp);  // [tile][C]
+  float* sums = xs + p.tile * C;                               // [tile][C/32]
+  float* xk = sums + al4(p.tile * (C / 32));                   // [tile]
+  __shared__ GSeg s_seg[2];
+  __shared__ int s_asg[2][kTile], s_tok[2][kTile], s_hexp[kTile];
+  __shared__ unsigned s_hmax[2][kTile];
+  const int cpl = (C / 32 + 31) / 32;  // chunks per lane and row
+  const uint64_t pol = policy_evict_first();
+  if (threadIdx.x == 0) {
+    GSeg none;
+    none.valid = 0;
+    next_segment<MODE>(p, none, s_seg[0], s_asg[0], s_tok[0]);
+    if (s_seg[0].valid) next_segment<MODE>(p, s_seg[0], s_seg[1], s_asg[1], s_tok[1]);
+    else s_seg[1].valid = 0;
+  }
+  __syncthreads();
+  {
+    const int nst = s_seg[0].valid ? seg_steps<MODE>(s_seg[0], warp, cpl) : 0;
 #pragma unroll
-        for (int t = 0; t < 2 * kTT; ++t) v[t] = 0.f;
-        if (bits == 4) down_rows<4>(s_d, r, two, I, nt, hs_sm, hsum_sm, hk_sm, v, lane);
-        else down_rows<2>(s_d, r, two, I, nt, hs_sm, hsum_sm, hk_sm, v, lane);
-        const float sv = warp_reduce_rows<2 * kTT>(v, lane);
-        const int row = reduced_row_of_lane<2 * kTT>(lane);
-        const int q = row / kTT, t = row - q * kTT;
-        if (t < nt && q < two && lane == lane_of_reduced_row<2 * kTT>(row))
-          p.y[(size_t)asg[t] * H + r + q] = sv;
-      }
-      __syncthreads();
+    for (int j = 0; j < kSlots; ++j) {
+      if (j < nst)
+        issue_step<MODE>(s_seg[0], C, j / cpl, j % cpl, warp, lane, ring + j * (4 * 32 * 16),
+                         (uint32_t*)(ring + kRingWords) + j * (4 * 2 * 32), pol);
+      cp_async_commit();
     }
   }
+  int cur = 0;
+  while (s_seg[cur].valid) {
+    const GSeg& S = s_seg[cur];
+    const GSeg& N = s_seg[cur ^ 1];
+    if (threadIdx.x < kTile) s_hmax[cur][threadIdx.x] = 0u;
+    stage_segment<MODE>(p, S, s_asg[cur], s_tok[cur], xs, sums, xk, s_hexp);
+    __syncthreads();
+    if (S.bits == 4)
+      run_segment_nt<MODE, 4>(p, S, N, s_asg[cur], C, cpl, xs, sums, xk, s_hmax[cur], ring, warp, lane, pol);
+    else
+      run_segment_nt<MODE, 2>(p, S, N, s_asg[cur], C, cpl, xs, sums, xk, s_hmax[cur], ring, warp, lane, pol);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      if (MODE == 0)
+        for (int t = 0; t < S.nt; ++t) atomicMax(&p.hamax[s_asg[cur][t]], s_hmax[cur][t]);
+      // the buffer of S takes the segment after N
+      if (N.valid) next_segment<MODE>(p, N, s_seg[cur], s_asg[cur], s_tok[cur]);
+      else s_seg[cur].valid = 0;
+    }
+    cur ^= 1;
+  }
+  cp_async_wait<0>();
 }
 
-static size_t gateup_smem(int H, int tile) {
-  return 4 * ((size_t)al4(tile * H) + al4(tile * (H / 32)) + 3 * (size_t)al4(tile));
-}
-
-static size_t down_smem(int I, int tile) {
-  return 4 * ((size_t)al4(tile * I) + al4(tile * (I / 32)) + 3 * (size_t)al4(tile));
-}
-
-// Largest token tile (<= kTT) whose buffers fit in shared memory.
-int grouped_tile(int H, int I, int smem_optin) {
-  for (int t = kTT; t >= 1; --t)
-    if (gateup_smem(H, t) <= (size_t)smem_optin && down_smem(I, t) <= (size_t)smem_optin) return t;
+// Largest token pass (4, 2 or 1) whose shared memory fits.
+static int expert_tile(int C, size_t avail) {
+  for (int t = kTile; t >= 1; t >>= 1)
+    if (expert_smem(C, t) <= avail) return t;
   return 0;
 }
 
@@ -474,37 +574,48 @@ cudaError_t launch_grouped(const GroupedParams& gp, cudaStream_t s) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (tc && (e = launch_tc_gateup(gp, ctl, gp.budget_ns, s)) != cudaSuccess) return e;
-  int dev = 0, sms = 148, optin = 0;
+  int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  cudaFuncAttributes fa{}, fb{};
-  if ((e = cudaFuncGetAttributes(&fa, grouped_gateup_kernel)) != cudaSuccess) return e;
-  if ((e = cudaFuncGetAttributes(&fb, grouped_down_kernel)) != cudaSuccess) return e;
-  // static shared memory counts against the per-block limit
-  const int avail = optin - (int)(fa.sharedSizeBytes > fb.sharedSizeBytes ? fa.sharedSizeBytes : fb.sharedSizeBytes);
+  static int attr_dev = -1;
+  static size_t avail = 0;
+  if (attr_dev != dev) {
+    int optin = 0;
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cudaFuncAttributes fa{}, fb{};
+    if ((e = cudaFuncGetAttributes(&fa, grouped_expert_kernel<0>)) != cudaSuccess) return e;
+    if ((e = cudaFuncGetAttributes(&fb, grouped_expert_kernel<1>)) != cudaSuccess) return e;
+    const size_t st = fa.sharedSizeBytes > fb.sharedSizeBytes ? fa.sharedSizeBytes : fb.sharedSizeBytes;
+    avail = (size_t)optin > st ? (size_t)optin - st : 0;
+    if ((e = cudaFuncSetAttribute(grouped_expert_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)avail)) != cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(grouped_expert_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)avail)) != cudaSuccess)
+      return e;
+    attr_dev = dev;
+  }
   GroupedKParams p{};
   p.H = gp.H; p.I = gp.I; p.K = gp.K; p.T = gp.T;
-  p.tile = grouped_tile(gp.H, gp.I, avail);
-  if (p.tile == 0) return cudaErrorInvalidConfiguration;
   p.experts = gp.experts;
   p.xp4 = gp.xp4; p.xp2 = gp.xp2; p.xsum = gp.xsum; p.xexp = gp.xexp;
   p.count = gp.grp_count; p.start = gp.grp_start; p.list = gp.grp_list; p.order = gp.grp_order; p.ctl = ctl;
   p.h = gp.h; p.hamax = gp.hamax; p.y = gp.y; p.err = gp.err;
-  static int attr_dev = -1;
-  if (attr_dev != dev) {
-    if ((e = cudaFuncSetAttribute(grouped_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, avail)) !=
-        cudaSuccess)
-      return e;
-    if ((e = cudaFuncSetAttribute(grouped_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, avail)) !=
-        cudaSuccess)
-      return e;
-    attr_dev = dev;
-  }
-  grouped_gateup_kernel<<<sms, kGThreads, gateup_smem(gp.H, p.tile), s>>>(p);
+  const int ta = expert_tile(gp.H, avail), tb = expert_tile(gp.I, avail);
+  if (ta == 0 || tb == 0) return cudaErrorInvalidConfiguration;
+  p.tile = ta;
+  grouped_expert_kernel<0><<<sms, kGThreads, expert_smem(gp.H, ta), s>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  grouped_down_kernel<<<sms, kGThreads, down_smem(gp.I, p.tile), s>>>(p);
+  p.tile = tb;
+  grouped_expert_kernel<1><<<sms, kGThreads, expert_smem(gp.I, tb), s>>>(p);
   return cudaGetLastError();
+}
+
+// Largest token pass of the gate/up kernel at these sizes.
+int grouped_tile(int H, int I, int smem_optin) {
+  const size_t a = (size_t)smem_optin;
+  const int ta = expert_tile(H, a), tb = expert_tile(I, a);
+  return ta < tb ? ta : tb;
 }
 
 }  // namespace qe
