@@ -158,14 +158,23 @@ struct GSeg {
 };
 
 // Per-warp ring of kSlots steps in shared memory.  A step is, for each lane,
-// the packed 32-column chunk of four matrix rows (16 bytes each; 8 at 2-bit)
-// and the 4-byte words holding the chunk's bf16 scale and bias in each row.
-// Layout [slot][row][lane] (words) and [slot][row][scale|bias][lane], so a
-// warp's accesses to one row fall on consecutive addresses.  Each lane reads
-// only what it copied itself.
+// the packed 32-column chunk of four matrix rows (16 bytes each; 8 at 2-bit,
+// layout [slot][row][lane], each lane reads what it copied) and the bf16
+// scales and biases of the step's groups.  When a row holds a multiple of 8
+// groups the scale/bias runs are 16-byte aligned and lanes 0..15 copy the
+// step's 16 groups of each row and array in one 16-byte copy each (layout
+// [slot][row][scale|bias][16 entries]); otherwise every lane copies the
+// 4-byte word holding its own group's entry ([slot][row][scale|bias][lane]).
 constexpr int kRingWords = kSlots * 4 * 32 * 16;
 constexpr int kRingSb = kSlots * 4 * 2 * 32 * 4;
 constexpr int kRingWarp = kRingWords + kRingSb;  // 9 KiB
+
+// Staged x' vectors keep each 32-column chunk in pair order and pad it to
+// 36 floats: lane L's chunk then starts 36 L floats in, so the eight
+// 16-byte pieces of a chunk are read at fixed offsets from one address and
+// the lanes of a quarter warp fall on distinct bank groups.
+constexpr int kXPad = 36;
+static __host__ __device__ __forceinline__ int xs_stride(int C) { return (C / 32) * kXPad; }
 
 // Token-pass width for nt live tokens: 1, 2 or 4.
 static __host__ __device__ __forceinline__ int nt_pad(int nt) { return nt <= 1 ? 1 : (nt <= 2 ? 2 : 4); }
@@ -195,25 +204,36 @@ static __device__ __forceinline__ int unit_row(const GSeg& s, int q, int m) {
 // commits the group.
 template <int MODE>
 static __device__ __forceinline__ void issue_step(const GSeg& s, int C, int k, int c, int warp, int lane,
-                                                  unsigned char* rw, uint32_t* rsb, uint64_t pol) {
+                                                  unsigned char* rw, uint32_t* rsb, bool coop, uint64_t pol) {
   const int q = warp + kGWarps * k;
   const int lc = 32 * c + lane;
-  if (lc >= C / 32) return;
   const int bits = s.bits;
   const size_t rowb = (size_t)C * bits / 8;
   const int gpr = C / kGroup;
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
+  for (int m = 0; m < 4 && lc < C / 32; ++m) {
     const qe_qmat& mat = (MODE == 0 && m >= 2) ? s.m1 : s.m0;
     const int row = unit_row<MODE>(s, q, m);
     const unsigned char* rp = (const unsigned char*)mat.wq + (size_t)row * rowb;
     if (bits == 4) cp_async16(rw + (m * 32 + lane) * 16, rp + (size_t)lc * 16, pol);
     else cp_async8(rw + (m * 32 + lane) * 16, rp + (size_t)lc * 8, pol);
-    // the 4-byte word holding group gi's entry (gi rounded down to even; the
-    // arrays hold an even number of entries, so the word is in bounds)
-    const size_t gi2 = ((size_t)row * gpr + (lc >> 1)) & ~(size_t)1;
-    cp_async4(rsb + (m * 2 + 0) * 32 + lane, mat.scales + gi2);
-    cp_async4(rsb + (m * 2 + 1) * 32 + lane, mat.biases + gi2);
+    if (!coop) {
+      // the 4-byte word holding group gi's entry (gi rounded down to even;
+      // the arrays hold an even number of entries, so the word is in bounds)
+      const size_t gi2 = ((size_t)row * gpr + (lc >> 1)) & ~(size_t)1;
+      cp_async4(rsb + (m * 2 + 0) * 32 + lane, mat.scales + gi2);
+      cp_async4(rsb + (m * 2 + 1) * 32 + lane, mat.biases + gi2);
+    }
+  }
+  if (coop && lane < 16) {
+    // piece lane = (row m, array a, half h): groups 16c + 8h .. +7 of row m
+    const int m = lane >> 2, a = (lane >> 1) & 1, h = lane & 1;
+    const int g0 = 16 * c + 8 * h;
+    if (g0 < gpr) {
+      const qe_qmat& mat = (MODE == 0 && m >= 2) ? s.m1 : s.m0;
+      const uint16_t* src = (a ? mat.biases : mat.scales) + (size_t)unit_row<MODE>(s, q, m) * gpr + g0;
+      cp_async16((unsigned char*)rsb + (m * 2 + a) * 32 + h * 16, src, pol);
+    }
   }
 }
 
@@ -237,22 +257,24 @@ static __device__ __forceinline__ void piece_masks(const ulonglong2 w, int i, fl
 }
 
 // One step: chunk lc of the four matrix rows in ring slot (rw, rsb) against
-// the NT staged token vectors (x' swizzled, [NT][C]); v[m*NT + t] gets row m,
-// token t.  par[m] = parity of the chunk's group index in row m (which half
-// of the copied 4-byte scale/bias word is the chunk's).
+// the NT staged token vectors (x' padded, [NT][xs_stride(C)]); v[m*NT + t]
+// gets row m, token t.  par[m] = parity of the chunk's group index in row m
+// (which half of the copied 4-byte scale/bias word is the chunk's; per-lane
+// copies only).
 template <int BITS, int NT>
 static __device__ __forceinline__ void compute_step(const unsigned char* rw, const uint32_t* rsb, const int (&par)[4],
-                                                    const float* xs, const float* sums, const float* xk, int C,
-                                                    int lc, int lane, float (&v)[4 * NT]) {
+                                                    bool coop, const float* xs, const float* sums, const float* xk,
+                                                    int C, int lc, int lane, float (&v)[4 * NT]) {
   const int nch = C / 32;
   if (lc >= nch) return;
   ulonglong2 w[4];
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
+    const unsigned char* src = rw + (m * 32 + lane) * 16;
     if (BITS == 4) {
-      w[m] = *(const ulonglong2*)(rw + (m * 32 + lane) * 16);
+      w[m] = *(const ulonglong2*)src;
     } else {
-      w[m].x = *(const unsigned long long*)(rw + (m * 32 + lane) * 16);
+      w[m].x = *(const unsigned long long*)src;
       w[m].y = 0ull;
     }
   }
@@ -261,13 +283,13 @@ static __device__ __forceinline__ void compute_step(const unsigned char* rw, con
   for (int m = 0; m < 4; ++m)
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[m][t] = make_float2(0.f, 0.f);
-  const float4* xb = (const float4*)(xs + lc * 32);
-  const int sw = lc & 7;
+  const float4* xb = (const float4*)(xs + lc * kXPad);
+  const int ts = xs_stride(C) / 4;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     float4 xp[NT];
 #pragma unroll
-    for (int t = 0; t < NT; ++t) xp[t] = xb[t * (C / 4) + (i ^ sw)];
+    for (int t = 0; t < NT; ++t) xp[t] = xb[t * ts + i];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       float2 m0, m1;
@@ -281,9 +303,16 @@ static __device__ __forceinline__ void compute_step(const unsigned char* rw, con
   }
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    const uint32_t sw2 = rsb[(m * 2 + 0) * 32 + lane], bw2 = rsb[(m * 2 + 1) * 32 + lane];
-    const float sc = __uint_as_float(par[m] ? (sw2 & 0xFFFF0000u) : (sw2 << 16));
-    const float bi = __uint_as_float(par[m] ? (bw2 & 0xFFFF0000u) : (bw2 << 16));
+    float sc, bi;
+    if (coop) {
+      const uint16_t* e = (const uint16_t*)rsb + (m * 2) * 16 + ((lc >> 1) & 15);
+      sc = __uint_as_float((uint32_t)e[0] << 16);
+      bi = __uint_as_float((uint32_t)e[16] << 16);
+    } else {
+      const uint32_t sw2 = rsb[(m * 2 + 0) * 32 + lane], bw2 = rsb[(m * 2 + 1) * 32 + lane];
+      sc = __uint_as_float(par[m] ? (sw2 & 0xFFFF0000u) : (sw2 << 16));
+      bi = __uint_as_float(par[m] ? (bw2 & 0xFFFF0000u) : (bw2 << 16));
+    }
 #pragma unroll
     for (int t = 0; t < NT; ++t)
       v[m * NT + t] += sc * xk[t] * (acc[m][t].x + acc[m][t].y) + bi * sums[t * nch + lc];
@@ -330,6 +359,7 @@ static __device__ __forceinline__ void run_segment(const GroupedKParams& p, cons
   const int nstp = (nst + kSlots - 1) / kSlots * kSlots;
   const int nstN = N.valid ? seg_steps<MODE>(N, warp, cpl) : 0;
   const int gpr = C / kGroup;
+  const bool coop = (gpr & 7) == 0;
   float v[4 * NT];
 #pragma unroll
   for (int i = 0; i < 4 * NT; ++i) v[i] = 0.f;
@@ -342,12 +372,13 @@ static __device__ __forceinline__ void run_segment(const GroupedKParams& p, cons
       uint32_t* rsb = (uint32_t*)(ring + kRingWords) + j * (4 * 2 * 32);
       const int l = l0 + j;
       cp_async_wait<kSlots - 1>();
+      __syncwarp();  // the slot's shared scale/bias copies are visible to every lane
       if (l < nst) {
         const int q = warp + kGWarps * kc, lc = 32 * cc + lane;
         int par[4];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) par[m] = (unit_row<MODE>(S, q, m) * gpr + (lc >> 1)) & 1;
-        compute_step<BITS, NT>(rw, rsb, par, xs, sums, xk, C, lc, lane, v);
+        for (int m = 0; m < 4; ++m) par[m] = coop ? 0 : (unit_row<MODE>(S, q, m) * gpr + (lc >> 1)) & 1;
+        compute_step<BITS, NT>(rw, rsb, par, coop, xs, sums, xk, C, lc, lane, v);
         if (cc == cpl - 1) {
           unit_epilogue<MODE, NT>(p, S, asg, q, v, hmax, lane);
 #pragma unroll
@@ -359,15 +390,16 @@ static __device__ __forceinline__ void run_segment(const GroupedKParams& p, cons
         }
       }
       const int ln = l + kSlots;
+      __syncwarp();  // every lane is done with the slot before it is refilled
       if (ln < nst) {
-        issue_step<MODE>(S, C, ki, ci, warp, lane, rw, rsb, pol);
+        issue_step<MODE>(S, C, ki, ci, warp, lane, rw, rsb, coop, pol);
         if (++ci == cpl) {
           ci = 0;
           ++ki;
         }
       } else if (ln >= nstp && ln - nstp < nstN) {
         const int lN = ln - nstp, kN = lN / cpl;
-        issue_step<MODE>(N, C, kN, lN - kN * cpl, warp, lane, rw, rsb, pol);
+        issue_step<MODE>(N, C, kN, lN - kN * cpl, warp, lane, rw, rsb, coop, pol);
       }
       cp_async_commit();
     }
@@ -379,7 +411,7 @@ static __device__ __forceinline__ void run_segment(const GroupedKParams& p, cons
     for (int j = 0; j < kSlots; ++j) {
       unsigned char* rw = ring + j * (4 * 32 * 16);
       uint32_t* rsb = (uint32_t*)(ring + kRingWords) + j * (4 * 2 * 32);
-      if (j < nstN) issue_step<MODE>(N, C, j / cpl, j % cpl, warp, lane, rw, rsb, pol);
+      if (j < nstN) issue_step<MODE>(N, C, j / cpl, j % cpl, warp, lane, rw, rsb, coop, pol);
       cp_async_commit();
     }
   }
@@ -451,7 +483,7 @@ static __device__ void stage_segment(const GroupedKParams& p, const GSeg& s, con
     for (int i = tid; i < ntp * (H / 4); i += kGThreads) {
       const int t = i / (H / 4), c = (i - t * (H / 4)) * 4;
       const float4 v = t < nt ? *(const float4*)(src + (size_t)toks[t] * H + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-      *(float4*)(xs + t * H + xswz(c)) = v;  // global x' is in pair order; pieces move whole
+      *(float4*)(xs + t * xs_stride(H) + (c >> 5) * kXPad + (c & 31)) = v;  // pair order; pieces move whole
     }
     for (int i = tid; i < ntp * (H / 32); i += kGThreads) {
       const int t = i / (H / 32), c = i - t * (H / 32);
@@ -469,7 +501,8 @@ static __device__ void stage_segment(const GroupedKParams& p, const GSeg& s, con
     for (int i = tid; i < ntp * I; i += kGThreads) {
       const int t = i / I, c = i - t * I;
       const float hv = t < nt ? __ldcg(p.h + (size_t)asg[t] * I + c) : 0.f;
-      xs[t * I + (s.bits == 4 ? swz_q4(c) : swz_q2(c))] =
+      const int pos = s.bits == 4 ? xperm_q4(c) : xperm_q2(c);
+      xs[t * xs_stride(I) + (pos >> 5) * kXPad + (pos & 31)] =
           s.bits == 4 ? xprime_q4(hv, c, hexp[t]) : xprime_q2(hv, c, hexp[t]);
     }
     for (int i = warp; i < ntp * (I / 32); i += kGWarps) {
@@ -494,7 +527,7 @@ static __device__ __forceinline__ void run_segment_nt(const GroupedKParams& p, c
 // Dynamic shared memory: the warps' rings, then x' of `tile` tokens, their
 // 32-column sums and scales.
 static __host__ __device__ __forceinline__ size_t expert_smem(int C, int tile) {
-  return (size_t)kGWarps * kRingWarp + 4 * ((size_t)tile * C + al4(tile * (C / 32)) + al4(tile));
+  return (size_t)kGWarps * kRingWarp + 4 * ((size_t)tile * xs_stride(C) + al4(tile * (C / 32)) + al4(tile));
 }
 
 // MODE 0: gate/up (C = H columns); MODE 1: down (C = I columns).
@@ -504,8 +537,8 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_expert_kernel(const Grou
   const int C = MODE == 0 ? p.H : p.I;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* ring = smem + (size_t)warp * kRingWarp;
-  float* xs = (float*)(smem + (size_t)kGWarps * kRingWarp);  // [tile][C]
-  float* sums = xs + p.tile * C;                               // [tile][C/32]
+  float* xs = (float*)(smem + (size_t)kGWarps * kRingWarp);  // [tile][xs_stride(C)]
+  float* sums = xs + p.tile * xs_stride(C);                    // [tile][C/32]
   float* xk = sums + al4(p.tile * (C / 32));                   // [tile]
   __shared__ GSeg s_seg[2];
   __shared__ int s_asg[2][kTile], s_tok[2][kTile], s_hexp[kTile];
@@ -526,7 +559,7 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_expert_kernel(const Grou
     for (int j = 0; j < kSlots; ++j) {
       if (j < nst)
         issue_step<MODE>(s_seg[0], C, j / cpl, j % cpl, warp, lane, ring + j * (4 * 32 * 16),
-                         (uint32_t*)(ring + kRingWords) + j * (4 * 2 * 32), pol);
+                         (uint32_t*)(ring + kRingWords) + j * (4 * 2 * 32), ((C / kGroup) & 7) == 0, pol);
       cp_async_commit();
     }
   }
