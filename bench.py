@@ -428,7 +428,8 @@ def run_ours(args, wl, rank, world, local_rank):
     achieved = alg / per_step_s / 1e9
     peak = float(peaks["hbm_gbs"])
     cpu = None if args.no_cpu_baseline else cpu_baseline(wl, seed)
-    kern = "qe_fused_layer_kernel" if T == 1 else "grouped_gateup_kernel + grouped_down_kernel (+ route, group, combine)"
+    kern = ("qe_fused_layer_kernel" if T == 1 else
+            "grouped_expert_kernel<0> (gate/up) + grouped_expert_kernel<1> (down) (+ route, group, combine)")
     line = {
         "metric": wl["metric"], "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
@@ -449,7 +450,9 @@ def run_ours(args, wl, rank, world, local_rank):
                 "d2h_bytes_per_step": T * H * 4, "steps": n_e2e,
                 "how": "per step: moe_layer_step_host on pinned host buffers (H2D of x, layer step, D2H of "
                        "out, stream sync)"},
-        "gpu_launches": args.steps * (1 if T == 1 else 6),
+        # T == 1: the fused kernel; else route norm, logits, top-K, grouping,
+        # gate/up, down and combine
+        "gpu_launches": args.steps * (1 if T == 1 else 7),
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -767,7 +767,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
 // ------------------------------------------------------------ host side
 
 static int align_up(int v, int a) { return (v + a - 1) / a * a; }
-static int gcd_int(int a, int b) { while (b) { int t = a % b; a = b; b = t; } return a; }
 
 int fused_geometry(int H, int E, int K, int I, int sms, int smem_optin, FusedGeometry* out) {
   FusedGeometry g{};

@@ -1,12 +1,15 @@
 // qe_route.cu -- RMSNorm + router + top-K for T tokens (moe_route and the
 // batched layer step).  Norm and router logits are evaluated in double
 // precision so the expert choice is an fp64 decision.
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 #include <math.h>
 
 #include "qe_device.cuh"
 
 namespace qe {
+
+namespace cg = cooperative_groups;
 
 // One CTA per token: two-pass RMSNorm; x*gamma (fp64) for the router; xn
 // (fp32) and, if requested, x' for the expert matvecs with its 32-column sums.
@@ -99,49 +102,100 @@ __global__ void __launch_bounds__(256) route_logits_gemv_kernel(const RouteParam
   }
 }
 
-// Router logits for many tokens: fp64 tiled product, 32 experts x 32
-// tokens per CTA (enough CTAs to cover the SMs), 2x2 outputs per thread,
-// 32-column steps through shared memory with float4 loads of W.
-constexpr int kRT = 32, kRK = 32;
-__global__ void __launch_bounds__(256) route_logits_tiled_kernel(const RouteParams p) {
-  __shared__ __align__(16) double sW[kRK][kRT + 2];
-  __shared__ __align__(16) double sX[kRK][kRT + 2];
+// Router logits for many tokens: fp64 tiled product.  A CTA takes a tile of
+// 64 experts x 64 tokens and one eighth of the hidden columns; the eight
+// CTAs of a thread-block cluster take the eight eighths of the same tile and
+// add their partial tiles through distributed shared memory, in rank order,
+// so the result does not depend on timing.  Each thread keeps 4 x 4 partial
+// sums; columns come in 32-wide chunks, loaded into registers one chunk
+// ahead and staged in shared memory (W converted to fp64), transposed to
+// [k][expert] and [k][token] with the row index XOR-ed by rsw(k) (a multiple
+// of 4): the transposing stores spread over the banks and the compute reads
+// of four consecutive rows stay contiguous.
+constexpr int kRT = 64;     // experts and tokens per tile
+constexpr int kRK = 32;     // columns per chunk
+constexpr int kRSplit = 8;  // CTAs per cluster (column eighths)
+static __device__ __forceinline__ int rsw(int k) { return ((k >> 2) & 3) << 2; }
+__global__ void __cluster_dims__(kRSplit, 1, 1) __launch_bounds__(256)
+    route_logits_tiled_kernel(const RouteParams p) {
+  __shared__ __align__(16) double sbuf[2 * kRK * kRT];  // sW [k][e], sX [k][t]; later the partial tile [t][e]
+  double* sW = sbuf;
+  double* sX = sbuf + kRK * kRT;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
   const int H = p.H, E = p.E, T = p.T;
-  const int e0 = blockIdx.x * kRT, t0 = blockIdx.y * kRT;
+  const int tiles_e = (E + kRT - 1) / kRT;
+  const int tile = blockIdx.x / kRSplit;
+  const int e0 = (tile % tiles_e) * kRT, t0 = (tile / tiles_e) * kRT;
+  const int nch = H / kRK;  // H is a multiple of 64
+  const int ch0 = rank * nch / kRSplit, ch1 = (rank + 1) * nch / kRSplit;
   const int tid = threadIdx.x;
-  const int te = (tid & 15) * 2, tt = (tid >> 4) * 2;
-  double acc[2][2] = {};
-  for (int c0 = 0; c0 < H; c0 += kRK) {
-    // 32 rows x 32 columns of W (fp32 -> fp64) and of x*gamma (fp64)
-    {
-      const int r = tid >> 3, c4 = (tid & 7) * 4;
-      const int e = e0 + r, t = t0 + r;
-      if (e < E) {
-        const float4 v = *(const float4*)(p.router_w + (size_t)e * H + c0 + c4);
-        sW[c4][r] = v.x; sW[c4 + 1][r] = v.y; sW[c4 + 2][r] = v.z; sW[c4 + 3][r] = v.w;
-      } else {
-        sW[c4][r] = 0.0; sW[c4 + 1][r] = 0.0; sW[c4 + 2][r] = 0.0; sW[c4 + 3][r] = 0.0;
-      }
-      for (int u = 0; u < 4; ++u) sX[c4 + u][r] = t < T ? p.xg[(size_t)t * H + c0 + c4 + u] : 0.0;
+  const int te = (tid & 15) * 4, tt = (tid >> 4) * 4;
+  double acc[4][4] = {};
+  float4 wn[2];
+  double2 xn[4];
+  auto fetch = [&](int ch) {
+    const int k0 = ch * kRK;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int u = tid + 256 * j, r = u >> 3, c4 = (u & 7) * 4;
+      wn[j] = e0 + r < E ? __ldg((const float4*)(p.router_w + (size_t)(e0 + r) * H + k0 + c4))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int u = tid + 256 * j, r = u >> 4, c2 = (u & 15) * 2;
+      xn[j] = t0 + r < T ? *(const double2*)(p.xg + (size_t)(t0 + r) * H + k0 + c2) : make_double2(0.0, 0.0);
+    }
+  };
+  if (ch0 < ch1) fetch(ch0);
+  for (int ch = ch0; ch < ch1; ++ch) {
+    __syncthreads();  // the previous chunk is consumed
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int u = tid + 256 * j, r = u >> 3, c4 = (u & 7) * 4;
+      sW[(c4 + 0) * kRT + (r ^ rsw(c4 + 0))] = wn[j].x;
+      sW[(c4 + 1) * kRT + (r ^ rsw(c4 + 1))] = wn[j].y;
+      sW[(c4 + 2) * kRT + (r ^ rsw(c4 + 2))] = wn[j].z;
+      sW[(c4 + 3) * kRT + (r ^ rsw(c4 + 3))] = wn[j].w;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int u = tid + 256 * j, r = u >> 4, c2 = (u & 15) * 2;
+      sX[(c2 + 0) * kRT + (r ^ rsw(c2 + 0))] = xn[j].x;
+      sX[(c2 + 1) * kRT + (r ^ rsw(c2 + 1))] = xn[j].y;
     }
     __syncthreads();
-#pragma unroll 8
-    for (int c = 0; c < kRK; ++c) {
-      const double w0 = sW[c][te], w1 = sW[c][te + 1];
-      const double x0 = sX[c][tt], x1 = sX[c][tt + 1];
-      acc[0][0] = fma(w0, x0, acc[0][0]);
-      acc[0][1] = fma(w0, x1, acc[0][1]);
-      acc[1][0] = fma(w1, x0, acc[1][0]);
-      acc[1][1] = fma(w1, x1, acc[1][1]);
+    if (ch + 1 < ch1) fetch(ch + 1);
+#pragma unroll 4
+    for (int k = 0; k < kRK; ++k) {
+      const int we = te ^ rsw(k), xt = tt ^ rsw(k);
+      const double2 wa = *(const double2*)(sW + k * kRT + we), wb = *(const double2*)(sW + k * kRT + we + 2);
+      const double2 xa = *(const double2*)(sX + k * kRT + xt), xb = *(const double2*)(sX + k * kRT + xt + 2);
+      const double w[4] = {wa.x, wa.y, wb.x, wb.y}, x[4] = {xa.x, xa.y, xb.x, xb.y};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fma(w[i], x[j], acc[i][j]);
     }
-    __syncthreads();
   }
-  for (int a = 0; a < 2; ++a)
-    for (int b = 0; b < 2; ++b) {
-      const int e = e0 + te + a, t = t0 + tt + b;
-      if (e < E && t < T)
-        p.logits[(size_t)t * E + e] = acc[a][b] * p.rinv[t] + (p.offset ? (double)p.offset[e] : 0.0);
-    }
+  __syncthreads();
+  double* part = sbuf;  // [t][e] partial tile of this CTA's columns
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) part[(tt + j) * kRT + te + i] = acc[i][j];
+  cluster.sync();
+  // rank r adds the partials of token rows [8r, 8r + 8)
+  for (int u = tid; u < kRT * kRT / kRSplit; u += 256) {
+    const int tl = rank * (kRT / kRSplit) + u / kRT, el = u % kRT;
+    double sum = 0.0;
+#pragma unroll
+    for (int q = 0; q < kRSplit; ++q) sum += cluster.map_shared_rank(part, q)[tl * kRT + el];
+    const int t = t0 + tl, e = e0 + el;
+    if (t < T && e < E) p.logits[(size_t)t * E + e] = sum * p.rinv[t] + (p.offset ? (double)p.offset[e] : 0.0);
+  }
+  cluster.sync();  // no CTA leaves while another still reads its partial tile
 }
 
 // Top-K + renormalised softmax weights: one warp per token.
@@ -188,8 +242,8 @@ cudaError_t launch_route(const RouteParams& p, cudaStream_t s) {
     const int blocks = (p.E * 32 + 255) / 256;
     route_logits_gemv_kernel<<<blocks, 256, 0, s>>>(p);
   } else {
-    dim3 grid((p.E + kRT - 1) / kRT, (p.T + kRT - 1) / kRT);
-    route_logits_tiled_kernel<<<grid, 256, 0, s>>>(p);
+    const int tiles = ((p.E + kRT - 1) / kRT) * ((p.T + kRT - 1) / kRT);
+    route_logits_tiled_kernel<<<tiles * kRSplit, 256, 0, s>>>(p);
   }
   route_topk_kernel<<<(p.T * 32 + 255) / 256, 256, 0, s>>>(p);
   return cudaGetLastError();
