@@ -21,11 +21,14 @@
 //                   x' form -> y[assignment][H]
 //   combine       : out[t] = sum_k w[t,k] y[t*K+k] (+ x[t])
 //
-// The expert kernels are bound by the bytes they stream, so each warp keeps
-// kSlots steps of packed words in flight in registers: the slot of a step is
-// refilled with the step kSlots ahead as soon as it has been used, and at the
-// end of a segment the refills already fetch the next segment's first steps,
-// so the loads run across the staging of the next segment's activations.
+// Each warp streams its packed words through a ring of kSlots steps in shared
+// memory, filled by asynchronous copies with one commit group per step: the
+// slot of a step is refilled with the step kSlots ahead as soon as it has
+// been used, and at the end of a segment the refills already fetch the next
+// segment's first steps, so the loads run across the staging of the next
+// segment's activations.  With the loads hidden, the kernels are bound by
+// instruction issue (one mask per weight, one multiply-add per weight and
+// token), not by the bytes they stream.
 #include <math.h>
 
 #include "qe_device.cuh"
@@ -642,13 +645,6 @@ cudaError_t launch_grouped(const GroupedParams& gp, cudaStream_t s) {
   p.tile = tb;
   grouped_expert_kernel<1><<<sms, kGThreads, expert_smem(gp.I, tb), s>>>(p);
   return cudaGetLastError();
-}
-
-// Largest token pass of the gate/up kernel at these sizes.
-int grouped_tile(int H, int I, int smem_optin) {
-  const size_t a = (size_t)smem_optin;
-  const int ta = expert_tile(H, a), tb = expert_tile(I, a);
-  return ta < tb ? ta : tb;
 }
 
 }  // namespace qe

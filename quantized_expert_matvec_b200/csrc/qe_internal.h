@@ -180,7 +180,6 @@ cudaError_t launch_grouped(const GroupedParams& p, cudaStream_t s);
 bool tc_eligible(int H, int I);
 int tc_min_tokens();
 cudaError_t launch_tc_gateup(const GroupedParams& gp, int* ctl, unsigned long long budget_ns, cudaStream_t s);
-int grouped_tile(int H, int I, int smem_optin);
 
 
 // ---- shared host helpers (qe_abi.cu)
