@@ -38,8 +38,8 @@ namespace qe {
 constexpr int kGWarps = 16;
 constexpr int kGThreads = kGWarps * 32;
 constexpr int kTile = 4;     // tokens sharing one pass over the weights
-constexpr int kRowsA = 128;  // gate/up rows (of gate and of up) per item
-constexpr int kRowsB = 512;  // down rows per item
+constexpr int kRowsA = 256;  // gate/up rows (of gate and of up) per item
+constexpr int kRowsB = 1024; // down rows per item
 constexpr int kSlots = 3;    // steps of packed words in flight per warp
 constexpr bool kTcEnabled = false;  // see launch_grouped
 
