@@ -206,9 +206,11 @@ QE_API int moe_combine(const float* y, const float* w, const float* residual, in
  * (+ x[t] if add_residual).  x [T,H] device fp32 or bf16 (x_dtype); out
  * [T,H] fp32 device (must not alias x); topk_idx/topk_w [T,K] device outputs
  * or NULL.  For T == 1 this is one persistent kernel covering the router,
- * the K experts and the combine.  For T > 1 the tokens are one batch:
- * assignments are grouped per expert so each selected expert's weights are
- * read once per step. */
+ * the K experts and the combine (a shape whose shared-memory plan does not
+ * fit that kernel, such as hidden 8192, takes the batched path).  For T > 1
+ * the tokens are one batch: assignments are grouped per expert, and each
+ * selected expert's weights are read once per pass over up to 4 of its
+ * tokens. */
 QE_API int moe_layer_step(const qe_cfg* cfg, const qe_layer* layer, const void* x, int x_dtype, int T,
                    float* out, int add_residual, int32_t* topk_idx, float* topk_w, void* dev_ws,
                    size_t ws_bytes, qe_stream_t stream);
