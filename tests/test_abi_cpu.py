@@ -127,3 +127,16 @@ def test_host_buffer_step_arguments_checked_first(q):
                                    None) == q.QE_ERR_INVALID_ARG
     assert "workspace" in q.qe_last_error()
     assert lib.moe_layer_step_host(ctypes.byref(cfg), ctypes.byref(layer), buf, 0, 0, buf, 0, None, 0, None) == q.QE_OK
+
+
+def test_build_script_loads_without_the_library():
+    """A fresh checkout has no libqexpert.so, and importing the package needs
+    it: the build entry point must reach the build script without importing
+    the package."""
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import sys, __graft_entry__ as g; b = g._library_builder(); "
+            "assert callable(b.build) and b.sources(), 'no build()'; "
+            "assert 'quantized_expert_matvec_b200' not in sys.modules, 'package imported'; print('ok')")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
