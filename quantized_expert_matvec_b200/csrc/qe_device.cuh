@@ -1,5 +1,5 @@
 // qe_device.cuh -- device building blocks of the sm_100a kernels:
-// bf16 decode, bounded waits, mbarrier / bulk-copy wrappers and the
+// bf16 decode, bounded waits, mbarrier and asynchronous-copy wrappers and the
 // dequant-dot cores of the 4-bit and 2-bit matvecs.
 #pragma once
 
@@ -89,12 +89,6 @@ QE_DEV void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-QE_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
 QE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -117,7 +111,7 @@ QE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t deadline, volatil
   return true;
 }
 
-// ------------------------------------------------------------ bulk copies
+// ---------------------------------------------------- asynchronous copies
 
 // L2 policy: streamed expert weights are read once per token, so they are
 // marked evict-first and do not push the router or activations out of L2.
@@ -127,22 +121,13 @@ QE_DEV uint64_t policy_evict_first() {
   return pol;
 }
 
-// Global -> shared bulk copy (no tensor map, no multicast); completion is
-// counted in bytes on `bar`.  dst, src and bytes must be 16-byte multiples.
-QE_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
-      : "memory");
-}
-
 // 16-byte asynchronous global -> shared copy (LDGSTS), L2 evict-first.
 QE_DEV void cp_async16(void* dst, const void* src, uint64_t pol) {
   asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
                "l"(pol)
                : "memory");
 }
+
 // 8- and 4-byte asynchronous copies (cached form; dst and src aligned to the size).
 QE_DEV void cp_async8(void* dst, const void* src, uint64_t pol) {
   asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 8, %2;" ::"r"(smem_u32(dst)), "l"(src),
