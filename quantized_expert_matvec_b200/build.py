@@ -33,11 +33,9 @@ def build(verbose: bool = False, ptxas_info: bool = False) -> str:
     srcs = sources()
     objs = [os.path.join(BUILD, os.path.basename(s)[:-3] + ".o") for s in srcs]
 
-    extra = os.environ.get("QE_NVCC_EXTRA", "").split()  # e.g. -DQE_TC_DEBUG for a diagnostic build
-
     def compile_one(src_obj):
         src, obj = src_obj
-        cmd = ["nvcc", *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
+        cmd = ["nvcc", *NVCC_FLAGS, "-c", src, "-o", obj]
         if ptxas_info:
             cmd += ["-Xptxas", "-v"]
         if verbose:

@@ -58,22 +58,7 @@ struct TcParams {
   unsigned* hamax;     // [T*K]
   int* err;
   unsigned long long budget_ns;
-  unsigned* dbg;  // diagnostic builds only: per-CTA progress in host-mapped memory
 };
-
-// Diagnostic builds (-DQE_TC_DEBUG) record each CTA's progress in host-mapped
-// memory, which stays readable on the host whatever happens on the device.
-#ifdef QE_TC_DEBUG
-#define TC_DBG(slot, v)                                                                   \
-  do {                                                                                    \
-    if (threadIdx.x == 0 && p.dbg) {                                                      \
-      *(volatile unsigned*)&p.dbg[blockIdx.x * 8 + (slot)] = (unsigned)(v);               \
-      __threadfence_system();                                                             \
-    }                                                                                     \
-  } while (0)
-#else
-#define TC_DBG(slot, v) do {} while (0)
-#endif
 
 // Offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled K-major tile.
 static __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
@@ -226,14 +211,12 @@ static __device__ void tc_item(const TcParams& p, const qe_expert& ex, int r0, c
     for (int o = 0; o < gpr * 2; o += 128) prefetch_l2((const unsigned char*)(base + (size_t)(r0 + rr) * gpr) + o);
   }
 
-  TC_DBG(2, 0x10000u | (unsigned)nt);
   const int pre = nkb < kTcRing - 1 ? nkb : kTcRing - 1;
   for (int kb = 0; kb < pre; ++kb) issue(kb);
   float sb[4], sbn[4];
   load_sb(0, sb);
   bool ok = true;
   for (int kb = 0; kb < nkb && ok; ++kb) {
-    TC_DBG(3, 0x100000u | (unsigned)kb);
     const int issued = kb + 3 < nkb ? kb + 3 : nkb;  // blocks whose copies are committed
     const int later = issued - kb - 1;
     if (later >= 2) cp_async_wait<2>();
@@ -249,7 +232,6 @@ static __device__ void tc_item(const TcParams& p, const qe_expert& ex, int r0, c
     tc_dequant<BITS>(st + kTcBTile + kTcPk + r * PB, r, hf, sb[2], sb[3], ag + kTcATile);
     fence_proxy_async_smem();
     __syncthreads();
-    TC_DBG(3, 0x200000u | (unsigned)kb);
     if (tid == 0) {
       tc_fence_after();
       const uint32_t sa = smem_u32(ag), sbt = smem_u32(st);
@@ -261,7 +243,6 @@ static __device__ void tc_item(const TcParams& p, const qe_expert& ex, int r0, c
       }
       tc_commit(&mma_done[kb & 1]);
     }
-    TC_DBG(3, 0x300000u | (unsigned)kb);
     ++ncommit[kb & 1];
     // block kb-1's MMAs done: its ring stage and A tile pair may be reused
     if (kb >= 1) {
@@ -289,7 +270,6 @@ static __device__ void tc_item(const TcParams& p, const qe_expert& ex, int r0, c
     __syncthreads();
     return;
   }
-  TC_DBG(4, 1);
   tc_fence_after();
   // epilogue: warp w reads rows 32*(w & 3) .. +31 (its tensor-memory lane
   // quadrant) and the tokens of half w >> 2, 8 columns at a time
@@ -315,7 +295,6 @@ static __device__ void tc_item(const TcParams& p, const qe_expert& ex, int r0, c
   }
   tc_fence_before();
   __syncthreads();
-  TC_DBG(4, 2);
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1) grouped_tc_gateup_kernel(const TcParams p) {
@@ -349,7 +328,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) grouped_tc_gateup_kernel(const 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  TC_DBG(0, 0xA0000000u | (tmem & 0xFFFFu));
   uint32_t ncommit[2] = {0u, 0u};
   for (;;) {
     if (tid == 0) s_item = atomicAdd(&p.ctl[4], 1);
@@ -358,7 +336,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) grouped_tc_gateup_kernel(const 
     if (item >= n_items || *abort_flag) break;
     const int e = p.order[item / ipe];
     const int r0 = (item % ipe) * kTcM;
-    TC_DBG(1, (unsigned)item);
     if (tid == 0) s_ex = p.experts[e];
     __syncthreads();
     const int bits = s_ex.gate.bits;
@@ -388,15 +365,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) grouped_tc_gateup_kernel(const 
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols) : "memory");
   }
-  TC_DBG(5, 0xDEADu);
 }
-
-#ifdef QE_TC_DEBUG
-static unsigned* g_tc_dbg_host = nullptr;
-}  // namespace qe
-extern "C" __attribute__((visibility("default"))) void* qe_tc_debug_host(void) { return qe::g_tc_dbg_host; }
-namespace qe {
-#endif
 
 bool tc_eligible(int H, int I) { return I % kTcM == 0 && H % kTcKB == 0; }
 
@@ -417,18 +386,6 @@ cudaError_t launch_tc_gateup(const GroupedParams& gp, int* ctl, unsigned long lo
   p.experts = gp.experts; p.xh = gp.xh;
   p.count = gp.grp_count; p.start = gp.grp_start; p.list = gp.grp_list; p.order = gp.grp_order;
   p.ctl = ctl; p.h = gp.h; p.hamax = gp.hamax; p.err = gp.err; p.budget_ns = budget_ns;
-#ifdef QE_TC_DEBUG
-  static unsigned* dbg_h = nullptr;
-  static unsigned* dbg_d = nullptr;
-  if (!dbg_h) {
-    if (cudaHostAlloc((void**)&dbg_h, 8 * 1024 * sizeof(unsigned), cudaHostAllocMapped) == cudaSuccess) {
-      memset(dbg_h, 0, 8 * 1024 * sizeof(unsigned));
-      cudaHostGetDevicePointer((void**)&dbg_d, dbg_h, 0);
-      g_tc_dbg_host = dbg_h;
-    }
-  }
-  p.dbg = dbg_d;
-#endif
   grouped_tc_gateup_kernel<<<sms, kTcThreads, kTcSmem, s>>>(p);
   return cudaGetLastError();
 }
