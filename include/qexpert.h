@@ -145,8 +145,10 @@ QE_API int qe_pool_table(const qe_cfg* cfg, void* dev_base, int bits, int n, qe_
 /* Bytes of device workspace the calls below need for T tokens. */
 QE_API size_t qe_workspace_bytes(const qe_cfg* cfg, int T);
 
-/* Zero a workspace (device).  Call once after allocating it, and again after
- * a call reported QE_ERR_TIMEOUT. */
+/* Zero a workspace (device).  Call once after allocating it.  After a call
+ * that reported QE_ERR_TIMEOUT the workspace stays usable: the single-token
+ * kernel tags what it publishes with a launch epoch kept in the workspace,
+ * so nothing a timed-out launch left behind is mistaken for new data. */
 QE_API int qe_workspace_init(void* dev_ws, size_t ws_bytes, qe_stream_t stream);
 
 /* Synchronise `stream`, then return (and clear) the status the device wrote
@@ -206,8 +208,11 @@ QE_API int moe_combine(const float* y, const float* w, const float* residual, in
  * (+ x[t] if add_residual).  x [T,H] device fp32 or bf16 (x_dtype); out
  * [T,H] fp32 device (must not alias x); topk_idx/topk_w [T,K] device outputs
  * or NULL.  For T == 1 this is one persistent kernel covering the router,
- * the K experts and the combine (a shape whose shared-memory plan does not
- * fit that kernel, such as hidden 8192, takes the batched path).  For T > 1
+ * the K experts and the combine; it keeps each SM's share of the K selected
+ * experts resident in shared memory, so it takes hidden <= 4096, inter <=
+ * 1024 and n_experts <= 8 x the SM count whose share fits, with x 16-byte
+ * aligned (8 for bf16) and gamma 16-byte aligned.  Other single tokens take
+ * the batched path.  For T > 1
  * the tokens are one batch: assignments are grouped per expert, and each
  * selected expert's weights are read once per pass over up to 4 of its
  * tokens. */
@@ -232,7 +237,7 @@ QE_API int moe_layer_step_host(const qe_cfg* cfg, const qe_layer* layer, const v
  * lives.
  *
  * Instead of a workspace it uses a fixed scratch array built into the
- * library (139,520 bytes, 256-byte aligned), which every GPU that loads the
+ * library (180,480 bytes, 256-byte aligned), which every GPU that loads the
  * library holds until the process exits.  It calls no allocation routine.
  *   x       [1,H] device, fp32 or bf16 bits (x_dtype); out [1,H] fp32
  *           device (must not alias x); topk_idx/topk_w [1,K] device outputs
@@ -240,15 +245,20 @@ QE_API int moe_layer_step_host(const qe_cfg* cfg, const qe_layer* layer, const v
  *   dev_status  int32 device output or NULL: after the step it holds the
  *           device-side status of this call (QE_OK, QE_ERR_TIMEOUT or
  *           QE_ERR_INVALID_ARG), read by the caller after synchronising.
- * Limits: top_k * inter <= 32768; hidden a multiple of 256 and <= 4096;
- * n_experts <= 8 x the SM count.  Larger shapes are rejected with
- * QE_ERR_INVALID_ARG (top_k * inter) or QE_ERR_UNSUPPORTED (the others)
- * before anything is launched.
+ * Limits: top_k * inter <= 16384, plus the single-token kernel's own: hidden
+ * <= 4096, inter <= 1024, n_experts <= 8 x the SM count, the experts' share
+ * of one SM within its shared memory, x 16-byte aligned (8 for bf16) and
+ * gamma 16-byte aligned.  Anything else is rejected before anything is
+ * launched: QE_ERR_INVALID_ARG for top_k * inter and the alignment,
+ * QE_ERR_UNSUPPORTED for the rest.
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.  Every call clears the array's
- * control block on `stream` before its kernel, so a call that timed out
- * needs no re-initialisation.  All calls on a device share the array and
+ * (cudaGetSymbolAddress, with that device current) and caches it per device
+ * ordinal, for the device's primary context (the one the CUDA runtime uses);
+ * do not call it under another driver-API context of the same device.  Make
+ * that first call before any stream capture.  Every call clears the array's
+ * error word on `stream` before its kernel; the launch epoch kept in the
+ * array advances with every call, so a call after one that timed out needs
+ * no re-initialisation.  All calls on a device share the array and
  * its contents outlive the call: two calls whose work overlaps on the GPU
  * (other streams, other threads) race and give wrong results; order them
  * on one stream or with events. */
@@ -321,22 +331,38 @@ QE_API int qe_tier_slots(const qe_tier* t);
  * no-op. */
 QE_API void qe_tier_destroy(qe_tier* t);
 
-/* Test hook: make CTA `cta` of the next fused single-token launches skip its
- * arrival at the routing barrier (-1 disables).  The other CTAs' bounded
- * waits then give up and the workspace reports QE_ERR_TIMEOUT. */
+/* Test hook: make CTA `cta` of the next fused single-token launches skip
+ * publishing its router logits (-1 disables).  Every CTA's bounded wait for
+ * those logits then gives up and the workspace reports QE_ERR_TIMEOUT. */
 QE_API void qe_test_skip_arrival(int cta);
 
-/* Tracing: while dev_buf (device, uint64 [SMs][64]) is set, every fused
+/* Test hook, host only (no GPU involved): the single-token kernel's plan for
+ * CTA `cta` of a grid of `sms` CTAs with `smem_optin` bytes of shared memory
+ * per block, computed by the functions the kernel itself uses.  bits[K]: the
+ * bits of the K selected experts; seg[K*9]: their segment addresses in
+ * qe_pool_table's order (any 16-byte aligned values).  Writes geom[24] (the
+ * geometry; geom[21] = copies, geom[22] = reads, geom[23] = first gate/up
+ * row), copies[n][4] = {shared-memory offset, source address, bytes,
+ * mbarrier} and reads[n][6] = {kind, expert, a, b, shared-memory offset,
+ * bytes} (kind 0 gate/up word, a = 2*pair + up, b = 32-column chunk; 1
+ * gate/up scale or bias, a = 4*pair + segment, b = group; 2 down word, a =
+ * owned row, b = chunk; 3 down scale or bias, a = 2*row + segment, b =
+ * group).  Returns QE_ERR_UNSUPPORTED for a shape the kernel does not take
+ * and QE_ERR_INVALID_ARG if the arrays are too small. */
+QE_API int qe_fused_plan_probe(int H, int E, int K, int I, int sms, int smem_optin, int cta, const int* bits,
+                               const uint64_t* seg, int* geom, long long* copies, int max_copies, long long* reads,
+                               int max_reads);
+
+/* Tracing: while dev_buf (device, uint64 [SMs][16]) is set, every fused
  * single-token launch writes globaltimer stamps (ns) of its phases per CTA:
- * 0 start, 1 router logits written, 2 routing barrier passed, 3 top-K
- * done, 7 gate/up phase done, 8 h barrier passed, 9 h staged, 10 last down
- * row done, 11 end; 12 and 13 the SM cycle counter at start and end; 16+w
- * and 32+w: warp w done with gate/up and with down; 48 CTA joined after the
- * expert phase, 49 combine done; 56-58 routing
- * sub-steps (router loop, first barrier, RMSNorm pass 2); 59/60 warp 0's
- * first gate/up item landed / computed, 61 its group past that item, 62/63
- * the same for the second item.  Slots a CTA does not reach keep their old
- * value.  NULL disables tracing. */
+ * 0 start, 1 router dot products done, 2 all logits received, 3 top-K done,
+ * 4 expert copies issued, 5 first row pair landed, 6 gate/up done, 7 all of
+ * h received and staged, 8 down rows done, 9 end, 10 experts and weights
+ * known (before their descriptors are read), 11 warp 0 has the last
+ * expert's gate/up rows, 12 warp 0 has its down rows, 13 all of h
+ * received, 14 every thread has its logits, 15 warp 0 done with its top-K
+ * rounds.  Slots a CTA does not
+ * reach keep their old value.  NULL disables tracing. */
 QE_API void qe_trace_fused(void* dev_buf);
 
 #ifdef __cplusplus

@@ -48,6 +48,11 @@ WsLayout ws_layout(int H, int E, int K, int I, int T) {
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off = al(off + bytes); return o; };
   L.control = take(sizeof(WsControl));
+  // the single-token kernel's records first: their place depends on the
+  // shape only, not on T, so no batched call on the same workspace writes there
+  L.f_logit = take(16 * (size_t)E);
+  L.f_h = take(8 * (size_t)K * I);
+  L.f_done = take(8 * (size_t)kMaxGrid * kDoneStride);
   const size_t nlog = (size_t)E * (t > 2 ? t : 2);
   L.logits = take(8 * nlog);
   L.rinv = take(8 * t);
@@ -161,7 +166,16 @@ static int ffn_impl(const qe_cfg* c, const qe_expert* experts, const float* xn, 
   return QE_OK;
 }
 
-bool fused_fits(const qe_cfg* c) {
+// The single-token kernel reads x (and gamma) four elements at a time: it
+// takes a token whose x is 16-byte aligned (8 for bf16) and whose gamma, if
+// any, is 16-byte aligned; other tokens take the multi-kernel path.
+bool fused_aligned(const void* x, int x_dtype, const float* gamma) {
+  if (((uintptr_t)x & (x_dtype == QE_BF16 ? 7u : 15u)) != 0) return false;
+  return gamma == nullptr || ((uintptr_t)gamma & 15u) == 0;
+}
+
+bool fused_fits(const qe_cfg* c, const void* x, int x_dtype, const float* gamma) {
+  if (!fused_aligned(x, x_dtype, gamma)) return false;
   const DevInfo d = dev_info();
   FusedGeometry g;
   return fused_geometry(c->hidden, c->n_experts, c->top_k, c->inter, d.sms, d.optin, &g) == QE_OK;
@@ -180,8 +194,9 @@ int fused_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_dtyp
   p.gamma = layer->gamma; p.router_w = layer->router_w; p.offset = layer->logit_offset;
   p.experts = layer->experts; p.out = out; p.topk_idx = topk_idx; p.topk_w = topk_w;
   p.ctl = at<WsControl>(ws, L.control);
-  p.logit_part = at<double>(ws, L.logits);
-  p.hbuf = at<float>(ws, L.h);
+  p.rec_logit = at<unsigned long long>(ws, L.f_logit);
+  p.rec_h = at<unsigned long long>(ws, L.f_h);
+  p.rec_done = at<unsigned long long>(ws, L.f_done);
   p.given_idx = given_idx;
   p.given_w = given_w;
   p.budget_ns = g_budget_ns;
@@ -333,7 +348,7 @@ int moe_layer_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_
   if ((const void*)out == x) return fail(QE_ERR_INVALID_ARG, "out must not alias x");
   cudaStream_t s = (cudaStream_t)stream;
   const WsLayout L = ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, T);
-  if (T == 1 && fused_fits(c)) return fused_step(c, layer, x, x_dtype, out, add_residual, topk_idx, topk_w, ws,
+  if (T == 1 && fused_fits(c, x, x_dtype, layer->gamma)) return fused_step(c, layer, x, x_dtype, out, add_residual, topk_idx, topk_w, ws,
                                                    nullptr, nullptr, s);
   // batched (or a single token whose shape does not fit the fused kernel):
   // route all tokens, then the expert FFNs, then the combine
@@ -406,18 +421,19 @@ extern "C" int moe_layer_step_host(const qe_cfg* c, const qe_layer* layer, const
 // ---------------------------------------------------------------------------
 // Single-token layer step whose scratch lives in the library itself.
 //
-// The fused single-token kernel needs three pieces of device scratch besides
-// its inputs and outputs: the control block (grid counters, error word, per
-// expert |h| maxima), the E router logits and the K x I SwiGLU activations.
+// The fused single-token kernel needs device scratch besides its inputs and
+// outputs: the control block (error word, launch epoch), the tagged router
+// logits, the tagged SwiGLU activations and one "h published" record per CTA.
 // moe_layer_step takes them from a caller-allocated workspace; the entry
 // point below takes them from a fixed array that every GPU loading this
 // library holds until the process exits.
 namespace qe {
 
-constexpr size_t kStaticLogitsOff = sizeof(WsControl);              // 256
-constexpr size_t kStaticHOff = kStaticLogitsOff + 8 * (size_t)kMaxE;  // 8 KiB of fp64 logits
-constexpr size_t kStaticMaxKI = 32768;                               // top_k * inter
-constexpr size_t kStaticBytes = kStaticHOff + 4 * kStaticMaxKI;       // 139,520 bytes
+constexpr size_t kStaticMaxKI = 16384;                                   // top_k * inter: 16 x 1024
+constexpr size_t kStaticLogitsOff = sizeof(WsControl);                   // 256
+constexpr size_t kStaticHOff = kStaticLogitsOff + 16 * (size_t)kMaxE;    // + 16 KiB of logit records
+constexpr size_t kStaticDoneOff = kStaticHOff + 8 * kStaticMaxKI;        // + 128 KiB of h records
+constexpr size_t kStaticBytes = kStaticDoneOff + 8 * (size_t)kMaxGrid * kDoneStride;  // + 32 KiB: 180,480 bytes
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticBytes];
 
@@ -465,28 +481,33 @@ extern "C" int moe_layer_step_noalloc(const qe_cfg* c, const qe_layer* layer, co
       (rc = check_ptr(dev_status, "dev_status", true)))
     return rc;
   if ((const void*)out == x) return fail(QE_ERR_INVALID_ARG, "out must not alias x");
+  if (!fused_aligned(x, x_dtype, layer->gamma))
+    return fail(QE_ERR_INVALID_ARG,
+                "moe_layer_step_noalloc: x must be 16-byte aligned (8 for bf16) and gamma 16-byte aligned");
   FusedParams p{};
   const DevInfo d = dev_info();
   if (fused_geometry(c->hidden, c->n_experts, c->top_k, c->inter, d.sms, d.optin, &p.g) != QE_OK)
     return fail(QE_ERR_UNSUPPORTED,
-                "moe_layer_step_noalloc: shape not supported by the single-token kernel (hidden %d must be a "
-                "multiple of 256 and <= 4096; n_experts %d must be <= 8 x SMs)",
-                c->hidden, c->n_experts);
+                "moe_layer_step_noalloc: shape not supported by the single-token kernel (hidden %d must be <= "
+                "4096, inter %d <= 1024, n_experts %d <= 8 x SMs, and the experts' share of one SM must fit "
+                "in its shared memory)",
+                c->hidden, c->inter, c->n_experts);
   unsigned char* scratch = nullptr;
   if ((rc = static_scratch(&scratch))) return rc;
   cudaStream_t s = (cudaStream_t)stream;
   WsControl* ctl = (WsControl*)scratch;
-  // the previous call (possibly one that timed out) left its counters and
-  // error word here: the kernel expects them at zero
-  cudaError_t e = cudaMemsetAsync(ctl, 0, sizeof(WsControl), s);
-  if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step_noalloc: clear control block");
+  // the previous call's error word is cleared; its launch epoch stays, so
+  // this call's records carry a tag no earlier call wrote
+  cudaError_t e = cudaMemsetAsync(&ctl->err, 0, sizeof(ctl->err), s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_layer_step_noalloc: clear the error word");
   p.H = c->hidden; p.E = c->n_experts; p.K = c->top_k; p.I = c->inter; p.eps = c->eps;
   p.x = x; p.x_bf16 = x_dtype == QE_BF16; p.add_residual = add_residual != 0;
   p.gamma = layer->gamma; p.router_w = layer->router_w; p.offset = layer->logit_offset;
   p.experts = layer->experts; p.out = out; p.topk_idx = topk_idx; p.topk_w = topk_w;
   p.ctl = ctl;
-  p.logit_part = (double*)(scratch + kStaticLogitsOff);
-  p.hbuf = (float*)(scratch + kStaticHOff);
+  p.rec_logit = (unsigned long long*)(scratch + kStaticLogitsOff);
+  p.rec_h = (unsigned long long*)(scratch + kStaticHOff);
+  p.rec_done = (unsigned long long*)(scratch + kStaticDoneOff);
   p.budget_ns = g_budget_ns;
   p.skip_cta = g_skip_cta;
   p.trace = g_trace;

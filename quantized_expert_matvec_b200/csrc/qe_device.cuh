@@ -101,12 +101,25 @@ QE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that may suspend the thread for up to `ns` nanoseconds while the
+// phase is incomplete (it resumes as soon as the phase completes).
+QE_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.
 QE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t deadline, volatile int* abort_flag) {
   unsigned spins = 0;
   while (!mbar_try_wait(bar, parity)) {
-    if (*abort_flag) return false;
-    if ((++spins & 7u) == 0 && gtimer() > deadline) return false;
+    if ((++spins & 15u) == 0 && (*abort_flag || gtimer() > deadline)) return false;
   }
   return true;
 }
@@ -142,6 +155,56 @@ template <int N>
 QE_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 QE_DEV void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p)); }
 QE_DEV void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
+
+// 1-D bulk copy (TMA engine) of `bytes` (a multiple of 16; both addresses
+// 16-byte aligned) from global to this CTA's shared memory; its completion
+// counts `bytes` against the transaction count of mbarrier `bar`.  No
+// multicast: the copy lands in the issuing CTA only.
+QE_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
+// Arrive on `bar` and raise its expected transaction count by `bytes`.
+QE_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Tagged records: an aligned 64-bit word {32-bit value, 32-bit tag of the
+// launch that wrote it}.  A reader that sees the tag it expects in a word
+// also sees that launch's value in it (single-copy atomicity of an aligned
+// 64-bit access), so records need no fence or flag; a 16-byte access moves
+// two of them (each word still atomic on its own).
+QE_DEV unsigned long long rec_word(uint32_t value, uint32_t tag) { return ((unsigned long long)tag << 32) | value; }
+QE_DEV uint32_t rec_tag(unsigned long long w) { return (uint32_t)(w >> 32); }
+QE_DEV uint32_t rec_val(unsigned long long w) { return (uint32_t)w; }
+QE_DEV void st_rec(unsigned long long* p, unsigned long long w) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+QE_DEV unsigned long long ld_rec(const unsigned long long* p) {
+  unsigned long long w;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return w;
+}
+QE_DEV void st_rec2(unsigned long long* p, unsigned long long a, unsigned long long b) {
+  asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(p), "l"(a), "l"(b) : "memory");
+}
+QE_DEV void ld_rec2(const unsigned long long* p, unsigned long long& a, unsigned long long& b) {
+  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+}
+
+QE_DEV unsigned ld_relaxed_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+QE_DEV void st_relaxed_u32(unsigned* p, unsigned v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 // Named barrier over `count` threads (non-aligned form: counts threads).
 QE_DEV void named_barrier(int id, int count) {
@@ -394,5 +457,147 @@ QE_DEV void load_xs32_q2(const float* xp, int lc, float2 (&xs)[16]) { load_xs32(
 
 // 2^(60+E): turns acc back into sum q*x.
 QE_DEV float acc_scale(int E) { return __int_as_float((127 + 60 + E) << 23); }
+
+// ------------------------------------------------ integer dequant-dot cores
+//
+// The activation vector v is held as 22-bit fixed point under one power-of-
+// two scale per vector: v_c = vi_c * 2^(e-22), |vi_c| < 2^22, where e is the
+// least exponent with max|v| < 2^e (fixed_scale_exponent).  vi is split into
+// three byte limbs, vi = b2 * 2^16 + b1 * 2^8 + b0 (b2 signed, b1 and b0
+// unsigned).  A packed word of q fields is spread into bytes with masks (two
+// LOP3 and a shift per eight 4-bit fields) and dp4a multiplies four q bytes
+// with four limb bytes, accumulating exactly in int32.  Per 32-column chunk
+// and row the three limb sums give
+//   sum_c q_c vi_c = A2 * 2^16 + A1 * 2^8 + A0,
+// and the group's affine term is then  s * 2^(e-22) * that + b * sum_c v_c.
+// Everything before the final fp32 combination is exact integer arithmetic,
+// and the fixed point keeps 22 bits below max|v|.  This costs 0.375 integer
+// ops and 0.75 dp4a per weight, against one mask per weight for a float
+// operand per q field.  Integers below 2^22 in magnitude move to and from
+// fp32 by adding 1.5 * 2^23 (round to nearest, exact), so neither direction
+// uses the slow conversion unit.
+//
+// Byte order of the limb words of one 32-column chunk:
+//   4-bit: word r = 2w + h (w = packed word 0..3, h = 0 even fields, 1 odd
+//          fields): byte i holds column 8w + 2i + h;
+//   2-bit: word r = 4w + t (w = packed word 0..1, t = shift 0..3): byte i
+//          holds column 16w + 4i + t.
+
+struct XLimbs {
+  int b2[8];       // signed high limbs
+  unsigned b1[8];  // unsigned middle limbs
+  unsigned b0[8];  // unsigned low limbs
+};
+
+QE_DEV int dp4a_us(unsigned a, int b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+QE_DEV int dp4a_uu(unsigned a, unsigned b, int c) {
+  int d;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+QE_DEV unsigned prmt(unsigned a, unsigned b, unsigned sel) {
+  unsigned d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr int kMagicBits = 0x4B400000;
+// Nearest integer of f, |f| < 2^22.
+QE_DEV int round_small(float f) { return __float_as_int(f + kMagic) - kMagicBits; }
+// i as a float, |i| < 2^22 (exact).
+QE_DEV float small_to_float(int i) { return __int_as_float(i + kMagicBits) - kMagic; }
+
+// Least e with max|v| < 2^e (amax = max|v|), kept where both 2^(22-e) and
+// 2^(e-22) are normal floats; 0 for an all-zero vector.
+QE_DEV int fixed_scale_exponent(float amax) {
+  if (!(amax > 0.0f)) return 0;
+  const int e = ((int)((__float_as_uint(amax) >> 23) & 0xFF)) - 127 + 1;
+  return e < -100 ? -100 : (e > 120 ? 120 : e);
+}
+QE_DEV float pow2f(int k) { return __int_as_float((127 + k) << 23); }  // 2^k, |k| <= 126
+
+// The limbs of one 32-column chunk under exponent e; also returns the sum of
+// the 32 raw values (column order).  src is the chunk's 32 floats in shared
+// memory with its eight 16-byte pieces swizzled (piece i at i ^ sw, sw = the
+// chunk's index & 7, as xswz lays them out), so the lanes of a warp reading
+// consecutive chunks spread over all banks.
+template <int BITS>
+QE_DEV float build_limbs(const float* src, int sw, int e, XLimbs& x) {
+  const float in = pow2f(22 - e);
+  int vi[32];
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 f = ((const float4*)src)[i ^ sw];
+    sum += f.x; sum += f.y; sum += f.z; sum += f.w;
+    vi[4 * i] = round_small(f.x * in);
+    vi[4 * i + 1] = round_small(f.y * in);
+    vi[4 * i + 2] = round_small(f.z * in);
+    vi[4 * i + 3] = round_small(f.w * in);
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    unsigned v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      v[i] = (unsigned)vi[BITS == 4 ? 8 * (r >> 1) + 2 * i + (r & 1) : 16 * (r >> 2) + 4 * i + (r & 3)];
+    // byte k of v[0..3] into bytes 0..3 of limb word k
+    const unsigned t01 = prmt(v[0], v[1], 0x5140u), t23 = prmt(v[2], v[3], 0x5140u);
+    const unsigned s01 = prmt(v[0], v[1], 0x0062u), s23 = prmt(v[2], v[3], 0x0062u);
+    x.b0[r] = prmt(t01, t23, 0x5410u);
+    x.b1[r] = prmt(t01, t23, 0x7632u);
+    x.b2[r] = (int)prmt(s01, s23, 0x5410u);
+  }
+  return sum;
+}
+
+QE_DEV float limb_sum(int a2, int a1, int a0) {
+  return fmaf(small_to_float(a2), 65536.0f, fmaf(small_to_float(a1), 256.0f, small_to_float(a0)));
+}
+
+// sum_c q_c vi_c of one 32-column chunk of 4-bit weights (words 0..3).
+QE_DEV float idot32_q4(const uint4 w, const XLimbs& x) {
+  int a2 = 0, a1 = 0, a0 = 0;
+  const unsigned ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const unsigned lo = ws[j] & 0x0F0F0F0Fu, hi = (ws[j] >> 4) & 0x0F0F0F0Fu;
+    a2 = dp4a_us(lo, x.b2[2 * j], a2);
+    a1 = dp4a_uu(lo, x.b1[2 * j], a1);
+    a0 = dp4a_uu(lo, x.b0[2 * j], a0);
+    a2 = dp4a_us(hi, x.b2[2 * j + 1], a2);
+    a1 = dp4a_uu(hi, x.b1[2 * j + 1], a1);
+    a0 = dp4a_uu(hi, x.b0[2 * j + 1], a0);
+  }
+  return limb_sum(a2, a1, a0);
+}
+
+// Same for 2-bit weights (words 0..1).
+QE_DEV float idot32_q2(const uint2 w, const XLimbs& x) {
+  int a2 = 0, a1 = 0, a0 = 0;
+  const unsigned ws[2] = {w.x, w.y};
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const unsigned q = (ws[j] >> (2 * t)) & 0x03030303u;
+      a2 = dp4a_us(q, x.b2[4 * j + t], a2);
+      a1 = dp4a_uu(q, x.b1[4 * j + t], a1);
+      a0 = dp4a_uu(q, x.b0[4 * j + t], a0);
+    }
+  }
+  return limb_sum(a2, a1, a0);
+}
+
+template <int BITS>
+QE_DEV float idot32(const unsigned char* w, const XLimbs& x) {
+  if (BITS == 4) return idot32_q4(*(const uint4*)w, x);
+  return idot32_q2(*(const uint2*)w, x);
+}
 
 }  // namespace qe

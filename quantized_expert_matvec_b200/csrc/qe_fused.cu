@@ -2,61 +2,69 @@
 // RMSNorm -> router (fp64) -> top-K -> gate/up dequant-matvec + SwiGLU ->
 // down dequant-matvec -> weighted combine (+ residual).
 //
-// One CTA per SM (16 warps), launched cooperatively so all CTAs are resident.
+// One CTA of 16 warps per SM, launched cooperatively so every CTA is
+// resident; the kernel is bound by HBM bytes and by the latency of the two
+// grid-wide exchanges the step needs (all logits before top-K, all of h
+// before the down matvecs).
 //
-// Routing: CTA c owns router rows c, c+G, ...; each warp covers one 1/16
-// column slice of them, and the same x loads feed the RMSNorm sum of squares
-// (the router dot does not depend on the norm scale).  After a grid-wide
-// counter, every CTA ranks all E logits itself: per-warp top-K candidates by
-// redux reductions, then one merge.
+// Exchanges.  The step needs two grid-wide exchanges: all logits before
+// top-K, all of h before the down matvecs.  Each CTA publishes its values
+// as tagged records (a 64-bit word {value, tag}; a logit takes two, written
+// and read as one 16-byte access) and the readers poll exactly the records
+// they need, with 16-byte relaxed loads, until every word carries this
+// launch's tag: one L2 round trip both waits and delivers.  (Per-CTA flags
+// or a shared counter need a fence and a second round trip, and were about
+// twice as slow on B200.)  For h, every CTA also publishes one "done" record
+// after its h records; readers poll those G records first and then read all
+// of h once (checking every tag, re-polling the rare stale one), so waiting
+// CTAs put little load on L2 while others still stream their down rows.  The
+// tag is (epoch + 1) with the top bit set: every launch reads the workspace
+// epoch, and CTA 0 advances it at the end, once it has seen every CTA's done
+// record (so no CTA of the launch still has to read the old epoch).
+
+// Expert streaming.  Right after top-K, warp k issues the CTA's share of
+// selected expert k as 1-D bulk copies (TMA engine) into shared memory: its
+// gate and up rows and their scale/bias runs first (one mbarrier), then,
+// once every such warp has issued those, its down rows (another).  The
+// layout and the copy list are in qe_fused_plan.h.  Nothing waits for a
+// copy before all are issued, so the HBM sees the whole step's expert bytes
+// at once.
 //
-// Expert phase.  Gate/up: the selected experts' rows are cut into items of
-// RB rows of gate and of up; the four 4-warp groups take items in turn and
-// each warp of a group copies (16-byte cp.async into the group's ring, one
-// copy group per item) and dequantises one column quarter of every row,
-// keeping the x' of its columns in registers; the four quarter sums meet in
-// shared memory behind a named barrier, and h = silu(g) * u goes to global
-// memory.  Each warp then loads its first down rows into registers.  A second
-// grid-wide counter waits for every CTA's h rows; every CTA then reads all
-// of h, finds max |h_k| itself and stages h_k in x' form in shared memory.
-// Down: warp w works on expert w % K and computes full rows (RC-row blocks of
-// the output rows this CTA owns); the CTA combines its rows (+ residual).
-// All waits are bounded (QE_ERR_TIMEOUT).  The grid counters only grow: each
-// launch adds its grid size, and a CTA's arrival ticket gives the count it
-// waits for, so nothing has to be reset between launches.
+// Gate/up: warp (row group rg, column quarter qd) keeps one 32-column chunk
+// of xn per lane in registers, as 24-bit fixed-point byte limbs for the dp4a
+// dequant core (qe_device.cuh), and walks the row pairs rg, rg+nrg, ... in
+// arrival order; quarter sums meet in shared memory.  h records are
+// published, every CTA stages all K*I of h in shared memory (the gate/up
+// slots are free by then), and warp w computes the owned down rows of
+// expert w % K with its lane's chunk of h as limbs in registers.  The CTA
+// combines its rows (+ residual).  Every wait is bounded (QE_ERR_TIMEOUT).
 #include <math.h>
 
-#include <type_traits>
-
 #include "qe_device.cuh"
+#include "qe_fused_plan.h"
 
 namespace qe {
 
 constexpr int kWarps = 16;
-constexpr int kGroups = 4;  // 4-warp groups of the gate/up phase
-constexpr int kRB = 4;      // rows of gate (and of up) in one gate/up item
-constexpr int kRC = 4;      // rows of one down block
 constexpr int kFusedThreads = kWarps * 32;
 constexpr int kRouterRows = 8;  // router rows one CTA owns at most: E <= 8 * grid
-constexpr int kRouterBatch = 4; // router rows accumulated together
-constexpr int kChunkMax = 8;    // 32-column chunks one warp converts: H <= 8 * 32 * 16
 
 struct FusedMisc {
   int abort;
-  float xK;
+  unsigned tag;
+  int Ex;    // fixed-point exponent of xn: max|xn| < 2^Ex
+  float xK;  // 2^(Ex - 22)
+  int ubits; // bits shared by all K selected experts (4 or 2), 0 if mixed
   int idx[kMaxK];
   float wk[kMaxK];
+  int hexp[kMaxK];  // fixed-point exponent of h_k
+  float hK[kMaxK];  // 2^(hexp - 22)
+  unsigned hamax[kMaxK];  // max |h_k| as float bits
+  int mis_gu[kMaxK][4];   // offsets of the gate/up scale/bias runs in their copies
+  int mis_d[kMaxK][2];
   qe_expert ex[kMaxK];
-  float hK[kMaxK];
-  int hexp[kMaxK];  // vector exponent of h_k (x' form of the down input)
-  unsigned long long route_target;  // routing counter value that completes this launch
-  unsigned cand_idx[kWarps][kMaxK];
-  unsigned long long cand_key[kWarps][kMaxK];
-  double cand_val[kWarps][kMaxK];
-  double lsel[kMaxK];
-  float gred[kGroups][2][4][2 * kRB];  // gate/up partial sums [group][item parity][quarter][row]
-  unsigned hamax[kMaxK];               // max |h_k| of this CTA's rows, as float bits
-  unsigned long long t_lastC;
+  ExpertAddr ea[kMaxK];   // the same descriptors as addresses (copy plan)
+  unsigned long long selkey[kMaxK];  // keys of the selected experts, in rank order
   float redf[kWarps];
   double redd[kWarps];
   double rpart[kRouterRows][kWarps];
@@ -64,11 +72,11 @@ struct FusedMisc {
 
 // Optional phase trace: globaltimer stamps per CTA (qe_trace_fused).
 enum {
-  kTrStart, kTrRouterDone, kTrRouteBarrier, kTrTopK, kTrIssuedB, kTrIssuedC, kTrFirstB, kTrLastB,
-  kTrHFirst, kTrHLast, kTrLastC, kTrEnd
+  kTrStart, kTrRouter, kTrLogits, kTrTopK, kTrIssued, kTrFirstPair, kTrGateUp, kTrHStaged, kTrDown, kTrEnd,
+  kTrMerged, kTrLastGateUpData, kTrDownData, kTrHPolled, kTrPolledAll, kTrRounds
 };
 #define QE_TRACE(slot) \
-  do { if (p.trace) p.trace[(size_t)blockIdx.x * 64 + (slot)] = gtimer(); } while (0)
+  do { if (p.trace) p.trace[(size_t)blockIdx.x * 16 + (slot)] = gtimer(); } while (0)
 
 static __device__ __forceinline__ float load_x(const FusedParams& p, int c) {
   return p.x_bf16 ? bf16f(((const uint16_t*)p.x)[c]) : ((const float*)p.x)[c];
@@ -90,10 +98,21 @@ static __device__ __forceinline__ bool desc_ok(const qe_qmat& m, int bits) {
          ((uintptr_t)m.scales & 15) == 0 && ((uintptr_t)m.biases & 15) == 0;
 }
 
-// Order-preserving map of a double onto an unsigned 64-bit key.
+static __device__ __forceinline__ bool expert_ok(const qe_expert& ex) {
+  const int bits = ex.gate.bits;
+  return (bits == 4 || bits == 2) && desc_ok(ex.gate, bits) && desc_ok(ex.up, bits) && desc_ok(ex.down, bits);
+}
+
+// Order-preserving map of a double onto an unsigned 64-bit key (-0 and +0
+// map to the same key, as they compare equal) and its inverse.
 static __device__ __forceinline__ unsigned long long dkey(double d) {
+  if (d == 0.0) d = 0.0;
   const unsigned long long u = (unsigned long long)__double_as_longlong(d);
   return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+static __device__ __forceinline__ double dkey_inv(unsigned long long k) {
+  const unsigned long long u = (k >> 63) ? (k & 0x7FFFFFFFFFFFFFFFull) : ~k;
+  return __longlong_as_double((long long)u);
 }
 
 // Largest key over the warp, the lowest index among equal keys.  Lanes
@@ -107,149 +126,162 @@ static __device__ __forceinline__ unsigned warp_argmax_key(unsigned long long ke
   return __reduce_min_sync(0xffffffffu, (top && lo == lmax) ? idx : 0xffffffffu);
 }
 
-// ------------------------------------------------------- gate/up (groups)
-// A gate/up item is kRB rows of gate and kRB rows of up of one expert.  The
-// four warps of a group split the columns into quarters; warp qd copies and
-// dequantises quarter qd of every row, so the x' of its columns stays in
-// registers.  Slot layout: packed words of (quarter, matrix, row) at
-// ((qd*2 + mat)*kRB + rr) * H/8, then per warp four segments [gate s | gate
-// b | up s | up b] of sseg bytes at kRB*H + qd*4*sseg.  When H is a multiple
-// of 2048 a segment holds only the quarter's groups of each row (H/128 bytes
-// a row); otherwise it holds whole rows.
-
-struct GateUpCtx {
-  int H, gpr, nlc;  // nlc: 32-column lane chunks per quarter
-  int qsc;          // segments hold quarter rows
-  int sseg;         // bytes of one segment
-  int srow;         // entries (uint16) per row in a segment
-};
-
-static __device__ __forceinline__ GateUpCtx make_gateup_ctx(int H) {
-  GateUpCtx c;
-  c.H = H;
-  c.gpr = H / kGroup;
-  c.nlc = H / 128;
-  c.qsc = (H % 2048) == 0;
-  c.srow = c.qsc ? H / 256 : c.gpr;
-  c.sseg = kRB * c.srow * 2;
-  return c;
+// Bounded poll of N 16-byte record pairs (p[i] 16-byte aligned, or null to
+// skip) until both words of each carry `tag`; every round reloads all pairs
+// still stale at once (one L2 round trip per round).
+template <int N>
+static __device__ __forceinline__ bool poll_rec2(const unsigned long long* const (&p)[N], unsigned tag,
+                                                 uint64_t deadline, volatile int* abort_flag,
+                                                 unsigned long long (&a)[N], unsigned long long (&b)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    a[i] = b[i] = 0ull;
+    if (p[i]) ld_rec2(p[i], a[i], b[i]);
+  }
+  for (unsigned spins = 0;; ++spins) {
+    bool stale = false;
+#pragma unroll
+    for (int i = 0; i < N; ++i) stale |= p[i] && (rec_tag(a[i]) != tag || rec_tag(b[i]) != tag);
+    if (!stale) return true;
+    if (*abort_flag) return false;
+    if ((spins & 7u) == 7u && gtimer() > deadline) return false;
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if (p[i] && (rec_tag(a[i]) != tag || rec_tag(b[i]) != tag)) ld_rec2(p[i], a[i], b[i]);
+  }
 }
 
-static __device__ __forceinline__ void issue_gateup(const qe_expert& ex, int r0, unsigned char* slot, int qd,
-                                                    const GateUpCtx& c, int lane, uint64_t pol) {
-  const int bits = ex.gate.bits;
-  const uint32_t qb = (uint32_t)(c.H * bits / 32);  // bytes of one row quarter
-  const size_t rowb = (size_t)c.H * bits / 8;
-  const unsigned char* gsrc = (const unsigned char*)ex.gate.wq + (size_t)r0 * rowb + qd * qb;
-  const unsigned char* usrc = (const unsigned char*)ex.up.wq + (size_t)r0 * rowb + qd * qb;
-#pragma unroll
-  for (int rr = 0; rr < kRB; ++rr) {
-    warp_copy_async(slot + ((qd * 2 + 0) * kRB + rr) * (c.H / 8), gsrc + rr * rowb, qb, lane, pol);
-    warp_copy_async(slot + ((qd * 2 + 1) * kRB + rr) * (c.H / 8), usrc + rr * rowb, qb, lane, pol);
-  }
-  unsigned char* sd = slot + kRB * c.H + qd * 4 * c.sseg;
-  const uint16_t* segsrc[4] = {ex.gate.scales, ex.gate.biases, ex.up.scales, ex.up.biases};
-  if (c.qsc) {
-    const int npc = c.H / 2048;  // 16-byte pieces of one quarter row
-    const int per_seg = kRB * npc;
-    for (int u = lane; u < 4 * per_seg; u += 32) {
-      const int seg = u / per_seg, rem = u - seg * per_seg;
-      const int rr = rem / npc, pc = rem - rr * npc;
-      const unsigned char* src = (const unsigned char*)(segsrc[seg] + (size_t)(r0 + rr) * c.gpr + qd * (c.H / 256)) + pc * 16;
-      cp_async16(sd + seg * c.sseg + rr * (c.H / 128) + pc * 16, src, pol);
-    }
-  } else {
-#pragma unroll
-    for (int seg = 0; seg < 4; ++seg)
-      warp_copy_async(sd + seg * c.sseg, segsrc[seg] + (size_t)r0 * c.gpr, (uint32_t)c.sseg, lane, pol);
-  }
-  cp_async_commit();
-}
+static __device__ __forceinline__ float ld_bf16(const unsigned char* p) { return bf16f(*(const uint16_t*)p); }
 
-// Partial sums of the 2*kRB rows over this warp's quarter; returns the
-// warp-reduced value (row reduced_row_of_lane<2*kRB>(lane)).
+// Gate/up phase of one warp: row group rg = warp / nq, column quarter
+// qd = warp % nq, this lane's 32-column chunk lc = 32 qd + lane.  The warp
+// takes the row pairs P = rg, rg + nrg, ... of the flattened (expert, row)
+// list in batches of kPB (one transposed warp reduction per batch: warp
+// shuffles are a scarce resource when all 16 warps reduce), waits for an
+// expert's mbarrier when it first meets that expert, and leaves each pair's
+// two quarter sums in gred.  BITS is the bits of every selected expert, or
+// 0 when they differ (each pair then picks its core).
+constexpr int kPB = 4;
 template <int BITS>
-static __device__ __forceinline__ float gateup_partial(const unsigned char* slot, int qd, const GateUpCtx& c,
-                                                       const float* xp, const float* xs_sum, float xK,
-                                                       float2 (&xs)[16], bool xs_cached, int lane) {
-  float yv[2 * kRB];
+static __device__ __forceinline__ void gateup_phase(const FusedParams& p, const FusedCta& t, FusedMisc* misc,
+                                                    uint64_t* bars, const float* xn_s, float* gred,
+                                                    unsigned char* smem, uint64_t deadline, int warp, int lane) {
+  const FusedGeometry& g = p.g;
+  const int H = p.H, K = p.K;
+  volatile int* abort_flag = &misc->abort;
+  const int qd = warp % g.nq, rg = warp / g.nq;
+  const int lc = qd * 32 + lane;
+  const bool live = lc < H / 32;
+  const int gi = lc >> 1;
+  const int npairs = K * t.np;
+  const float xK = misc->xK;
+  XLimbs xl;
+  float xsl = 0.f;  // sum of this lane's 32 columns of xn
+  int xl_bits = 0;
+  int have_k = -1;  // experts [0, have_k] have landed
+#pragma unroll 1
+  for (int p0 = rg; p0 < npairs; p0 += g.nrg * kPB) {
+    if (__any_sync(0xffffffffu, *abort_flag != 0)) break;  // one decision per warp
+    float acc[2 * kPB];
 #pragma unroll
-  for (int i = 0; i < 2 * kRB; ++i) yv[i] = 0.f;
-  const uint16_t* sc = (const uint16_t*)(slot + kRB * c.H + qd * 4 * c.sseg);
-  const int segs = c.sseg / 2;  // uint16 entries per segment
-  const int goff = c.qsc ? qd * (c.H / 256) : 0;
-  for (int l = lane; l < c.nlc; l += 32) {
-    const int lc = qd * c.nlc + l;  // 32-column chunk of the full row
-    if (!xs_cached) load_xs32(xp, lc, xs);
-    const int gi = (lc >> 1) - goff;
-    const float xsum = xs_sum[lc];
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-#pragma unroll
-      for (int rr = 0; rr < kRB; ++rr) {
-        const unsigned char* wp = slot + ((qd * 2 + m) * kRB + rr) * (c.H / 8);
-        float2 a;
-        if (BITS == 4) a = dot32_q4(*(const ulonglong2*)(wp + l * 16), xs, make_float2(0.f, 0.f));
-        else a = dot32_q2(*(const unsigned long long*)(wp + l * 8), xs, make_float2(0.f, 0.f));
-        const float sv = bf16f(sc[(2 * m) * segs + rr * c.srow + gi]);
-        const float bv = bf16f(sc[(2 * m + 1) * segs + rr * c.srow + gi]);
-        yv[m * kRB + rr] += sv * xK * (a.x + a.y) + bv * xsum;
+    for (int i = 0; i < kPB; ++i) {
+      acc[2 * i] = acc[2 * i + 1] = 0.f;
+      const int P = p0 + g.nrg * i;
+      if (P < npairs) {  // uniform over the warp
+        const int k = P / t.np, j = P - k * t.np;
+        const int bits = BITS ? BITS : misc->ex[k].gate.bits;
+        if (bits != xl_bits) {
+          if (live) xsl = bits == 4 ? build_limbs<4>(xn_s + 32 * lc, lc & 7, misc->Ex, xl)
+                                    : build_limbs<2>(xn_s + 32 * lc, lc & 7, misc->Ex, xl);
+          xl_bits = bits;
+        }
+        if (k > have_k) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars[bar_gu(k)], 0, deadline, abort_flag))) {
+            set_error(&p.ctl->err, QE_ERR_TIMEOUT);
+            misc->abort = 1;
+            break;
+          }
+          have_k = k;
+          if (warp == 0 && lane == 0 && P == 0) QE_TRACE(kTrFirstPair);
+          if (warp == 0 && lane == 0 && k == K - 1) QE_TRACE(kTrLastGateUpData);
+        }
+        if (live) {
+          const unsigned char* wg = smem + gu_word_smem(g, H, k, j, 0, lc, bits);
+          const unsigned char* wu = smem + gu_word_smem(g, H, k, j, 1, lc, bits);
+          float ag, au;
+          if (BITS) {
+            ag = idot32<BITS ? BITS : 4>(wg, xl);
+            au = idot32<BITS ? BITS : 4>(wu, xl);
+          } else if (bits == 4) {
+            ag = idot32<4>(wg, xl);
+            au = idot32<4>(wu, xl);
+          } else {
+            ag = idot32<2>(wg, xl);
+            au = idot32<2>(wu, xl);
+          }
+          const float sg = ld_bf16(smem + gu_scale_smem(g, H, k, 0, misc->mis_gu[k][0], j, gi));
+          const float bg = ld_bf16(smem + gu_scale_smem(g, H, k, 1, misc->mis_gu[k][1], j, gi));
+          const float su = ld_bf16(smem + gu_scale_smem(g, H, k, 2, misc->mis_gu[k][2], j, gi));
+          const float bu = ld_bf16(smem + gu_scale_smem(g, H, k, 3, misc->mis_gu[k][3], j, gi));
+          acc[2 * i] = sg * xK * ag + bg * xsl;
+          acc[2 * i + 1] = su * xK * au + bu * xsl;
+        }
       }
     }
-  }
-  return warp_reduce_rows<2 * kRB>(yv, lane);
-}
-
-// ------------------------------------------------------------ down (warps)
-// A warp computes full rows of one expert's down matrix: RC-row blocks of the
-// output blocks this CTA owns, up to 8 rows per batch; batch row i is row
-// (i % RC) of block wi + nwk * (i / RC).  Each lane takes one 32-column chunk
-// of every row; the packed words and the scale/bias pair of that chunk are
-// loaded into registers (before h is ready, for the first chunk).
-struct DownRows {
-  ulonglong2 w[8];  // 4-bit: words 0..3; 2-bit: words 0..1 in .x
-  // bf16 scale and bias, kept as loaded: combining them would make the warp
-  // wait for the loads here instead of at their first use after the h barrier
-  unsigned short sc[8], bi[8];
-};
-
-static __device__ __forceinline__ int down_row(int cta, int G, int RC, int wi, int nwk, int ri) {
-  const int blk = ri / RC;
-  return (cta + G * (wi + nwk * blk)) * RC + (ri - blk * RC);
-}
-
-static __device__ __forceinline__ void down_load(const qe_qmat& d, int cta, int G, int RC, int wi, int nwk, int b0,
-                                                 int nr, int I, int lc, DownRows& R) {
-  const int gpr = I / kGroup;
-  const size_t rowb = (size_t)I * d.bits / 8;
-  const int g = lc >> 1;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (i < nr) {
-      const int row = down_row(cta, G, RC, wi, nwk, b0 + i);
-      const unsigned char* rp = (const unsigned char*)d.wq + (size_t)row * rowb;
-      if (d.bits == 4) R.w[i] = __ldcs((const ulonglong2*)rp + lc);
-      else R.w[i].x = __ldcs((const unsigned long long*)rp + lc);
-      R.sc[i] = __ldg(d.scales + (size_t)row * gpr + g);
-      R.bi[i] = __ldg(d.biases + (size_t)row * gpr + g);
-    }
+    // batch row 2i = gate, 2i + 1 = up of pair p0 + nrg*i
+    const float r = warp_reduce_rows<2 * kPB>(acc, lane);
+    const int row = reduced_row_of_lane<2 * kPB>(lane);
+    const int P = p0 + g.nrg * (row >> 1);
+    if (lane == lane_of_reduced_row<2 * kPB>(row) && P < npairs) gred[(P * g.nq + qd) * 2 + (row & 1)] = r;
   }
 }
 
+// Down phase of one warp: expert k = warp % K, its owned rows wi, wi + nwk,
+// ... (wi = warp / K, nwk = warps per expert), one row at a time, with this
+// lane's 32-column chunk of h_k as limbs in registers; row results go to
+// ycomb.
 template <int BITS>
-static __device__ __forceinline__ void down_accum(const DownRows& R, int nr, int lc, const float* hpk,
-                                                  const float* hsk, float hK, float (&yv)[8]) {
-  float2 xs[16];
-  if (BITS == 4) load_xs32_q4(hpk, lc, xs);
-  else load_xs32_q2(hpk, lc, xs);
-  const float xsum = hsk[lc];
+static __device__ __forceinline__ void down_phase(const FusedParams& p, const FusedCta& t, FusedMisc* misc,
+                                                  uint64_t* bars, const float* hst, float* ycomb,
+                                                  unsigned char* smem, uint64_t deadline, int warp, int lane) {
+  const FusedGeometry& g = p.g;
+  const int K = p.K, I = p.I;
+  volatile int* abort_flag = &misc->abort;
+  const int k = warp % K, wi = warp / K, nwk = kWarps / K;
+  const bool live = lane < I / 32;
+  const int gi = lane >> 1;
+  XLimbs hl;
+  float hs = 0.f;
+  const int ch = k * (I / 32) + lane;  // this lane's chunk of the staged h
+  if (live) hs = build_limbs<BITS>(hst + 32 * ch, ch & 7, misc->hexp[k], hl);
+  const float hK = misc->hK[k];
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[bar_down(K, k)], 0, deadline, abort_flag));
+  if (warp == 0 && lane == 0) QE_TRACE(kTrDownData);
+  if (!ok) {
+    set_error(&p.ctl->err, QE_ERR_TIMEOUT);
+    misc->abort = 1;
+    return;
+  }
+  const int ms0 = misc->mis_d[k][0], ms1 = misc->mis_d[k][1];
+  // batches of 8 rows: ri = b0 + nwk * i, one transposed reduction each
+#pragma unroll 1
+  for (int b0 = wi; b0 < t.no; b0 += nwk * 8) {
+    float acc[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (i < nr) {
-      const float2 a = BITS == 4 ? dot32_q4(R.w[i], xs, make_float2(0.f, 0.f))
-                                 : dot32_q2(R.w[i].x, xs, make_float2(0.f, 0.f));
-      yv[i] += bf16f(R.sc[i]) * hK * (a.x + a.y) + bf16f(R.bi[i]) * xsum;
+    for (int i = 0; i < 8; ++i) {
+      acc[i] = 0.f;
+      const int ri = b0 + nwk * i;
+      if (live && ri < t.no) {
+        const float a = idot32<BITS>(smem + d_word_smem(g, I, k, ri, lane, BITS), hl);
+        const float s = ld_bf16(smem + d_scale_smem(g, I, k, 0, ms0, ri, gi));
+        const float b = ld_bf16(smem + d_scale_smem(g, I, k, 1, ms1, ri, gi));
+        acc[i] = s * hK * a + b * hs;
+      }
     }
+    const float r = warp_reduce_rows<8>(acc, lane);
+    const int row = reduced_row_of_lane<8>(lane);
+    const int ri = b0 + nwk * row;
+    if (lane == lane_of_reduced_row<8>(row) && ri < t.no) ycomb[k * g.no_max + ri] = r;
   }
 }
 
@@ -260,507 +292,399 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   const int G = gridDim.x, cta = blockIdx.x;
   const int H = p.H, E = p.E, K = p.K, I = p.I;
   const uint64_t deadline = gtimer() + p.budget_ns;
+  const FusedCta t = fused_cta(H, I, G, cta);
+  const bool given = p.given_idx != nullptr;
 
   FusedMisc* misc = (FusedMisc*)(smem + g.off_misc);
   volatile int* abort_flag = &misc->abort;
-  float* xp4 = (float*)(smem + g.off_xp4);
-  float* xp2 = (float*)(smem + g.off_xp2);
-  float* xsum = (float*)(smem + g.off_xs);
-  float* hp = (float*)(smem + g.off_hp);    // [K][I]
-  float* hsum = (float*)(smem + g.off_hs);  // [K][I/32]
-  float* ycomb = (float*)(smem + g.off_ycomb);
+  uint64_t* bars = (uint64_t*)(smem + g.off_bar);
+  float* xn_s = (float*)(smem + g.off_xn);      // raw x, then xn; pieces swizzled per chunk (xswz)
+  float* gred = (float*)(smem + g.off_gred);    // [K*np_max][nq][2] quarter sums
+  float* ycomb = (float*)(smem + g.off_ycomb);  // [K][no_max]
   WsControl* ctl = p.ctl;
 
+  unsigned epoch = 0;
   if (tid == 0) {
+    epoch = ld_relaxed_u32(&ctl->epoch);  // used once the router loads are in flight
     misc->abort = 0;
-    misc->t_lastC = 0;
+    for (int b = 0; b < g.nbar; ++b) mbar_init(&bars[b], 1);
+    fence_mbar_init();
     QE_TRACE(kTrStart);
-    if (p.trace) p.trace[(size_t)cta * 64 + 12] = clock64();
   }
-  if (tid < kMaxK) {
-    misc->hexp[tid] = 0;
-  }
+  if (tid < kMaxK) misc->hamax[tid] = 0u;
 
   // ------------------------------------------------------------- routing
   // The router dot s_e = sum_c W[e,c] x_c gamma_c does not depend on the
-  // RMSNorm scale, so it runs on the same loads as the sum of squares; the
-  // logit is s_e * rinv (+ offset_e), all in fp64.  Warp w covers the column
-  // slice [w*S, (w+1)*S), S = H/16, of each router row its CTA owns; the 16
-  // slice sums are added in slice order.
-  const bool given = p.given_idx != nullptr;
+  // RMSNorm scale, so it runs on the same x loads as the sum of squares; the
+  // logit is s_e * rinv (+ offset_e), in fp64.  CTA c owns rows c, c+G, ...;
+  // thread t covers float4 columns t and t + 512 of each of them.
   const int nrows = (!given && E > cta) ? (E - cta + G - 1) / G : 0;
+  const int nf4 = H / 4;
   {
-    const int S = H / kWarps;
+    // the first (usually only) batch of router rows is requested before x
+    float4 wv[4][2];
+    auto load_rows = [&](int r0) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          const int f = tid + s * kFusedThreads;
+          wv[m][s] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (r0 + m < nrows && f < nf4)
+            wv[m][s] = __ldg((const float4*)(p.router_w + (size_t)(cta + G * (r0 + m)) * H) + f);
+        }
+    };
+    load_rows(0);
+    double xg[2][4];
     double ss = 0.0;
-    for (int r0 = 0; r0 < (nrows > 0 ? nrows : 1); r0 += kRouterBatch) {
-      double acc[kRouterBatch];
 #pragma unroll
-      for (int m = 0; m < kRouterBatch; ++m) acc[m] = 0.0;
-      for (int i = lane; i < S / 4; i += 32) {
-        const int c = warp * S + 4 * i;
-        float4 wv[kRouterBatch];
+    for (int s = 0; s < 2; ++s) {
+      const int f = tid + s * kFusedThreads;
 #pragma unroll
-        for (int m = 0; m < kRouterBatch; ++m)
-          if (r0 + m < nrows) wv[m] = __ldg((const float4*)(p.router_w + (size_t)(cta + G * (r0 + m)) * H + c));
-        double xv[4];
-        load_x4(p, c, xv);
-        if (r0 == 0) {
-          ss += xv[0] * xv[0] + xv[1] * xv[1] + xv[2] * xv[2] + xv[3] * xv[3];
-          // raw x for RMSNorm pass 2 (the x' buffer is free until then)
-          *(float4*)(xp4 + c) = make_float4((float)xv[0], (float)xv[1], (float)xv[2], (float)xv[3]);
-        }
+      for (int i = 0; i < 4; ++i) xg[s][i] = 0.0;
+      if (f < nf4) {
+        load_x4(p, 4 * f, xg[s]);
+        ss += xg[s][0] * xg[s][0] + xg[s][1] * xg[s][1] + xg[s][2] * xg[s][2] + xg[s][3] * xg[s][3];
+        // raw x for RMSNorm pass 2
+        *(float4*)(xn_s + xswz(4 * f)) = make_float4((float)xg[s][0], (float)xg[s][1], (float)xg[s][2], (float)xg[s][3]);
         if (p.gamma) {
-          const float4 gm = *(const float4*)(p.gamma + c);
-          xv[0] *= (double)gm.x; xv[1] *= (double)gm.y; xv[2] *= (double)gm.z; xv[3] *= (double)gm.w;
-        }
-#pragma unroll
-        for (int m = 0; m < kRouterBatch; ++m) {
-          if (r0 + m < nrows) {
-            double a = acc[m];
-            a = fma((double)wv[m].x, xv[0], a);
-            a = fma((double)wv[m].y, xv[1], a);
-            a = fma((double)wv[m].z, xv[2], a);
-            a = fma((double)wv[m].w, xv[3], a);
-            acc[m] = a;
-          }
-        }
-      }
-#pragma unroll
-      for (int m = 0; m < kRouterBatch; ++m) {
-        if (r0 + m < nrows) {
-          const double t = warp_sum_d(acc[m]);
-          if (lane == 0) misc->rpart[r0 + m][warp] = t;
+          const float4 gm = *(const float4*)(p.gamma + 4 * f);
+          xg[s][0] *= (double)gm.x; xg[s][1] *= (double)gm.y; xg[s][2] *= (double)gm.z; xg[s][3] *= (double)gm.w;
         }
       }
     }
-    if (tid == 0) QE_TRACE(56);
+    for (int r0 = 0; r0 < nrows; r0 += 4) {
+      if (r0 > 0) load_rows(r0);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        double a = 0.0;
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          a = fma((double)wv[m][s].x, xg[s][0], a);
+          a = fma((double)wv[m][s].y, xg[s][1], a);
+          a = fma((double)wv[m][s].z, xg[s][2], a);
+          a = fma((double)wv[m][s].w, xg[s][3], a);
+        }
+        if (r0 + m < nrows) {  // uniform over the CTA
+          a = warp_sum_d(a);
+          if (lane == 0) misc->rpart[r0 + m][warp] = a;
+        }
+      }
+    }
     ss = warp_sum_d(ss);
     if (lane == 0) misc->redd[warp] = ss;
   }
+  if (tid == 0) misc->tag = 0x80000000u | ((epoch + 1u) & 0x7FFFFFFFu);
   __syncthreads();
-  if (tid == 0) QE_TRACE(57);
+  if (tid == 0) QE_TRACE(kTrRouter);
+  const unsigned tag = misc->tag;
   double rinv;
   {
     double tot = 0.0;
     for (int w = 0; w < kWarps; ++w) tot += misc->redd[w];
     rinv = 1.0 / sqrt(tot / (double)H + (double)p.eps);
   }
-  if (tid < nrows) {
+  if (tid < nrows && cta != p.skip_cta) {
     double sl = 0.0;
     for (int w = 0; w < kWarps; ++w) sl += misc->rpart[tid][w];
     const int e = cta + G * tid;
-    p.logit_part[e] = sl * rinv + (p.offset ? (double)p.offset[e] : 0.0);
+    const unsigned long long key = dkey(sl * rinv + (p.offset ? (double)p.offset[e] : 0.0));
+    st_rec2(&p.rec_logit[2 * e], rec_word((uint32_t)key, tag), rec_word((uint32_t)(key >> 32), tag));
   }
-  // RMSNorm pass 2 in 32-column chunks (lane = column): xn stays in
-  // registers until the vector exponent of x' is known
-  // (fp32 suffices here: xn feeds the expert matvecs, not the routing)
-  float xnv[kChunkMax];
+  // RMSNorm pass 2 (fp32 suffices: xn feeds the expert matvecs, not the
+  // routing) and max |xn|
   {
     const float rinv_f = (float)rinv;
     float amax = 0.f;
 #pragma unroll
-    for (int q = 0; q < kChunkMax; ++q) {
-      const int ch = warp + kWarps * q;
-      xnv[q] = 0.f;
-      if (ch < H / 32) {
-        const int c = ch * 32 + lane;
-        const float gm = p.gamma ? p.gamma[c] : 1.0f;
-        xnv[q] = xp4[c] * rinv_f * gm;
-        amax = fmaxf(amax, fabsf(xnv[q]));
+    for (int s = 0; s < 2; ++s) {
+      const int f = tid + s * kFusedThreads;
+      if (f < nf4) {
+        float4 v = *(const float4*)(xn_s + xswz(4 * f));
+        float4 gm = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (p.gamma) gm = *(const float4*)(p.gamma + 4 * f);
+        v.x = v.x * rinv_f * gm.x; v.y = v.y * rinv_f * gm.y; v.z = v.z * rinv_f * gm.z; v.w = v.w * rinv_f * gm.w;
+        *(float4*)(xn_s + xswz(4 * f)) = v;
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
       }
     }
     amax = warp_max(amax);
     if (lane == 0) misc->redf[warp] = amax;
   }
-  if (tid == 0) QE_TRACE(58);
-  __syncthreads();
-  if (tid == 0) {
-    QE_TRACE(kTrRouterDone);
-    if (!given) {
-      // the release publishes this CTA's logits; the ticket names the count
-      // that completes this launch's arrivals (a CTA told to skip its
-      // arrival, a test hook, waits for the same count and times out too)
-      const unsigned long long t =
-          cta != p.skip_cta ? atom_add_release_u64(&ctl->route_ctr, 1ull) : ld_acquire_u64(&ctl->route_ctr);
-      misc->route_target = (t / (unsigned)G + 1ull) * (unsigned)G;
-    }
-  }
-  {
-    float m = 0.f;
-    for (int w = 0; w < kWarps; ++w) m = fmaxf(m, misc->redf[w]);
-    const int Ex = xscale_exponent(m);
-    if (tid == 0) misc->xK = acc_scale(Ex);
-    {
-      // the chunk sums of this warp's kChunkMax chunks in one transposed
-      // reduction (chunks past the end hold 0)
-      float sv[kChunkMax];
-#pragma unroll
-      for (int q = 0; q < kChunkMax; ++q) sv[q] = xnv[q];
-      const float sm = warp_reduce_rows<kChunkMax>(sv, lane);
-      const int row = reduced_row_of_lane<kChunkMax>(lane);
-      const int ch = warp + kWarps * row;
-      if (lane == lane_of_reduced_row<kChunkMax>(row) && ch < H / 32) xsum[ch] = sm;
-    }
-#pragma unroll
-    for (int q = 0; q < kChunkMax; ++q) {
-      const int ch = warp + kWarps * q;
-      if (ch < H / 32) {
-        const int c = ch * 32 + lane;
-        xp4[swz_q4(c)] = xprime_q4(xnv[q], c, Ex);
-        xp2[swz_q2(c)] = xprime_q2(xnv[q], c, Ex);
-      }
-    }
-  }
-  if (tid == 0) {
-    if (!given && !wait_geq64(&ctl->route_ctr, misc->route_target, deadline, abort_flag)) {
+
+  // ---------------------------------------------------------------- top-K
+  // Thread t polls the records of experts t and t + 512 and stages their
+  // keys in the expert slots (unused until the copies are issued); warp 0
+  // then takes the top K in K rounds: each lane scans its keys (experts
+  // lane, lane + 32, ...) for the largest one not yet taken, and a warp
+  // arg-max picks the winner (equal keys: the lower expert index).
+  unsigned long long* keys = (unsigned long long*)(smem + g.off_gu);  // [E]
+  if (!given) {
+    const unsigned iA = (unsigned)tid, iB = (unsigned)(tid + kFusedThreads);
+    const bool hasA = (int)iA < E, hasB = (int)iB < E;
+    const unsigned long long* const rp[2] = {hasA ? &p.rec_logit[2 * iA] : nullptr,
+                                             hasB ? &p.rec_logit[2 * iB] : nullptr};
+    unsigned long long lo[2], hi[2];
+    if (!poll_rec2<2>(rp, tag, deadline, abort_flag, lo, hi)) {
       set_error(&ctl->err, QE_ERR_TIMEOUT);
       misc->abort = 1;
     }
-    QE_TRACE(kTrRouteBarrier);
+    if (hasA) keys[iA] = ((unsigned long long)rec_val(hi[0]) << 32) | rec_val(lo[0]);
+    if (hasB) keys[iB] = ((unsigned long long)rec_val(hi[1]) << 32) | rec_val(lo[1]);
+    if (tid == 0) QE_TRACE(kTrLogits);
   }
   __syncthreads();
-
-  // ---------------------------------------------------------------- top-K
-  // Thread t ranks logits t and t+512.  Each warp finds its own top-K by K
-  // rounds of warp_argmax_key (a sorted candidate list, keys and values kept
-  // in shared memory); warp 0 then merges the 16 lists, one list per lane.
-  if (!given && !*abort_flag) {
-    const unsigned iA = (unsigned)tid, iB = (unsigned)(tid + kFusedThreads);
-    bool hasA = tid < E, hasB = tid + kFusedThreads < E;
-    const double vA = hasA ? __ldcg(&p.logit_part[iA]) : 0.0;
-    const double vB = hasB ? __ldcg(&p.logit_part[iB]) : 0.0;
-    const unsigned long long kA = dkey(vA), kB = dkey(vB);
-    for (int k = 0; k < K; ++k) {
-      const bool useA = hasA && (!hasB || kA >= kB);  // equal keys: A has the lower index
-      const unsigned bi = (hasA || hasB) ? (useA ? iA : iB) : 0xffffffffu;
-      const unsigned win = warp_argmax_key(useA ? kA : kB, bi);
-      if (lane == 0) misc->cand_idx[warp][k] = win;
-      if (bi != 0xffffffffu && bi == win) {
-        misc->cand_key[warp][k] = useA ? kA : kB;
-        misc->cand_val[warp][k] = useA ? vA : vB;
-        // warm L1 with the candidate's descriptor while the rounds go on
-        prefetch_l1(&p.experts[win]);
-        prefetch_l1((const unsigned char*)&p.experts[win] + 64);
-        if (useA) hasA = false;
-        else hasB = false;
+  if (warp == 0 && !*abort_flag) {
+    if (given) {
+      // routing decided beforehand: take its experts and weights as they are
+      if (lane < K) {
+        const int e = p.given_idx[lane];
+        misc->idx[lane] = e;
+        misc->wk[lane] = p.given_w[lane];
       }
+    } else {
+      if (lane == 0) QE_TRACE(kTrPolledAll);
+      unsigned taken = 0;  // bit j: expert lane + 32 j is selected
+      for (int k = 0; k < K; ++k) {
+        unsigned bi = 0xffffffffu;
+        unsigned long long bk = 0;
+        for (int j = 0, e = lane; e < E; ++j, e += 32) {
+          const unsigned long long v = keys[e];
+          if (!(taken >> j & 1u) && (bi == 0xffffffffu || v > bk)) {
+            bk = v;
+            bi = (unsigned)e;
+          }
+        }
+        const unsigned win = warp_argmax_key(bk, bi);
+        if (bi != 0xffffffffu && bi == win) {
+          misc->idx[k] = (int)win;
+          misc->selkey[k] = bk;
+          taken |= 1u << ((win - lane) / 32);
+        }
+      }
+      if (lane == 0) QE_TRACE(kTrRounds);
+      __syncwarp();
+      // renormalised softmax over the K kept logits (sum in k order)
+      const double lmax = dkey_inv(misc->selkey[0]);
+      const float ev = lane < K ? expf((float)(dkey_inv(misc->selkey[lane]) - lmax)) : 0.0f;
+      float s = 0.0f;
+      for (int k = 0; k < K; ++k) s += __shfl_sync(0xffffffffu, ev, k);
+      if (lane < K) misc->wk[lane] = ev / s;
     }
-  }
-  __syncthreads();
-  if (warp == 0 && given && !*abort_flag) {
-    // routing decided beforehand: take its experts and weights as they are
+    __syncwarp();
+    if (lane == 0) QE_TRACE(kTrMerged);
     if (lane < K) {
-      const int e = p.given_idx[lane];
-      misc->wk[lane] = p.given_w[lane];
+      const int e = misc->idx[lane];
       if (cta == 0 && p.topk_idx) p.topk_idx[lane] = e;
-      if (cta == 0 && p.topk_w) p.topk_w[lane] = p.given_w[lane];
-      bool ok = e >= 0 && e < E;
+      if (cta == 0 && p.topk_w) p.topk_w[lane] = misc->wk[lane];
       qe_expert ex{};
+      bool ok = e >= 0 && e < E;
       if (ok) {
         ex = p.experts[e];
-        const int bits = ex.gate.bits;
-        ok = (bits == 4 || bits == 2) && desc_ok(ex.gate, bits) && desc_ok(ex.up, bits) && desc_ok(ex.down, bits);
+        ok = expert_ok(ex);
       }
       if (!ok) {
         set_error(&ctl->err, QE_ERR_INVALID_ARG);
         misc->abort = 1;
       }
-      misc->idx[lane] = e;
       misc->ex[lane] = ex;
+      const ExpertAddr a = expert_addr(ex);
+      misc->ea[lane] = a;
+      misc->mis_gu[lane][0] = run_misalign(a.gs, t.r_lo, H / 32);
+      misc->mis_gu[lane][1] = run_misalign(a.gb, t.r_lo, H / 32);
+      misc->mis_gu[lane][2] = run_misalign(a.us, t.r_lo, H / 32);
+      misc->mis_gu[lane][3] = run_misalign(a.ub, t.r_lo, H / 32);
+      misc->mis_d[lane][0] = run_misalign(a.ds, t.o_lo, I / 32);
+      misc->mis_d[lane][1] = run_misalign(a.db, t.o_lo, I / 32);
+      // arm this expert's two mbarriers with the bytes their copies bring
+      if (ok) {
+        const uint32_t ngu = fused_bar_bytes(g, H, I, K, t, misc->ea, bar_gu(lane));
+        const uint32_t nd = fused_bar_bytes(g, H, I, K, t, misc->ea, bar_down(K, lane));
+        if (ngu) mbar_arrive_expect_tx(&bars[bar_gu(lane)], ngu);
+        if (nd) mbar_arrive_expect_tx(&bars[bar_down(K, lane)], nd);
+      }
+    }
+    if (lane == 0) {
+      float m = 0.f;
+      for (int w = 0; w < kWarps; ++w) m = fmaxf(m, misc->redf[w]);
+      misc->Ex = fixed_scale_exponent(m);
+      misc->xK = pow2f(misc->Ex - 22);
+      int ub = misc->ex[0].gate.bits;
+      for (int k = 1; k < K; ++k)
+        if (misc->ex[k].gate.bits != ub) ub = 0;
+      misc->ubits = ub;
     }
   }
-  if (warp == 0 && !given && !*abort_flag) {
-    int ptr = 0;
-    double myval = 0.0;
-    for (int k = 0; k < K; ++k) {
-      unsigned bi = 0xffffffffu;
-      unsigned long long bk = 0;
-      if (lane < kWarps && ptr < K) {
-        bi = misc->cand_idx[lane][ptr];
-        if (bi != 0xffffffffu) bk = misc->cand_key[lane][ptr];
-      }
-      const unsigned win = warp_argmax_key(bk, bi);
-      if (bi != 0xffffffffu && bi == win) {
-        misc->idx[k] = (int)win;
-        myval = misc->cand_val[lane][ptr];
-        ++ptr;
-        misc->lsel[k] = myval;
-      }
-    }
-    __syncwarp();
-    // renormalised softmax over the K kept logits (sum in k order); lanes
-    // k < K also fetch and check the K expert descriptors
-    const double lmax = misc->lsel[0];
-    const float ev = lane < K ? expf((float)(misc->lsel[lane] - lmax)) : 0.0f;
-    float s = 0.0f;
-    for (int k = 0; k < K; ++k) s += __shfl_sync(0xffffffffu, ev, k);
-    if (lane < K) {
-      misc->wk[lane] = ev / s;
-      if (cta == 0 && p.topk_idx) p.topk_idx[lane] = misc->idx[lane];
-      if (cta == 0 && p.topk_w) p.topk_w[lane] = misc->wk[lane];
-      const qe_expert ex = p.experts[misc->idx[lane]];
-      const int bits = ex.gate.bits;
-      if (!(bits == 4 || bits == 2) || !desc_ok(ex.gate, bits) || !desc_ok(ex.up, bits) ||
-          !desc_ok(ex.down, bits)) {
-        set_error(&ctl->err, QE_ERR_INVALID_ARG);
-        misc->abort = 1;
-      }
-      misc->ex[lane] = ex;
-    }
-  }
+  // the keys' generic stores and loads come before the bulk copies' writes
+  // into the same shared memory
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
   if (tid == 0) QE_TRACE(kTrTopK);
 
-  // ---------------------------------------------------------- expert phase
-  const int nBc = g.nB > cta ? (g.nB - cta + G - 1) / G : 0;
-  const int own = g.nCB > cta ? (g.nCB - cta + G - 1) / G : 0;
-  const int MR = g.max_own * kRC;  // rows of one expert's slice of ycomb
-  // down work of this warp: expert k = warp % K, blocks wi, wi + nwk, ...
-  const int ck = warp % K, wi = warp / K, nwk = (kWarps - ck + K - 1) / K;
-  const int myblocks = wi < own ? (own - wi + nwk - 1) / nwk : 0;
-
-  const qe_qmat dmat = misc->ex[ck].down;
-  const int nrow = myblocks * kRC;  // down rows of this warp
-  DownRows R;
-  if (tid < kMaxK) misc->hamax[tid] = 0u;
+  // ------------------------------------------------------- issue the copies
+  // Every warp first copies scale/bias runs with cp.async (so they are ahead
+  // of the bulk traffic), then warp k < K issues expert k's bulk row copies:
+  // gate and up rows, and, after every such warp has issued those, its down
+  // rows.  The CTA barrier below waits for the scale/bias runs.
+  bool issued = false;
+  if (!*abort_flag) {
+    issued = true;
+    const uint64_t pol = policy_evict_first();
+    // run r = 6k + u: u < 4 gate/up scale/bias segment u, u = 4, 5 down scales, biases
+    for (int r = warp; r < 6 * K; r += kWarps) {
+      const int k = r / 6, u = r - 6 * k;
+      if (u < 4 ? t.np > 0 : t.no > 0) {
+        const FusedCopy c =
+            fused_expert_copy(g, H, I, K, t, k, misc->ea[k], u < 4 ? 2 + u : gu_copies(t) + u - 3);
+        const unsigned char* src = (const unsigned char*)(uintptr_t)c.src;
+        for (uint32_t o = 16u * lane; o < c.bytes; o += 512u) cp_async16(smem + c.dst + o, src + o, pol);
+      }
+    }
+    cp_async_commit();
+    if (warp < K) {
+      const ExpertAddr& a = misc->ea[warp];
+      if (lane < 2 && t.np > 0) {
+        const FusedCopy c = fused_expert_copy(g, H, I, K, t, warp, a, lane);
+        bulk_g2s(smem + c.dst, (const void*)(uintptr_t)c.src, c.bytes, &bars[c.bar], pol);
+      }
+      named_barrier(1, 32 * K);
+      if (lane == 0 && t.no > 0) {
+        const FusedCopy c = fused_expert_copy(g, H, I, K, t, warp, a, gu_copies(t));
+        bulk_g2s(smem + c.dst, (const void*)(uintptr_t)c.src, c.bytes, &bars[c.bar], pol);
+      }
+      if (tid == 0) QE_TRACE(kTrIssued);
+    }
+    cp_async_wait<0>();
+  }
   __syncthreads();
 
-  if (!*abort_flag) {
-    // ------------------------------------------------ gate/up, 4-warp groups
-    const int gr = warp >> 2, qd = warp & 3;
-    const int ng = nBc > gr ? (nBc - gr + kGroups - 1) / kGroups : 0;
-    unsigned char* gring = smem + g.off_ring + (size_t)gr * g.nslot * g.slot;
-    const GateUpCtx cx = make_gateup_ctx(H);
-    const uint64_t pol = policy_evict_first();
-    // item t of this group is gate/up item gi = cta + G*(gr + 4t) of the
-    // grid: expert gi / nIB, rows (gi % nIB) * kRB
-    auto item_k = [&](int t, int* r0) {
-      const int gi = cta + G * (gr + kGroups * t);
-      const int k = gi / g.nIB;
-      *r0 = (gi - k * g.nIB) * kRB;
-      return k;
-    };
-    for (int t = 0; t < g.nslot && t < ng; ++t) {
-      int r0;
-      const int k = item_k(t, &r0);
-      issue_gateup(misc->ex[k], r0, gring + (size_t)t * g.slot, qd, cx, lane, pol);
+  // ------------------------------------------------------------- gate/up
+  if (issued && warp < g.nq * g.nrg && t.np > 0) {
+    const int ub = misc->ubits;
+    if (ub == 4) gateup_phase<4>(p, t, misc, bars, xn_s, gred, smem, deadline, warp, lane);
+    else if (ub == 2) gateup_phase<2>(p, t, misc, bars, xn_s, gred, smem, deadline, warp, lane);
+    else gateup_phase<0>(p, t, misc, bars, xn_s, gred, smem, deadline, warp, lane);
+  }
+  __syncthreads();
+  if (tid == 0) QE_TRACE(kTrGateUp);
+  // h = silu(g) * u of this CTA's row pairs, then this CTA's h flag
+  if (issued && !*abort_flag) {
+    for (int P = tid; P < K * t.np; P += kFusedThreads) {
+      float gs = 0.f, us = 0.f;
+      for (int q = 0; q < g.nq; ++q) {
+        gs += gred[(P * g.nq + q) * 2];
+        us += gred[(P * g.nq + q) * 2 + 1];
+      }
+      const float hv = gs / (1.0f + expf(-gs)) * us;
+      const int k = P / t.np, j = P - k * t.np;
+      st_rec(&p.rec_h[(size_t)k * I + t.r_lo + j], rec_word(__float_as_uint(hv), tag));
     }
-    float2 xs[16];
-    int xs_bits = 0;  // bits of the x' form cached in xs (0: none)
-    const bool cache = cx.nlc <= 32;  // one lane chunk of the quarter per lane
-    int slot_i = 0;
-    for (int t = 0; t < ng; ++t) {
-      int r0;
-      const int k = item_k(t, &r0);
-      unsigned char* sl = gring + (size_t)slot_i * g.slot;
-      // copy groups committed after this item's: the items already issued ahead
-      const int later = (t + g.nslot <= ng ? g.nslot : ng - t) - 1;
-      if (later >= 2) cp_async_wait<2>();
-      else if (later == 1) cp_async_wait<1>();
-      else cp_async_wait<0>();
-      __syncwarp();
-      if (threadIdx.x == 0 && t < 2) QE_TRACE(59 + 3 * t);  // item t landed (warp 0)
-      const int bits = misc->ex[k].gate.bits;
-      if (cache && xs_bits != bits && lane < cx.nlc) {
-        if (bits == 4) load_xs32_q4(xp4, qd * cx.nlc + lane, xs);
-        else load_xs32_q2(xp2, qd * cx.nlc + lane, xs);
-      }
-      xs_bits = bits;
-      const float s = bits == 4 ? gateup_partial<4>(sl, qd, cx, xp4, xsum, misc->xK, xs, cache, lane)
-                                : gateup_partial<2>(sl, qd, cx, xp2, xsum, misc->xK, xs, cache, lane);
-      float* red = misc->gred[gr][t & 1][qd];
-#pragma unroll
-      for (int i = 0; i < 2 * kRB; ++i)
-        if (lane == lane_of_reduced_row<2 * kRB>(i)) red[i] = s;
-      if (threadIdx.x == 0 && t < 2) QE_TRACE(60 + 3 * t);  // item t computed (warp 0)
-      named_barrier(1 + gr, 128);
-      if (threadIdx.x == 0 && t == 0) QE_TRACE(61);  // group 0 past item 0
-      if (qd == 0 && lane < kRB) {
-        // lane rr: h of row r0 + rr = silu(g) * u from the four quarter sums
-        float gv = 0.f, uv = 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          gv += misc->gred[gr][t & 1][q][lane];
-          uv += misc->gred[gr][t & 1][q][kRB + lane];
-        }
-        const float hv = gv / (1.0f + expf(-gv)) * uv;
-        p.hbuf[(size_t)k * I + r0 + lane] = hv;  // published once per CTA below
-      }
-      __syncwarp();
-      if (t + g.nslot < ng) {
-        int r1;
-        const int k1 = item_k(t + g.nslot, &r1);
-        issue_gateup(misc->ex[k1], r1, sl, qd, cx, lane, pol);
-      }
-      if (++slot_i == g.nslot) slot_i = 0;
-      if (*abort_flag) break;
-    }
-    cp_async_wait<0>();  // nothing may still be landing when the CTA exits
-    if (lane == 0) QE_TRACE(16 + warp);
-    // this warp's first down rows do not depend on h: load them now
-    if (nrow > 0 && lane < I / 32) down_load(dmat, cta, G, kRC, wi, nwk, 0, nrow < 8 ? nrow : 8, I, lane, R);
   }
 
-  // ------------------------------------- publish h, wait for every CTA's h
-  __syncthreads();
-  if (tid == 0) {
-    QE_TRACE(kTrLastB);
+  // ------------------------------------------------ stage all of h
+  // This CTA's done record goes out after its h records (same threads'
+  // stores, behind a barrier); thread c < G polls CTA c's done record, then
+  // every thread reads its share of h (two records per 16-byte load) into
+  // the gate/up slots (free by now), re-polling any record still stale, and
+  // the CTA finds max |h_k| itself.
+  float* hst = (float*)(smem + g.off_gu);  // [K][I], 16-byte pieces swizzled per 32-column chunk (xswz)
+  if (issued && !*abort_flag) {
+    __syncthreads();
+    if (tid == 0) st_rec(&p.rec_done[kDoneStride * cta], rec_word(0u, tag));
+    bool ok = true;
+    if (tid < G) {
+      unsigned long long w = ld_rec(&p.rec_done[kDoneStride * tid]);
+      for (unsigned spins = 0; rec_tag(w) != tag; ++spins) {
+        if (*abort_flag || ((spins & 7u) == 7u && gtimer() > deadline)) {
+          ok = false;
+          break;
+        }
+        w = ld_rec(&p.rec_done[kDoneStride * tid]);
+      }
+    }
+    if (!ok) {
+      set_error(&ctl->err, QE_ERR_TIMEOUT);
+      misc->abort = 1;
+    }
+    __syncthreads();
+    if (tid == 0) QE_TRACE(kTrHPolled);
     if (!*abort_flag) {
-      // the release publishes the h rows every thread of this CTA stored
-      // before the barrier above
-      const unsigned long long t = atom_add_release_u64(&ctl->h_ctr, 1ull);
-      if (!wait_geq64(&ctl->h_ctr, (t / (unsigned)G + 1ull) * (unsigned)G, deadline, abort_flag)) {
+      const int npair = K * I / 2;
+      for (int b0 = 0; b0 < npair; b0 += 4 * kFusedThreads) {
+        const unsigned long long* rp[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int q = b0 + tid + m * kFusedThreads;
+          rp[m] = q < npair ? &p.rec_h[2 * q] : nullptr;
+        }
+        unsigned long long a[4], b[4];
+        ok = poll_rec2<4>(rp, tag, deadline, abort_flag, a, b) && ok;
+        float mv[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int q = b0 + tid + m * kFusedThreads;
+          float2 v = make_float2(0.f, 0.f);
+          if (q < npair) {
+            v = make_float2(__uint_as_float(rec_val(a[m])), __uint_as_float(rec_val(b[m])));
+            *(float2*)(hst + xswz(2 * q)) = v;
+          }
+          mv[m] = fmaxf(fabsf(v.x), fabsf(v.y));
+        }
+        // the 32 lanes of a warp hold 64 consecutive values of one expert for
+        // each m: one transposed max over the four
+        const float am = warp_reduce_rows_max<4>(mv, lane);
+        const int m = reduced_row_of_lane<4>(lane);
+        const int q0 = b0 + warp * 32 + m * kFusedThreads;
+        if (lane == lane_of_reduced_row<4>(m) && q0 < npair) atomicMax(&misc->hamax[(2 * q0) / I], __float_as_uint(am));
+      }
+      if (!ok) {
         set_error(&ctl->err, QE_ERR_TIMEOUT);
         misc->abort = 1;
-      }
-    }
-    QE_TRACE(kTrHFirst);
-  }
-  __syncthreads();
-
-  // stage h in x' form, all warps: chunk ch of the K*I/32 chunks.  Every CTA
-  // loads all of h, so it finds max |h_k| itself (per-warp maxima, then one
-  // pass over the warps).  When the chunks fit in one round of 8 per warp the
-  // values stay in registers until their exponent is known; otherwise the raw
-  // values go through shared memory and are rewritten in x' form in place
-  // (the x' layout only permutes values inside a chunk).
-  const int per = I / 32, nch = K * per;
-  // every CTA reads all of h at once: start each CTA at another chunk so the
-  // requests spread over the L2 slices instead of queueing on one
-  const int rot = (int)(((unsigned)cta * 37u) % (unsigned)nch);
-  // (k, lc) of the 8 chunks of the round of this warp that starts at ch0
-  auto round_chunks = [&](int ch0, int (&kk)[8], int (&ll)[8]) {
-    int ch = ch0 + rot < nch ? ch0 + rot : ch0 + rot - nch;
-    int k = 0;
-    while (ch >= per) { ch -= per; ++k; }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      kk[i] = k;
-      ll[i] = ch;
-      ch += kWarps;
-      while (ch >= per) { ch -= per; ++k; }
-      while (k >= K) k -= K;  // wrapped past the last expert (rotation)
-    }
-  };
-  const bool one_round = nch <= 8 * kWarps;
-  float v[8];  // one round: the values stay here until their exponent is known
-  if (!*abort_flag) {
-    for (int ch0 = warp; ch0 < nch; ch0 += 8 * kWarps) {
-      int kk[8], ll[8];
-      round_chunks(ch0, kk, ll);
-      // loads issued before any of them is used
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (ch0 + i * kWarps < nch) v[i] = __ldcg(p.hbuf + (size_t)kk[i] * I + ll[i] * 32 + lane);
-      // the 8 chunks' sums and maxima in one transposed reduction each
-      // (chunks past the end hold 0, which changes neither)
-      float sv[8], mv[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (ch0 + i * kWarps >= nch) v[i] = 0.f;
-        sv[i] = v[i];
-        mv[i] = fabsf(v[i]);
-        if (!one_round && ch0 + i * kWarps < nch) hp[(size_t)kk[i] * I + ll[i] * 32 + lane] = v[i];
-      }
-      const float sm = warp_reduce_rows<8>(sv, lane);
-      const float am = warp_reduce_rows_max<8>(mv, lane);
-      const int row = reduced_row_of_lane<8>(lane);
-      if (lane == lane_of_reduced_row<8>(row) && ch0 + row * kWarps < nch) {
-        int k = 0, lc = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (i == row) { k = kk[i]; lc = ll[i]; }
-        hsum[(size_t)k * per + lc] = sm;
-        atomicMax(&misc->hamax[k], __float_as_uint(am));
       }
     }
   }
   __syncthreads();
   if (tid < K) {
-    const int Eh = xscale_exponent(__uint_as_float(misc->hamax[tid]));
+    const int Eh = fixed_scale_exponent(__uint_as_float(misc->hamax[tid]));
     misc->hexp[tid] = Eh;
-    misc->hK[tid] = acc_scale(Eh);
+    misc->hK[tid] = pow2f(Eh - 22);
   }
   __syncthreads();
-  if (!*abort_flag) {
-    if (one_round) {
-      int kk[8], ll[8];
-      round_chunks(warp, kk, ll);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (warp + i * kWarps < nch) {
-          const int k = kk[i], c = ll[i] * 32 + lane;
-          float* hpk = hp + (size_t)k * I;
-          if (misc->ex[k].down.bits == 4) hpk[swz_q4(c)] = xprime_q4(v[i], c, misc->hexp[k]);
-          else hpk[swz_q2(c)] = xprime_q2(v[i], c, misc->hexp[k]);
-        }
-      }
-    } else {
-      // raw values went through shared memory: rewrite each chunk in place
-      for (int ch = warp; ch < nch; ch += kWarps) {
-        int k = 0, lc = ch;
-        while (lc >= per) { lc -= per; ++k; }
-        float* hpk = hp + (size_t)k * I;
-        const int c = lc * 32 + lane;
-        const float x = hpk[c];
-        __syncwarp();
-        if (misc->ex[k].down.bits == 4) hpk[swz_q4(c)] = xprime_q4(x, c, misc->hexp[k]);
-        else hpk[swz_q2(c)] = xprime_q2(x, c, misc->hexp[k]);
-      }
-    }
-  }
-  __syncthreads();
-  if (tid == 0) QE_TRACE(kTrHLast);
+  if (tid == 0) QE_TRACE(kTrHStaged);
 
-  // -------------------------------------------------------- down, warps
-  if (!*abort_flag && nrow > 0) {
-    const int k = ck;
-    const float* hpk = hp + (size_t)k * I;
-    const float* hsk = hsum + (size_t)k * (I / 32);
-    const float hK = misc->hK[k];
-    float* yk = ycomb + (size_t)k * MR;
-    for (int b0 = 0; b0 < nrow; b0 += 8) {
-      const int nr = nrow - b0 < 8 ? nrow - b0 : 8;
-      float yv[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) yv[i] = 0.f;
-      for (int lc = lane; lc < I / 32; lc += 32) {
-        if (!(b0 == 0 && lc == lane)) down_load(dmat, cta, G, kRC, wi, nwk, b0, nr, I, lc, R);
-        if (dmat.bits == 4) down_accum<4>(R, nr, lc, hpk, hsk, hK, yv);
-        else down_accum<2>(R, nr, lc, hpk, hsk, hK, yv);
-      }
-      const float sred = warp_reduce_rows<8>(yv, lane);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (i < nr && lane == lane_of_reduced_row<8>(i)) {
-          const int ri = b0 + i, blk = ri / kRC;
-          yk[(wi + nwk * blk) * kRC + (ri - blk * kRC)] = sred;
-        }
-      }
-    }
-    if (lane == 0 && p.trace) atomicMax(&misc->t_lastC, (unsigned long long)gtimer());
+  // ------------------------------------------------------------------ down
+  // warp w: expert k = w % K, its owned rows wi, wi + nwk, ... (wi = w / K)
+  if (issued && !*abort_flag && t.no > 0 && warp < K * (kWarps / K)) {
+    if (misc->ex[warp % K].down.bits == 4) down_phase<4>(p, t, misc, bars, hst, ycomb, smem, deadline, warp, lane);
+    else down_phase<2>(p, t, misc, bars, hst, ycomb, smem, deadline, warp, lane);
   }
-  if (lane == 0) QE_TRACE(32 + warp);
   __syncthreads();
-  if (tid == 0) QE_TRACE(48);
+  if (tid == 0) QE_TRACE(kTrDown);
 
   // ----------------------------------------------- combine of owned rows
-  if (!*abort_flag) {
-    for (int lr = tid; lr < own * kRC; lr += kFusedThreads) {
-      const int ob = lr / kRC;
-      const int r = (cta + G * ob) * kRC + (lr - ob * kRC);
+  if (issued && !*abort_flag) {
+    for (int i = tid; i < t.no; i += kFusedThreads) {
+      const int r = t.o_lo + i;
       float acc = 0.f;
-      for (int k = 0; k < K; ++k) acc += misc->wk[k] * ycomb[(size_t)k * MR + lr];
+      for (int k = 0; k < K; ++k) acc += misc->wk[k] * ycomb[k * g.no_max + i];
       if (p.add_residual) acc += load_x(p, r);
       p.out[r] = acc;
     }
   }
+  // no copy may still be landing when the CTA exits (they all have, unless
+  // a wait gave up): wait for every armed mbarrier, bounded
+  if (issued) {
+    volatile int no_abort = 0;
+    const uint64_t dl2 = gtimer() + p.budget_ns;
+    for (int b = tid; b < g.nbar; b += kFusedThreads)
+      if (fused_bar_bytes(g, H, I, K, t, misc->ea, b)) mbar_wait(&bars[b], 0, dl2, &no_abort);
+  }
   __syncthreads();
   if (tid == 0) {
-    QE_TRACE(49);
-    if (p.trace) p.trace[(size_t)cta * 64 + kTrLastC] = misc->t_lastC;
+    // every CTA has read the epoch (CTA 0 saw all done records, or gave up
+    // after the wait budget): advance it for the next launch
+    if (cta == 0) st_relaxed_u32(&ctl->epoch, tag & 0x7FFFFFFFu);
     QE_TRACE(kTrEnd);
-    if (p.trace) p.trace[(size_t)cta * 64 + 13] = clock64();
   }
 }
 
@@ -770,47 +694,55 @@ static int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
 int fused_geometry(int H, int E, int K, int I, int sms, int smem_optin, FusedGeometry* out) {
   FusedGeometry g{};
-  // gate/up items of kRB rows in column quarters: H a multiple of 256 keeps
-  // every copied quarter row and scale segment a multiple of 16 bytes
-  if (H % 256 != 0 || I % kRB != 0 || H % kRC != 0) return QE_ERR_UNSUPPORTED;
-  if (E > kRouterRows * sms) return QE_ERR_UNSUPPORTED;
-  if (H > kChunkMax * 32 * kWarps) return QE_ERR_UNSUPPORTED;
-  g.RB = kRB;
-  g.RC = kRC;
-  g.nIB = I / kRB;
-  g.nB = K * g.nIB;
-  g.nCB = H / kRC;
+  // one 32-column chunk per lane: a gate/up row in at most 4 warps, a down
+  // row in one
+  if (H % 64 != 0 || I % 64 != 0 || H > 4096 || I > 1024) return QE_ERR_UNSUPPORTED;
+  if (K < 1 || K > kMaxK || E > 2 * kFusedThreads) return QE_ERR_UNSUPPORTED;
+  if (sms < 1 || sms > kMaxGrid || E > kRouterRows * sms) return QE_ERR_UNSUPPORTED;
   g.grid = sms;
-  g.max_own = (g.nCB + sms - 1) / sms;
-  const int srow = (H % 2048) == 0 ? H / 256 : H / kGroup;
-  g.slot = align_up(kRB * H + 4 * 4 * kRB * srow * 2, 128);
+  g.nq = (H / 32 + 31) / 32;
+  g.nrg = kWarps / g.nq;
+  g.np_max = (I + sms - 1) / sms;
+  g.no_max = (H + sms - 1) / sms;
+  g.gu_row = H / 2;
+  g.gu_sc = align_up(g.np_max * (H / 32) + 30, 16);
+  g.gu_bytes = 2 * g.np_max * g.gu_row + 4 * g.gu_sc;
+  g.d_row = I / 2;
+  g.d_sc = align_up(g.no_max * (I / 32) + 30, 16);
+  g.d_bytes = g.no_max * g.d_row + 2 * g.d_sc;
+  g.nbar = 2 * K;
   int off = 0;
-  g.off_xp4 = off; off = align_up(off + 4 * H, 128);
-  g.off_xp2 = off; off = align_up(off + 4 * H, 128);
-  g.off_xs = off; off = align_up(off + 4 * (H / 32), 128);
-  g.off_hp = off; off = align_up(off + 4 * K * I, 128);
-  g.off_hs = off; off = align_up(off + 4 * K * (I / 32), 128);
-  g.off_ycomb = off; off = align_up(off + 4 * K * g.max_own * kRC, 128);
-  g.off_misc = off; off = align_up(off + (int)sizeof(FusedMisc), 1024);
-  g.off_ring = off;
-  const int budget = smem_optin - off;
-  g.nslot = budget / (kGroups * g.slot);
-  if (g.nslot > 3) g.nslot = 3;
-  if (g.nslot < 1) return QE_ERR_UNSUPPORTED;
-  g.smem_bytes = off + g.nslot * kGroups * g.slot;
+  g.off_misc = off; off = align_up(off + (int)sizeof(FusedMisc), 128);
+  g.off_bar = off; off = align_up(off + 8 * g.nbar, 128);
+  g.off_xn = off; off = align_up(off + 4 * H, 128);
+  g.off_xsum = off; off = align_up(off + 4 * (H / 32), 128);
+  g.off_gred = off; off = align_up(off + 4 * 2 * g.nq * K * g.np_max, 128);
+  g.off_ycomb = off; off = align_up(off + 4 * K * g.no_max, 128);
+  g.off_gu = off;
+  // the top-K keys (8 bytes per expert) and, later, all of h are staged here too
+  int gu_total = K * g.gu_bytes;
+  if (gu_total < 4 * K * I) gu_total = 4 * K * I;
+  if (gu_total < 8 * E) gu_total = 8 * E;
+  off = align_up(off + gu_total, 128);
+  g.off_down = off;
+  off += K * g.d_bytes;
+  g.smem_bytes = align_up(off, 128);
+  if (g.smem_bytes > smem_optin) return QE_ERR_UNSUPPORTED;
   *out = g;
   return QE_OK;
 }
 
 cudaError_t launch_fused_layer(const FusedParams& p, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    int optin = 0, dev = 0;
-    cudaGetDevice(&dev);
+  static int attr_dev = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (attr_dev != dev) {
+    int optin = 0;
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    cudaError_t e = cudaFuncSetAttribute(qe_fused_layer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    e = cudaFuncSetAttribute(qe_fused_layer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_dev = dev;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.g.grid);
@@ -826,3 +758,71 @@ cudaError_t launch_fused_layer(const FusedParams& p, cudaStream_t s) {
 }
 
 }  // namespace qe
+
+// ---------------------------------------------------------------------------
+// Host probe of the single-token kernel's plan (no GPU involved): geometry,
+// the bulk copies of CTA `cta` and the shared-memory offset of every read
+// the kernel makes from them, computed by the same functions the kernel
+// uses.  The CPU tests check the copies against the buffers and every read
+// against the copies.
+extern "C" QE_API int qe_fused_plan_probe(int H, int E, int K, int I, int sms, int smem_optin, int cta,
+                                          const int* bits, const uint64_t* seg /* [K][9] */, int* geom /* [24] */,
+                                          long long* copies /* [max_copies][4] */, int max_copies,
+                                          long long* reads /* [max_reads][6] */, int max_reads) {
+  using namespace qe;
+  FusedGeometry g;
+  const int rc = fused_geometry(H, E, K, I, sms, smem_optin, &g);
+  if (rc != QE_OK) return rc;
+  const int gv[24] = {g.grid, g.nq, g.nrg, g.np_max, g.no_max, g.gu_row, g.gu_sc, g.gu_bytes,
+                      g.d_row, g.d_sc, g.d_bytes, g.nbar, g.off_xn, g.off_xsum, g.off_misc, g.off_bar,
+                      g.off_gred, g.off_ycomb, g.off_gu, g.off_down, g.smem_bytes, 0, 0, 0};
+  for (int i = 0; i < 24; ++i) geom[i] = gv[i];
+  const FusedCta t = fused_cta(H, I, sms, cta);
+  ExpertAddr a[kMaxK];
+  for (int k = 0; k < K; ++k) {
+    const uint64_t* s = seg + 9 * k;
+    a[k] = ExpertAddr{s[0], s[1], s[2], s[3], s[4], s[5], s[6], s[7], s[8], bits[k]};
+  }
+  const int nc = fused_ncopies(K, t);
+  if (nc > max_copies) return QE_ERR_INVALID_ARG;
+  for (int v = 0; v < nc; ++v) {
+    const FusedCopy c = fused_copy_at(g, H, I, K, t, a, v);
+    copies[4 * v] = c.dst;
+    copies[4 * v + 1] = (long long)c.src;
+    copies[4 * v + 2] = c.bytes;
+    copies[4 * v + 3] = c.bar;
+  }
+  // reads: {kind, k, a, b, smem offset, bytes}; kind 0 gate/up word (a =
+  // 2j + m, b = chunk), 1 gate/up scale/bias (a = 4j + s, b = group),
+  // 2 down word (a = row, b = chunk), 3 down scale/bias (a = 2i + s, b = group)
+  int nr = 0;
+  auto put = [&](int kind, int k, int x, int y, int off, int bytes) {
+    if (nr < max_reads) {
+      long long* r = reads + 6 * nr;
+      r[0] = kind; r[1] = k; r[2] = x; r[3] = y; r[4] = off; r[5] = bytes;
+    }
+    ++nr;
+  };
+  for (int k = 0; k < K; ++k) {
+    const int b = a[k].bits;
+    const uint64_t sg[4] = {a[k].gs, a[k].gb, a[k].us, a[k].ub};
+    for (int j = 0; j < t.np; ++j)
+      for (int m = 0; m < 2; ++m)
+        for (int lc = 0; lc < H / 32; ++lc) put(0, k, 2 * j + m, lc, gu_word_smem(g, H, k, j, m, lc, b), b == 4 ? 16 : 8);
+    for (int j = 0; j < t.np; ++j)
+      for (int s = 0; s < 4; ++s)
+        for (int gi = 0; gi < H / 64; ++gi)
+          put(1, k, 4 * j + s, gi, gu_scale_smem(g, H, k, s, run_misalign(sg[s], t.r_lo, H / 32), j, gi), 2);
+    for (int i = 0; i < t.no; ++i)
+      for (int lc = 0; lc < I / 32; ++lc) put(2, k, i, lc, d_word_smem(g, I, k, i, lc, b), b == 4 ? 16 : 8);
+    const uint64_t sd[2] = {a[k].ds, a[k].db};
+    for (int i = 0; i < t.no; ++i)
+      for (int s = 0; s < 2; ++s)
+        for (int gi = 0; gi < I / 64; ++gi)
+          put(3, k, 2 * i + s, gi, d_scale_smem(g, I, k, s, run_misalign(sd[s], t.o_lo, I / 32), i, gi), 2);
+  }
+  geom[21] = nc;
+  geom[22] = nr;
+  geom[23] = t.r_lo;
+  return nr > max_reads ? QE_ERR_INVALID_ARG : QE_OK;
+}

@@ -18,12 +18,11 @@ constexpr int kGroup = 64;
 // Control words at the start of every workspace.
 struct WsControl {
   int err;                       // first device-side error (QE_ERR_*), 0 if none
-  unsigned reserved;
-  // fused kernel grid counters: they only grow, every launch adds its grid
-  // size, and a CTA's arrival ticket tells it the count that ends its wait
-  unsigned long long route_ctr;  // CTAs past the router
-  unsigned long long h_ctr;      // CTAs that published their h rows
-  unsigned pad[58];
+  // launch epoch of the single-token kernel: every launch reads it, tags the
+  // records it publishes with epoch + 1 (top bit set) and, at the end, CTA 0
+  // advances it
+  unsigned epoch;
+  unsigned pad[62];
 };
 static_assert(sizeof(WsControl) == 256, "control block");
 
@@ -53,21 +52,37 @@ struct WsLayout {
   size_t xh;        // fp16   [T*H]  xn for the tensor-core gate/up
   size_t xin;       // float  [T*H]  device copy of a host x (moe_layer_step_host)
   size_t xout;      // float  [T*H]  device result before its copy to the host
+  size_t f_logit;   // u64 [2E]        single-token kernel: tagged router logits (16 B each)
+  size_t f_h;       // u64 [K*I]       single-token kernel: tagged SwiGLU outputs
+  size_t f_done;    // u64 [kMaxGrid * kDoneStride] single-token kernel: per-CTA "h published" records
   size_t total;
 };
 
 WsLayout ws_layout(int H, int E, int K, int I, int T);
 
-// Geometry of the fused single-token kernel.
+// Geometry of the fused single-token kernel (host-computed, passed by value).
+// Each CTA keeps its whole share of the selected experts resident in shared
+// memory: per expert a gate/up slot (np_max row pairs + four scale/bias
+// segments) and a down slot (no_max output rows + two segments).
+constexpr int kMaxGrid = 256;
+// one done record per 128-byte line: every CTA polls all of them, and
+// records packed into a few lines would put all that polling on a few L2
+// slices
+constexpr int kDoneStride = 16;
 struct FusedGeometry {
-  int RB, RC;            // rows of a gate/up item, rows of a down block
-  int nIB, nB, nCB;      // gate/up items per expert, gate/up items, output blocks
-  int max_own;           // most output blocks one CTA owns
-  int slot;              // bytes of one group ring slot
-  int nslot;             // slots per 4-warp group
-  int off_ring, off_xp4, off_xp2, off_xs, off_hp, off_hs, off_ycomb, off_misc;
-  int smem_bytes;
   int grid;
+  int nq, nrg;       // column quarters of a gate/up row; row groups (nq * nrg <= 16 warps)
+  int np_max;        // most gate/up row pairs of one expert in one CTA: ceil(I / grid)
+  int no_max;        // most output rows one CTA owns: ceil(H / grid)
+  int gu_row;        // bytes of a gate/up row slot (4-bit row: H / 2)
+  int gu_sc;         // bytes of a gate/up scale or bias segment slot
+  int gu_bytes;      // bytes of one expert's gate/up slot
+  int d_row;         // bytes of a down row (4-bit: I / 2)
+  int d_sc;          // bytes of a down scale or bias segment slot
+  int d_bytes;       // bytes of one expert's down slot
+  int nbar;          // mbarriers: K (scales) + K * np_max (row pairs) + K (down)
+  int off_xn, off_xsum, off_misc, off_bar, off_gred, off_ycomb, off_gu, off_down;
+  int smem_bytes;
 };
 
 struct FusedParams {
@@ -84,10 +99,11 @@ struct FusedParams {
   int32_t* topk_idx;
   float* topk_w;
   WsControl* ctl;
-  double* logit_part;  // [E] routing logits
-  float* hbuf;         // [K][I]
+  unsigned long long* rec_logit;  // [E][2] {low half | tag, high half | tag} of each fp64 logit
+  unsigned long long* rec_h;      // [K*I] {h bits | tag}
+  unsigned long long* rec_done;   // [grid * kDoneStride] {0 | tag} at c * kDoneStride: CTA c published its h
   // routing decided beforehand (device [K] each), or null: the kernel then
-  // skips the router, the routing barrier and the top-K
+  // skips the router and the top-K
   const int32_t* given_idx;
   const float* given_w;
   FusedGeometry g;
@@ -196,7 +212,8 @@ qe_expert pool_descriptor(const qe_cfg* c, void* base, int bits);
 int route_impl(const qe_cfg* c, const void* x, int x_dtype, const float* gamma, const float* router_w,
                const float* offset, int T, float* xn, int32_t* idx, float* w, void* ws, size_t ws_bytes,
                bool want_xprime, cudaStream_t s);
-bool fused_fits(const qe_cfg* c);
+bool fused_aligned(const void* x, int x_dtype, const float* gamma);
+bool fused_fits(const qe_cfg* c, const void* x, int x_dtype, const float* gamma);
 int fused_step(const qe_cfg* c, const qe_layer* layer, const void* x, int x_dtype, float* out, int add_residual,
                int32_t* topk_idx, float* topk_w, void* ws, const int32_t* given_idx, const float* given_w,
                cudaStream_t s);

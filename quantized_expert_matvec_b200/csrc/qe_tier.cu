@@ -279,7 +279,7 @@ int qe_tier_layer_step(qe_tier* t, int layer, const qe_layer* lw, const void* x,
   int32_t* idx = topk_idx ? topk_idx : (int32_t*)((char*)ws + L.idx);
   float* w = topk_w ? topk_w : (float*)((char*)ws + L.w);
   rc = route_impl(c, x, x_dtype, lw->gamma, lw->router_w, lw->logit_offset, T, nullptr, idx, w, ws, ws_bytes,
-                  !(T == 1 && fused_fits(c)), s);
+                  !(T == 1 && fused_fits(c, x, x_dtype, lw->gamma)), s);
   if (rc) return rc;
   std::lock_guard<std::mutex> lock(t->mu);
   const int n = T * c->top_k;
@@ -293,7 +293,7 @@ int qe_tier_layer_step(qe_tier* t, int layer, const qe_layer* lw, const void* x,
   if (rc) return rc;
   // one token: the fused kernel with this routing (it does not route again,
   // so it reads exactly the experts resolved above)
-  if (T == 1 && fused_fits(c))
+  if (T == 1 && fused_fits(c, x, x_dtype, lw->gamma))
     return fused_step(c, lw, x, x_dtype, out, add_residual, nullptr, nullptr, ws, idx, w, s);
   return experts_and_combine(c, lw->experts, idx, w, x, x_dtype, T, out, add_residual, ws, s);
 }

@@ -10,7 +10,7 @@ import pytest
 
 import oracle
 import synth
-from _util import dev_router, dev_tokens, host_x_f64, routing_matches
+from _util import assert_same_routing, dev_router, dev_tokens, host_x_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -56,9 +56,8 @@ def test_route_ragged_tiles_match_oracle(q, H, E, K, T):
         lg = oracle.router(W_host, xn_ref, offset)
         idx_ref, w_ref = oracle.topk(lg, K)
         assert np.max(np.abs(xn[t] - xn_ref)) <= 1e-6 * np.max(np.abs(xn_ref))
-        assert routing_matches(idx[t], lg, idx_ref, K), (t, idx[t], idx_ref)
-        if list(idx[t]) == list(idx_ref):
-            assert np.max(np.abs(w[t] - w_ref)) <= 1e-6
+        assert_same_routing(idx[t], idx_ref, lg)
+        assert np.max(np.abs(w[t] - w_ref)) <= 1e-6
 
 
 def test_route_deterministic_and_independent_of_batch_position(q):

@@ -10,7 +10,7 @@ import pytest
 
 import oracle
 import synth
-from _util import TOL, dev_router, dev_tokens, fill_pool, normwise_err, routing_matches
+from _util import TOL, assert_same_routing, dev_router, dev_tokens, fill_pool, normwise_err
 
 pytestmark = pytest.mark.gpu
 
@@ -68,13 +68,12 @@ def test_stack_40_layers_full_size(cuda):
         ref = oracle.layer_step(xin, W_h, lambda e: synth.host_expert(seed, l, e, H, I, 4), lambda e: 4, K,
                                 eps=EPS32, offset=offs[l], residual=True, nthreads=16)
         got = idxs[t][l].cpu().numpy()[0]
-        assert routing_matches(got, ref["logits"], ref["idx"], K), (t, l, got, ref["idx"])
+        assert_same_routing(got, ref["idx"], ref["logits"])
         hot_hits += int(synth.hot_set(seed, l, E, E // 4)[got].sum())
-        if list(got) == list(ref["idx"]):
-            err = normwise_err(outs[t][l].cpu().numpy()[0], ref["out"])
-            assert err <= TOL, (t, l, err)
-            n_ok += 1
-    assert n_ok >= len(checks) - 2
+        err = normwise_err(outs[t][l].cpu().numpy()[0], ref["out"])
+        assert err <= TOL, (t, l, err)
+        n_ok += 1
+    assert n_ok == len(checks)
     # the Zipf offset concentrates selections on the hottest quarter of experts
     assert hot_hits / (K * len(checks)) > 0.5
     del pools, Ws, layers, ws, ins, outs, idxs

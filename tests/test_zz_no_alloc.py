@@ -91,3 +91,46 @@ def test_noalloc_rejects_oversized_scratch(cuda):
         q.moe_layer_step_noalloc(cfg, layer, x, out)
     assert ei.value.code == q.QE_ERR_INVALID_ARG
     assert "scratch limit" in str(ei.value)
+
+
+def test_noalloc_at_the_scratch_limit(cuda):
+    """top_k * inter exactly at the built-in limit (16 x 1024): the SwiGLU
+    records fill the scratch array to its end; the result matches the
+    workspace entry point."""
+    import quantized_expert_matvec_b200 as q
+    cfg = q.Cfg(256, 32, 16, 1024)
+    L = _layer(q, cfg, seed=23, layer=0)
+    ws = q.workspace(cfg, 1)
+    x = dev_tokens(23, 5, 1, cfg.hidden)
+    got = _step(q, cfg, L, x, True, noalloc=True)
+    ref = _step(q, cfg, L, x, True, noalloc=False, ws=ws)
+    assert list(got[1]) == list(ref[1])
+    assert np.allclose(got[2], ref[2], rtol=2e-6, atol=1e-7)
+    assert normwise_err(got[0].astype(np.float64), ref[0].astype(np.float64)) <= TOL
+
+
+def test_noalloc_call_after_a_timed_out_call(cuda):
+    """A call whose bounded waits give up (one CTA withholds its router
+    logits, a 20 ms budget) reports QE_ERR_TIMEOUT in dev_status; the next
+    call needs no re-initialisation and matches the workspace entry point."""
+    import torch
+    import quantized_expert_matvec_b200 as q
+    cfg = q.Cfg(1024, 64, 4, 512)
+    L = _layer(q, cfg, seed=22, layer=1)
+    ws = q.workspace(cfg, 1)
+    x = dev_tokens(22, 9, 1, cfg.hidden)
+    out = torch.zeros((1, cfg.hidden), dtype=torch.float32, device="cuda")
+    status = torch.full((1,), -99, dtype=torch.int32, device="cuda")
+    q.qe_set_wait_budget_ns(20_000_000)
+    q.qe_test_skip_arrival(3)
+    try:
+        q.moe_layer_step_noalloc(cfg, L["struct"], x, out, False, None, None, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == q.QE_ERR_TIMEOUT
+    finally:
+        q.qe_test_skip_arrival(-1)
+        q.qe_set_wait_budget_ns(200_000_000)
+    got = _step(q, cfg, L, x, False, noalloc=True)
+    ref = _step(q, cfg, L, x, False, noalloc=False, ws=ws)
+    assert list(got[1]) == list(ref[1])
+    assert normwise_err(got[0].astype(np.float64), ref[0].astype(np.float64)) <= TOL
