@@ -237,7 +237,7 @@ QE_API int moe_layer_step_host(const qe_cfg* cfg, const qe_layer* layer, const v
  * lives.
  *
  * Instead of a workspace it uses a fixed scratch array built into the
- * library (180,480 bytes, 256-byte aligned), which every GPU that loads the
+ * library (172,288 bytes, 256-byte aligned), which every GPU that loads the
  * library holds until the process exits.  It calls no allocation routine.
  *   x       [1,H] device, fp32 or bf16 bits (x_dtype); out [1,H] fp32
  *           device (must not alias x); topk_idx/topk_w [1,K] device outputs
@@ -340,10 +340,11 @@ QE_API void qe_test_skip_arrival(int cta);
  * CTA `cta` of a grid of `sms` CTAs with `smem_optin` bytes of shared memory
  * per block, computed by the functions the kernel itself uses.  bits[K]: the
  * bits of the K selected experts; seg[K*9]: their segment addresses in
- * qe_pool_table's order (any 16-byte aligned values).  Writes geom[24] (the
+ * qe_pool_table's order (any 16-byte aligned values).  Writes geom[64] (the
  * geometry; geom[21] = copies, geom[22] = reads, geom[23] = first gate/up
- * row), copies[n][4] = {shared-memory offset, source address, bytes,
- * mbarrier} and reads[n][6] = {kind, expert, a, b, shared-memory offset,
+ * row, geom[24 + b] = the bytes mbarrier b is armed with), copies[n][4] =
+ * {shared-memory offset, source address, bytes, mbarrier} and reads[n][6] =
+ * {kind, expert, a, b, shared-memory offset,
  * bytes} (kind 0 gate/up word, a = 2*pair + up, b = 32-column chunk; 1
  * gate/up scale or bias, a = 4*pair + segment, b = group; 2 down word, a =
  * owned row, b = chunk; 3 down scale or bias, a = 2*row + segment, b =

@@ -50,7 +50,7 @@ WsLayout ws_layout(int H, int E, int K, int I, int T) {
   L.control = take(sizeof(WsControl));
   // the single-token kernel's records first: their place depends on the
   // shape only, not on T, so no batched call on the same workspace writes there
-  L.f_logit = take(16 * (size_t)E);
+  L.f_logit = take(128 * (size_t)kMaxGrid);
   L.f_h = take(8 * (size_t)K * I);
   L.f_done = take(8 * (size_t)kMaxGrid * kDoneStride);
   const size_t nlog = (size_t)E * (t > 2 ? t : 2);
@@ -423,7 +423,8 @@ extern "C" int moe_layer_step_host(const qe_cfg* c, const qe_layer* layer, const
 //
 // The fused single-token kernel needs device scratch besides its inputs and
 // outputs: the control block (error word, launch epoch), the tagged router
-// logits, the tagged SwiGLU activations and one "h published" record per CTA.
+// logits, the tagged SwiGLU activations and one "read the epoch" record per
+// CTA.
 // moe_layer_step takes them from a caller-allocated workspace; the entry
 // point below takes them from a fixed array that every GPU loading this
 // library holds until the process exits.
@@ -431,9 +432,9 @@ namespace qe {
 
 constexpr size_t kStaticMaxKI = 16384;                                   // top_k * inter: 16 x 1024
 constexpr size_t kStaticLogitsOff = sizeof(WsControl);                   // 256
-constexpr size_t kStaticHOff = kStaticLogitsOff + 16 * (size_t)kMaxE;    // + 16 KiB of logit records
-constexpr size_t kStaticDoneOff = kStaticHOff + 8 * kStaticMaxKI;        // + 128 KiB of h records
-constexpr size_t kStaticBytes = kStaticDoneOff + 8 * (size_t)kMaxGrid * kDoneStride;  // + 32 KiB: 180,480 bytes
+constexpr size_t kStaticHOff = kStaticLogitsOff + 128 * (size_t)kMaxGrid;  // + 32 KiB of logit records
+constexpr size_t kStaticDoneOff = kStaticHOff + 8 * kStaticMaxKI;          // + 128 KiB of h records
+constexpr size_t kStaticBytes = kStaticDoneOff + 8 * (size_t)kMaxGrid * kDoneStride;  // + 8 KiB: 172,288 bytes
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticBytes];
 

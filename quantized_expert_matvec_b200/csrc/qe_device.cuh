@@ -150,9 +150,26 @@ QE_DEV void cp_async8(void* dst, const void* src, uint64_t pol) {
 QE_DEV void cp_async4(void* dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
+QE_DEV void cp_async8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
 QE_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until every cp.async this thread has issued has landed (committed or not).
+QE_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Arrive on an mbarrier once every cp.async this thread has issued so far
+// has landed (the arrival is counted now and completed then, so the
+// barrier's expected count is unchanged).
+QE_DEV void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 template <int N>
 QE_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// Programmatic dependent launch: wait until the kernels this one depends on
+// have finished and their memory is visible (returns at once when the
+// launch had no such dependency), and let the next kernel of the stream
+// start its own prologue.
+QE_DEV void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+QE_DEV void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 QE_DEV void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p)); }
 QE_DEV void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 
@@ -210,6 +227,11 @@ QE_DEV void st_relaxed_u32(unsigned* p, unsigned v) {
 QE_DEV void named_barrier(int id, int count) {
   asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Arrive at named barrier `id` without waiting (a producer: its earlier
+// memory accesses are ordered before the waiters' later ones).
+QE_DEV void named_barrier_arrive(int id, int count) {
+  asm volatile("barrier.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 // Copy `bytes` (a multiple of 16) from global to shared with the 32 lanes of
 // a warp, 16 bytes per lane per step.
@@ -239,13 +261,14 @@ QE_DEV float warp_max(float v) {
   return v;
 }
 
-// Sum R per-lane values over the warp at once (R a power of two <= 32).
+// Sum R per-lane values (float or double) over the warp at once (R a power
+// of two <= 32).
 // Stage o halves the live values: lanes with bit o set keep the upper half.
 // Afterwards the total of value i sits in every lane whose bits
 // (lane>>4, lane>>3, ...) spell i in binary (most significant first);
 // reduced_row_of_lane() gives that index.
-template <int R>
-QE_DEV float warp_reduce_rows(float (&v)[R], int lane) {
+template <int R, typename T>
+QE_DEV T warp_reduce_rows(T (&v)[R], int lane) {
   int live = R;
   int o = 16;
 #pragma unroll
@@ -255,14 +278,14 @@ QE_DEV float warp_reduce_rows(float (&v)[R], int lane) {
 #pragma unroll
     for (int i = 0; i < R / 2; ++i) {
       if (i < half) {
-        float keep = up ? v[i + half] : v[i];
-        float send = up ? v[i] : v[i + half];
+        T keep = up ? v[i + half] : v[i];
+        T send = up ? v[i] : v[i + half];
         v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
       }
     }
     live = half;
   }
-  float s = v[0];
+  T s = v[0];
   for (; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   return s;
 }
@@ -554,6 +577,28 @@ QE_DEV float build_limbs(const float* src, int sw, int e, XLimbs& x) {
     x.b2[r] = (int)prmt(s01, s23, 0x5410u);
   }
   return sum;
+}
+
+// The limbs of one 32-column chunk held in registers (v[c] = column c) under
+// exponent e.
+template <int BITS>
+QE_DEV void build_limbs_reg(const float (&v)[32], int e, XLimbs& x) {
+  const float in = pow2f(22 - e);
+  int vi[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) vi[c] = round_small(v[c] * in);
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    unsigned w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      w[i] = (unsigned)vi[BITS == 4 ? 8 * (r >> 1) + 2 * i + (r & 1) : 16 * (r >> 2) + 4 * i + (r & 3)];
+    const unsigned t01 = prmt(w[0], w[1], 0x5140u), t23 = prmt(w[2], w[3], 0x5140u);
+    const unsigned s01 = prmt(w[0], w[1], 0x0062u), s23 = prmt(w[2], w[3], 0x0062u);
+    x.b0[r] = prmt(t01, t23, 0x5410u);
+    x.b1[r] = prmt(t01, t23, 0x7632u);
+    x.b2[r] = (int)prmt(s01, s23, 0x5410u);
+  }
 }
 
 QE_DEV float limb_sum(int a2, int a1, int a0) {

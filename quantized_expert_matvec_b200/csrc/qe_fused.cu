@@ -45,8 +45,12 @@
 
 namespace qe {
 
-constexpr int kWarps = 16;
-constexpr int kFusedThreads = kWarps * 32;
+constexpr int kWarps = 16;                           // compute warps
+constexpr int kComputeThreads = kWarps * 32;
+constexpr int kFusedThreads = kComputeThreads + 32;  // + the warp that issues the copies
+constexpr int kBarCompute = 1;                       // named barrier of the compute warps
+constexpr int kBarHandoff = 10;                      // warp 0's descriptors, out to the other warps
+// named barriers 2 .. 9: one per expert in the down phase (K <= 8 there)
 constexpr int kRouterRows = 8;  // router rows one CTA owns at most: E <= 8 * grid
 
 struct FusedMisc {
@@ -54,26 +58,23 @@ struct FusedMisc {
   unsigned tag;
   int Ex;    // fixed-point exponent of xn: max|xn| < 2^Ex
   float xK;  // 2^(Ex - 22)
-  int ubits; // bits shared by all K selected experts (4 or 2), 0 if mixed
   int idx[kMaxK];
   float wk[kMaxK];
-  int hexp[kMaxK];  // fixed-point exponent of h_k
-  float hK[kMaxK];  // 2^(hexp - 22)
-  unsigned hamax[kMaxK];  // max |h_k| as float bits
+  int gu_cnt[kMaxK];      // gate/up warps done with expert k
   int mis_gu[kMaxK][4];   // offsets of the gate/up scale/bias runs in their copies
   int mis_d[kMaxK][2];
-  qe_expert ex[kMaxK];
+  qe_expert ex[kMaxK];    // descriptors of the selected experts
   ExpertAddr ea[kMaxK];   // the same descriptors as addresses (copy plan)
   unsigned long long selkey[kMaxK];  // keys of the selected experts, in rank order
-  float redf[kWarps];
+  unsigned amax_bits;  // max |xn| (float bits)
   double redd[kWarps];
   double rpart[kRouterRows][kWarps];
 };
 
 // Optional phase trace: globaltimer stamps per CTA (qe_trace_fused).
 enum {
-  kTrStart, kTrRouter, kTrLogits, kTrTopK, kTrIssued, kTrFirstPair, kTrGateUp, kTrHStaged, kTrDown, kTrEnd,
-  kTrMerged, kTrLastGateUpData, kTrDownData, kTrHPolled, kTrPolledAll, kTrRounds
+  kTrStart, kTrRouter, kTrLogits, kTrTopK, kTrIssued, kTrFirstPair, kTrGateUp, kTrCombined, kTrDown, kTrEnd,
+  kTrMerged, kTrLastGateUpData, kTrDownData, kTrBarsDone, kTrPolledAll, kTrRounds
 };
 #define QE_TRACE(slot) \
   do { if (p.trace) p.trace[(size_t)blockIdx.x * 16 + (slot)] = gtimer(); } while (0)
@@ -115,15 +116,77 @@ static __device__ __forceinline__ double dkey_inv(unsigned long long k) {
   return __longlong_as_double((long long)u);
 }
 
-// Largest key over the warp, the lowest index among equal keys.  Lanes
-// without a candidate pass idx 0xffffffff.  Returns the winning index.
-static __device__ __forceinline__ unsigned warp_argmax_key(unsigned long long key, unsigned idx) {
-  const bool has = idx != 0xffffffffu;
+// Place of expert e's logit record (in 64-bit words): CTA c = e % G writes
+// the records of its rows r = e / G (at most 8) into its own 128-byte line.
+// A line written by several CTAs while every CTA polls it slows the whole
+// exchange down severalfold on B200; one writer per line avoids that.
+static __device__ __forceinline__ size_t logit_rec(int e, int G) { return ((size_t)(e % G) * 8 + e / G) * 2; }
+
+// One candidate of the two-level top-K: a key (0: none) and its expert.
+struct TopKCand {
+  unsigned long long key;
+  unsigned idx;
+  unsigned pad;
+};
+
+// Whether this lane's candidate (key, idx) is the largest key over the
+// warp, the lowest index among equal keys.  Lanes without a candidate pass
+// key 0 and never win.  Keys are compared by their high words first: when
+// one lane alone holds the largest high word (the usual case) it wins;
+// otherwise the low words, then the indices decide.
+static __device__ __forceinline__ bool lane_wins_argmax(unsigned long long key, unsigned idx) {
   const unsigned hi = (unsigned)(key >> 32), lo = (unsigned)key;
-  const unsigned hmax = __reduce_max_sync(0xffffffffu, has ? hi : 0u);
-  const bool top = has && hi == hmax;
+  const unsigned hmax = __reduce_max_sync(0xffffffffu, hi);
+  const bool top = key != 0ull && hi == hmax;
+  const unsigned mt = __ballot_sync(0xffffffffu, top);
+  if (__popc(mt) == 1) return top;  // the same branch for the whole warp
   const unsigned lmax = __reduce_max_sync(0xffffffffu, top ? lo : 0u);
-  return __reduce_min_sync(0xffffffffu, (top && lo == lmax) ? idx : 0xffffffffu);
+  const bool eq = top && lo == lmax;
+  const unsigned m = __ballot_sync(0xffffffffu, eq);
+  if (__popc(m) == 1) return eq;
+  return eq && idx == __reduce_min_sync(0xffffffffu, eq ? idx : 0xffffffffu);
+}
+
+// First level of the top-K, in every compute warp: the K largest of the
+// warp's keys (a lane holds up to two: experts lane + 32 w and that + 512),
+// written largest first to out[0..K) (key 0 where the warp has fewer).  In
+// each round the winning lane moves its second key up.
+static __device__ __forceinline__ void warp_topk_local(unsigned long long kA, unsigned iA, unsigned long long kB,
+                                                       unsigned iB, int K, int lane, TopKCand* out) {
+  const bool sw = kB > kA;  // equal keys: iA, the lower index, first
+  unsigned long long k1 = sw ? kB : kA, k2 = sw ? kA : kB;
+  unsigned i1 = sw ? iB : iA, i2 = sw ? iA : iB;
+  if (lane < K) out[lane] = TopKCand{0ull, 0xffffffffu, 0u};
+  __syncwarp();
+  for (int k = 0; k < K; ++k) {
+    if (lane_wins_argmax(k1, i1)) {
+      out[k] = TopKCand{k1, i1, 0u};
+      k1 = k2;
+      i1 = i2;
+      k2 = 0ull;
+    }
+  }
+}
+
+// Bounded poll of N 8-byte records (p[i], or null to skip) until each
+// carries `tag`; every round reloads all records still stale at once.
+template <int N>
+static __device__ __forceinline__ bool poll_rec(const unsigned long long* const (&p)[N], unsigned tag,
+                                                uint64_t deadline, volatile int* abort_flag) {
+  unsigned long long a[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) a[i] = p[i] ? ld_rec(p[i]) : 0ull;
+  for (unsigned spins = 0;; ++spins) {
+    bool stale = false;
+#pragma unroll
+    for (int i = 0; i < N; ++i) stale |= p[i] && rec_tag(a[i]) != tag;
+    if (!stale) return true;
+    if (*abort_flag) return false;
+    if ((spins & 7u) == 7u && gtimer() > deadline) return false;
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if (p[i] && rec_tag(a[i]) != tag) a[i] = ld_rec(p[i]);
+  }
 }
 
 // Bounded poll of N 16-byte record pairs (p[i] 16-byte aligned, or null to
@@ -153,117 +216,199 @@ static __device__ __forceinline__ bool poll_rec2(const unsigned long long* const
 
 static __device__ __forceinline__ float ld_bf16(const unsigned char* p) { return bf16f(*(const uint16_t*)p); }
 
-// Gate/up phase of one warp: row group rg = warp / nq, column quarter
-// qd = warp % nq, this lane's 32-column chunk lc = 32 qd + lane.  The warp
-// takes the row pairs P = rg, rg + nrg, ... of the flattened (expert, row)
-// list in batches of kPB (one transposed warp reduction per batch: warp
-// shuffles are a scarce resource when all 16 warps reduce), waits for an
-// expert's mbarrier when it first meets that expert, and leaves each pair's
-// two quarter sums in gred.  BITS is the bits of every selected expert, or
-// 0 when they differ (each pair then picks its core).
-constexpr int kPB = 4;
+// A gate/up warp has finished its row pairs of expert k: count it, and the
+// last of the CTA's gate/up warps to do so turns the quarter sums of expert
+// k's rows into h = silu(g) * u and publishes them as tagged records.
+static __device__ __forceinline__ void gateup_expert_done(const FusedParams& p, const FusedCta& t, FusedMisc* misc,
+                                                          const float* gred, int k, int ngu, int lane,
+                                                          unsigned tag) {
+  const FusedGeometry& g = p.g;
+  __threadfence_block();  // this warp's quarter sums before its count
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) last = atomicAdd(&misc->gu_cnt[k], 1) == ngu - 1;
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __threadfence_block();
+  for (int j = lane; j < t.np; j += 32) {
+    const int P = k * t.np + j;
+    float gs = 0.f, us = 0.f;
+    for (int q = 0; q < g.nq; ++q) {
+      gs += gred[(P * g.nq + q) * 2];
+      us += gred[(P * g.nq + q) * 2 + 1];
+    }
+    const float hv = gs / (1.0f + expf(-gs)) * us;
+    st_rec(&p.rec_h[(size_t)k * p.I + t.r_lo + j], rec_word(__float_as_uint(hv), tag));
+  }
+}
+
+// kPB row pairs (gate row j and up row j) of expert k at a time: pair i is
+// j0 + nrg*i.  The body has no branch (a pair past np is computed on pair
+// j0 and dropped), so the compiler interleaves the pairs' loads and dp4a
+// chains.  acc[2i] / acc[2i+1]: this lane's 32-column part of the gate /
+// up dot of pair i.
+constexpr int kPB = 2;
 template <int BITS>
+static __device__ __forceinline__ void gateup_batch(const FusedGeometry& g, int H, int k, int j0, int np,
+                                                    const FusedMisc* misc, const XLimbs& xl, float xsl, float xK,
+                                                    const unsigned char* smem, int lc, bool live,
+                                                    float (&acc)[2 * kPB]) {
+  const int lcs = live ? lc : 0, gi = lcs >> 1;
+#pragma unroll
+  for (int i = 0; i < kPB; ++i) {
+    const int jr = j0 + g.nrg * i;
+    const bool valid = jr < np && live;
+    const int j = jr < np ? jr : j0;
+    const float ag = idot32<BITS>(smem + gu_word_smem(g, H, k, j, 0, lcs, BITS), xl);
+    const float au = idot32<BITS>(smem + gu_word_smem(g, H, k, j, 1, lcs, BITS), xl);
+    const float sg = ld_bf16(smem + gu_scale_smem(g, H, k, 0, misc->mis_gu[k][0], j, gi));
+    const float bg = ld_bf16(smem + gu_scale_smem(g, H, k, 1, misc->mis_gu[k][1], j, gi));
+    const float su = ld_bf16(smem + gu_scale_smem(g, H, k, 2, misc->mis_gu[k][2], j, gi));
+    const float bu = ld_bf16(smem + gu_scale_smem(g, H, k, 3, misc->mis_gu[k][3], j, gi));
+    acc[2 * i] = valid ? sg * xK * ag + bg * xsl : 0.f;
+    acc[2 * i + 1] = valid ? su * xK * au + bu * xsl : 0.f;
+  }
+}
+
+// Gate/up phase of one warp: row group rg = warp / nq, column quarter
+// qd = warp % nq, this lane's 32-column chunk lc = 32 qd + lane.  Expert by
+// expert (the order their bytes arrive in), the warp waits for the
+// expert's copies, takes its row pairs rg, rg + nrg, ... in batches of kPB
+// (one transposed warp reduction per batch leaves each pair's two quarter
+// sums in gred), and reports the expert done.  Once the last expert's
+// bytes are in, a warp has at most one batch left.  The x limbs are
+// rebuilt when the bits change from one expert to the next.
 static __device__ __forceinline__ void gateup_phase(const FusedParams& p, const FusedCta& t, FusedMisc* misc,
                                                     uint64_t* bars, const float* xn_s, float* gred,
-                                                    unsigned char* smem, uint64_t deadline, int warp, int lane) {
+                                                    unsigned char* smem, uint64_t deadline, int warp, int lane,
+                                                    unsigned tag) {
   const FusedGeometry& g = p.g;
-  const int H = p.H, K = p.K;
+  const int H = p.H, K = p.K, np = t.np;
   volatile int* abort_flag = &misc->abort;
+  const int ngu = g.nq * g.nrg;
   const int qd = warp % g.nq, rg = warp / g.nq;
   const int lc = qd * 32 + lane;
   const bool live = lc < H / 32;
-  const int gi = lc >> 1;
-  const int npairs = K * t.np;
   const float xK = misc->xK;
   XLimbs xl;
   float xsl = 0.f;  // sum of this lane's 32 columns of xn
   int xl_bits = 0;
-  int have_k = -1;  // experts [0, have_k] have landed
+  for (int k = 0; k < K; ++k) {
+    if (rg < np) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars[bar_gu(k)], 0, deadline, abort_flag))) {
+        set_error(&p.ctl->err, QE_ERR_TIMEOUT);
+        misc->abort = 1;
+        return;
+      }
+      if (warp == 1 && lane == 0 && k == 0) QE_TRACE(kTrFirstPair);
+      if (warp == 1 && lane == 0 && k == K - 1) QE_TRACE(kTrLastGateUpData);
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) return;  // one decision per warp
+      const int bits = misc->ex[k].gate.bits;
+      if (bits != xl_bits) {
+        if (live) xsl = bits == 4 ? build_limbs<4>(xn_s + 32 * lc, lc & 7, misc->Ex, xl)
+                                  : build_limbs<2>(xn_s + 32 * lc, lc & 7, misc->Ex, xl);
+        xl_bits = bits;
+      }
 #pragma unroll 1
-  for (int p0 = rg; p0 < npairs; p0 += g.nrg * kPB) {
-    if (__any_sync(0xffffffffu, *abort_flag != 0)) break;  // one decision per warp
-    float acc[2 * kPB];
-#pragma unroll
-    for (int i = 0; i < kPB; ++i) {
-      acc[2 * i] = acc[2 * i + 1] = 0.f;
-      const int P = p0 + g.nrg * i;
-      if (P < npairs) {  // uniform over the warp
-        const int k = P / t.np, j = P - k * t.np;
-        const int bits = BITS ? BITS : misc->ex[k].gate.bits;
-        if (bits != xl_bits) {
-          if (live) xsl = bits == 4 ? build_limbs<4>(xn_s + 32 * lc, lc & 7, misc->Ex, xl)
-                                    : build_limbs<2>(xn_s + 32 * lc, lc & 7, misc->Ex, xl);
-          xl_bits = bits;
-        }
-        if (k > have_k) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars[bar_gu(k)], 0, deadline, abort_flag))) {
-            set_error(&p.ctl->err, QE_ERR_TIMEOUT);
-            misc->abort = 1;
-            break;
-          }
-          have_k = k;
-          if (warp == 0 && lane == 0 && P == 0) QE_TRACE(kTrFirstPair);
-          if (warp == 0 && lane == 0 && k == K - 1) QE_TRACE(kTrLastGateUpData);
-        }
-        if (live) {
-          const unsigned char* wg = smem + gu_word_smem(g, H, k, j, 0, lc, bits);
-          const unsigned char* wu = smem + gu_word_smem(g, H, k, j, 1, lc, bits);
-          float ag, au;
-          if (BITS) {
-            ag = idot32<BITS ? BITS : 4>(wg, xl);
-            au = idot32<BITS ? BITS : 4>(wu, xl);
-          } else if (bits == 4) {
-            ag = idot32<4>(wg, xl);
-            au = idot32<4>(wu, xl);
-          } else {
-            ag = idot32<2>(wg, xl);
-            au = idot32<2>(wu, xl);
-          }
-          const float sg = ld_bf16(smem + gu_scale_smem(g, H, k, 0, misc->mis_gu[k][0], j, gi));
-          const float bg = ld_bf16(smem + gu_scale_smem(g, H, k, 1, misc->mis_gu[k][1], j, gi));
-          const float su = ld_bf16(smem + gu_scale_smem(g, H, k, 2, misc->mis_gu[k][2], j, gi));
-          const float bu = ld_bf16(smem + gu_scale_smem(g, H, k, 3, misc->mis_gu[k][3], j, gi));
-          acc[2 * i] = sg * xK * ag + bg * xsl;
-          acc[2 * i + 1] = su * xK * au + bu * xsl;
-        }
+      for (int j0 = rg; j0 < np; j0 += g.nrg * kPB) {
+        float acc[2 * kPB];
+        if (bits == 4) gateup_batch<4>(g, H, k, j0, np, misc, xl, xsl, xK, smem, lc, live, acc);
+        else gateup_batch<2>(g, H, k, j0, np, misc, xl, xsl, xK, smem, lc, live, acc);
+        // batch row 2i = gate, 2i + 1 = up of pair j0 + nrg*i
+        const float r = warp_reduce_rows<2 * kPB>(acc, lane);
+        const int row = reduced_row_of_lane<2 * kPB>(lane);
+        const int j = j0 + g.nrg * (row >> 1);
+        if (lane == lane_of_reduced_row<2 * kPB>(row) && j < np)
+          gred[((k * np + j) * g.nq + qd) * 2 + (row & 1)] = r;
       }
     }
-    // batch row 2i = gate, 2i + 1 = up of pair p0 + nrg*i
-    const float r = warp_reduce_rows<2 * kPB>(acc, lane);
-    const int row = reduced_row_of_lane<2 * kPB>(lane);
-    const int P = p0 + g.nrg * (row >> 1);
-    if (lane == lane_of_reduced_row<2 * kPB>(row) && P < npairs) gred[(P * g.nq + qd) * 2 + (row & 1)] = r;
+    gateup_expert_done(p, t, misc, gred, k, ngu, lane, tag);
   }
 }
 
-// Down phase of one warp: expert k = warp % K, its owned rows wi, wi + nwk,
-// ... (wi = warp / K, nwk = warps per expert), one row at a time, with this
-// lane's 32-column chunk of h_k as limbs in registers; row results go to
-// ycomb.
+// Down phase of one warp, after its gate/up: expert k = warp / nwk, one of
+// the nwk = 16 / K warps of that expert (wi = warp % nwk).  The warp waits
+// until its own CTA has finished expert k's gate/up (the expert's gate/up
+// slot is then free and holds nothing anyone still reads), the nwk warps
+// poll h_k's records together and stage h_k into that slot (16-byte pieces
+// swizzled per 32-column chunk), meet at a named barrier, and compute the
+// owned down rows wi, wi + nwk, ... of expert k in batches of 8 with this
+// lane's 32-column chunk of h_k as limbs.
 template <int BITS>
-static __device__ __forceinline__ void down_phase(const FusedParams& p, const FusedCta& t, FusedMisc* misc,
-                                                  uint64_t* bars, const float* hst, float* ycomb,
-                                                  unsigned char* smem, uint64_t deadline, int warp, int lane) {
+static __device__ __forceinline__ bool down_phase(const FusedParams& p, const FusedCta& t, FusedMisc* misc,
+                                                  uint64_t* bars, float* ycomb, unsigned char* smem,
+                                                  uint64_t deadline, int warp, int lane, unsigned tag) {
   const FusedGeometry& g = p.g;
-  const int K = p.K, I = p.I;
+  const int I = p.I, K = p.K;
   volatile int* abort_flag = &misc->abort;
-  const int k = warp % K, wi = warp / K, nwk = kWarps / K;
-  const bool live = lane < I / 32;
-  const int gi = lane >> 1;
-  XLimbs hl;
-  float hs = 0.f;
-  const int ch = k * (I / 32) + lane;  // this lane's chunk of the staged h
-  if (live) hs = build_limbs<BITS>(hst + 32 * ch, ch & 7, misc->hexp[k], hl);
-  const float hK = misc->hK[k];
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[bar_down(K, k)], 0, deadline, abort_flag));
-  if (warp == 0 && lane == 0) QE_TRACE(kTrDownData);
-  if (!ok) {
-    set_error(&p.ctl->err, QE_ERR_TIMEOUT);
-    misc->abort = 1;
-    return;
+  const int nwk = kWarps / K, k = warp / nwk, wi = warp - k * nwk;
+  const int ngu = g.nq * g.nrg;
+  // Steps 1-2 may give up (abort flag, wait budget), but every warp of the
+  // expert still reaches the named barrier after them exactly once: a warp
+  // that left early would leave its partners waiting there for good.
+  bool ok = !*abort_flag;
+  // 1. this CTA is done with expert k's gate/up
+  if (ok) {
+    volatile int* cnt = &misc->gu_cnt[k];
+    for (unsigned spins = 0; *cnt < ngu; ++spins) {
+      __nanosleep(64);
+      if ((spins & 15u) == 15u && (*abort_flag || gtimer() > deadline)) {
+        ok = false;
+        break;
+      }
+    }
+    __threadfence_block();
   }
+  ok = __all_sync(0xffffffffu, ok);
+  // 2. stage h_k: this warp takes record pairs q = wi*32 + lane + 32*nwk*i,
+  // four at a time, all loads in flight together; the records carry their
+  // own tag, so the poll both waits for the producing CTAs and delivers
+  float* hst = (float*)(smem + gu_slot(g, k));
+  const unsigned long long* hrec = p.rec_h + (size_t)k * I;
+  for (int q0 = wi * 32 + lane; q0 < I / 2 && ok; q0 += 4 * 32 * nwk) {
+    const unsigned long long* rp[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int q = q0 + 32 * nwk * i;
+      rp[i] = q < I / 2 ? hrec + 2 * q : nullptr;
+    }
+    unsigned long long a[4], b[4];
+    ok = poll_rec2<4>(rp, tag, deadline, abort_flag, a, b);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (rp[i])
+        *(float2*)(hst + xswz(2 * (q0 + 32 * nwk * i))) =
+            make_float2(__uint_as_float(rec_val(a[i])), __uint_as_float(rec_val(b[i])));
+  }
+  ok = __all_sync(0xffffffffu, ok);
+  if (nwk > 1) named_barrier(2 + k, 32 * nwk);  // k < 8 when nwk > 1
+  else __syncwarp();
+  if (!ok) return false;
+  // 4. this lane's chunk of h_k, the expert's exponent from the warp's max
+  const bool live = lane < I / 32;
+  float v[32];
+  float amax = 0.f, hs = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (live) f = ((const float4*)(hst + 32 * lane))[i ^ (lane & 7)];
+    v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    hs += v[i];
+    amax = fmaxf(amax, fabsf(v[i]));
+  }
+  const int e = fixed_scale_exponent(warp_max(amax));
+  const float hK = pow2f(e - 22);
+  XLimbs hl;
+  build_limbs_reg<BITS>(v, e, hl);
+  if (t.no == 0) return true;
+  if (!__all_sync(0xffffffffu, mbar_wait(&bars[bar_down(K, k)], 0, deadline, abort_flag))) return false;
+  if (warp == 0 && lane == 0) QE_TRACE(kTrDownData);
+  // 5. rows ri = wi + nwk*i of batch b0, one transposed reduction per batch
+  const int gi = lane >> 1;
   const int ms0 = misc->mis_d[k][0], ms1 = misc->mis_d[k][1];
-  // batches of 8 rows: ri = b0 + nwk * i, one transposed reduction each
 #pragma unroll 1
   for (int b0 = wi; b0 < t.no; b0 += nwk * 8) {
     float acc[8];
@@ -283,6 +428,7 @@ static __device__ __forceinline__ void down_phase(const FusedParams& p, const Fu
     const int ri = b0 + nwk * row;
     if (lane == lane_of_reduced_row<8>(row) && ri < t.no) ycomb[k * g.no_max + ri] = r;
   }
+  return true;
 }
 
 __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const FusedParams p) {
@@ -291,7 +437,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
   const int H = p.H, E = p.E, K = p.K, I = p.I;
-  const uint64_t deadline = gtimer() + p.budget_ns;
   const FusedCta t = fused_cta(H, I, G, cta);
   const bool given = p.given_idx != nullptr;
 
@@ -303,386 +448,364 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   float* ycomb = (float*)(smem + g.off_ycomb);  // [K][no_max]
   WsControl* ctl = p.ctl;
 
+  // Prologue, which may run while the previous kernel of the stream is
+  // still finishing (programmatic dependent launch): shared-memory set-up
+  // and a prefetch of this CTA's router rows into L2 (a hint that reads
+  // nothing back), then the wait for the previous kernel's memory.
+  if (tid == 0) {
+    misc->abort = 0;
+    misc->amax_bits = 0u;
+    for (int b = 0; b < g.nbar; ++b) mbar_init(&bars[b], 1);
+    fence_mbar_init();
+  }
+  if (tid < kMaxK) misc->gu_cnt[tid] = 0;
+  if (!given) {
+    const int nrows_pf = E > cta ? (E - cta + G - 1) / G : 0, lines = H / 32;  // 128-byte lines per row
+    for (int i = tid; i < nrows_pf * lines; i += kFusedThreads)
+      prefetch_l2(p.router_w + (size_t)(cta + G * (i / lines)) * H + 32 * (i % lines));
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const uint64_t deadline = gtimer() + p.budget_ns;
   unsigned epoch = 0;
   if (tid == 0) {
     epoch = ld_relaxed_u32(&ctl->epoch);  // used once the router loads are in flight
-    misc->abort = 0;
-    for (int b = 0; b < g.nbar; ++b) mbar_init(&bars[b], 1);
-    fence_mbar_init();
     QE_TRACE(kTrStart);
   }
-  if (tid < kMaxK) misc->hamax[tid] = 0u;
 
-  // ------------------------------------------------------------- routing
-  // The router dot s_e = sum_c W[e,c] x_c gamma_c does not depend on the
-  // RMSNorm scale, so it runs on the same x loads as the sum of squares; the
-  // logit is s_e * rinv (+ offset_e), in fp64.  CTA c owns rows c, c+G, ...;
-  // thread t covers float4 columns t and t + 512 of each of them.
-  const int nrows = (!given && E > cta) ? (E - cta + G - 1) / G : 0;
-  const int nf4 = H / 4;
-  {
-    // the first (usually only) batch of router rows is requested before x
-    float4 wv[4][2];
-    auto load_rows = [&](int r0) {
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          const int f = tid + s * kFusedThreads;
-          wv[m][s] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (r0 + m < nrows && f < nf4)
-            wv[m][s] = __ldg((const float4*)(p.router_w + (size_t)(cta + G * (r0 + m)) * H) + f);
-        }
-    };
-    load_rows(0);
-    double xg[2][4];
-    double ss = 0.0;
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      const int f = tid + s * kFusedThreads;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) xg[s][i] = 0.0;
-      if (f < nf4) {
-        load_x4(p, 4 * f, xg[s]);
-        ss += xg[s][0] * xg[s][0] + xg[s][1] * xg[s][1] + xg[s][2] * xg[s][2] + xg[s][3] * xg[s][3];
-        // raw x for RMSNorm pass 2
-        *(float4*)(xn_s + xswz(4 * f)) = make_float4((float)xg[s][0], (float)xg[s][1], (float)xg[s][2], (float)xg[s][3]);
-        if (p.gamma) {
-          const float4 gm = *(const float4*)(p.gamma + 4 * f);
-          xg[s][0] *= (double)gm.x; xg[s][1] *= (double)gm.y; xg[s][2] *= (double)gm.z; xg[s][3] *= (double)gm.w;
-        }
-      }
-    }
-    for (int r0 = 0; r0 < nrows; r0 += 4) {
-      if (r0 > 0) load_rows(r0);
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        double a = 0.0;
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          a = fma((double)wv[m][s].x, xg[s][0], a);
-          a = fma((double)wv[m][s].y, xg[s][1], a);
-          a = fma((double)wv[m][s].z, xg[s][2], a);
-          a = fma((double)wv[m][s].w, xg[s][3], a);
-        }
-        if (r0 + m < nrows) {  // uniform over the CTA
-          a = warp_sum_d(a);
-          if (lane == 0) misc->rpart[r0 + m][warp] = a;
-        }
-      }
-    }
-    ss = warp_sum_d(ss);
-    if (lane == 0) misc->redd[warp] = ss;
-  }
-  if (tid == 0) misc->tag = 0x80000000u | ((epoch + 1u) & 0x7FFFFFFFu);
-  __syncthreads();
-  if (tid == 0) QE_TRACE(kTrRouter);
-  const unsigned tag = misc->tag;
-  double rinv;
-  {
-    double tot = 0.0;
-    for (int w = 0; w < kWarps; ++w) tot += misc->redd[w];
-    rinv = 1.0 / sqrt(tot / (double)H + (double)p.eps);
-  }
-  if (tid < nrows && cta != p.skip_cta) {
-    double sl = 0.0;
-    for (int w = 0; w < kWarps; ++w) sl += misc->rpart[tid][w];
-    const int e = cta + G * tid;
-    const unsigned long long key = dkey(sl * rinv + (p.offset ? (double)p.offset[e] : 0.0));
-    st_rec2(&p.rec_logit[2 * e], rec_word((uint32_t)key, tag), rec_word((uint32_t)(key >> 32), tag));
-  }
-  // RMSNorm pass 2 (fp32 suffices: xn feeds the expert matvecs, not the
-  // routing) and max |xn|
-  {
-    const float rinv_f = (float)rinv;
-    float amax = 0.f;
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      const int f = tid + s * kFusedThreads;
-      if (f < nf4) {
-        float4 v = *(const float4*)(xn_s + xswz(4 * f));
-        float4 gm = make_float4(1.f, 1.f, 1.f, 1.f);
-        if (p.gamma) gm = *(const float4*)(p.gamma + 4 * f);
-        v.x = v.x * rinv_f * gm.x; v.y = v.y * rinv_f * gm.y; v.z = v.z * rinv_f * gm.z; v.w = v.w * rinv_f * gm.w;
-        *(float4*)(xn_s + xswz(4 * f)) = v;
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-      }
-    }
-    amax = warp_max(amax);
-    if (lane == 0) misc->redf[warp] = amax;
-  }
-
-  // ---------------------------------------------------------------- top-K
-  // Thread t polls the records of experts t and t + 512 and stages their
-  // keys in the expert slots (unused until the copies are issued); warp 0
-  // then takes the top K in K rounds: each lane scans its keys (experts
-  // lane, lane + 32, ...) for the largest one not yet taken, and a warp
-  // arg-max picks the winner (equal keys: the lower expert index).
-  unsigned long long* keys = (unsigned long long*)(smem + g.off_gu);  // [E]
-  if (!given) {
-    const unsigned iA = (unsigned)tid, iB = (unsigned)(tid + kFusedThreads);
-    const bool hasA = (int)iA < E, hasB = (int)iB < E;
-    const unsigned long long* const rp[2] = {hasA ? &p.rec_logit[2 * iA] : nullptr,
-                                             hasB ? &p.rec_logit[2 * iB] : nullptr};
-    unsigned long long lo[2], hi[2];
-    if (!poll_rec2<2>(rp, tag, deadline, abort_flag, lo, hi)) {
-      set_error(&ctl->err, QE_ERR_TIMEOUT);
-      misc->abort = 1;
-    }
-    if (hasA) keys[iA] = ((unsigned long long)rec_val(hi[0]) << 32) | rec_val(lo[0]);
-    if (hasB) keys[iB] = ((unsigned long long)rec_val(hi[1]) << 32) | rec_val(lo[1]);
-    if (tid == 0) QE_TRACE(kTrLogits);
-  }
-  __syncthreads();
-  if (warp == 0 && !*abort_flag) {
-    if (given) {
-      // routing decided beforehand: take its experts and weights as they are
-      if (lane < K) {
-        const int e = p.given_idx[lane];
-        misc->idx[lane] = e;
-        misc->wk[lane] = p.given_w[lane];
-      }
-    } else {
-      if (lane == 0) QE_TRACE(kTrPolledAll);
-      unsigned taken = 0;  // bit j: expert lane + 32 j is selected
-      for (int k = 0; k < K; ++k) {
-        unsigned bi = 0xffffffffu;
-        unsigned long long bk = 0;
-        for (int j = 0, e = lane; e < E; ++j, e += 32) {
-          const unsigned long long v = keys[e];
-          if (!(taken >> j & 1u) && (bi == 0xffffffffu || v > bk)) {
-            bk = v;
-            bi = (unsigned)e;
-          }
-        }
-        const unsigned win = warp_argmax_key(bk, bi);
-        if (bi != 0xffffffffu && bi == win) {
-          misc->idx[k] = (int)win;
-          misc->selkey[k] = bk;
-          taken |= 1u << ((win - lane) / 32);
-        }
-      }
-      if (lane == 0) QE_TRACE(kTrRounds);
-      __syncwarp();
-      // renormalised softmax over the K kept logits (sum in k order)
-      const double lmax = dkey_inv(misc->selkey[0]);
-      const float ev = lane < K ? expf((float)(dkey_inv(misc->selkey[lane]) - lmax)) : 0.0f;
-      float s = 0.0f;
-      for (int k = 0; k < K; ++k) s += __shfl_sync(0xffffffffu, ev, k);
-      if (lane < K) misc->wk[lane] = ev / s;
-    }
-    __syncwarp();
-    if (lane == 0) QE_TRACE(kTrMerged);
-    if (lane < K) {
-      const int e = misc->idx[lane];
-      if (cta == 0 && p.topk_idx) p.topk_idx[lane] = e;
-      if (cta == 0 && p.topk_w) p.topk_w[lane] = misc->wk[lane];
-      qe_expert ex{};
-      bool ok = e >= 0 && e < E;
-      if (ok) {
-        ex = p.experts[e];
-        ok = expert_ok(ex);
-      }
-      if (!ok) {
-        set_error(&ctl->err, QE_ERR_INVALID_ARG);
-        misc->abort = 1;
-      }
-      misc->ex[lane] = ex;
-      const ExpertAddr a = expert_addr(ex);
-      misc->ea[lane] = a;
-      misc->mis_gu[lane][0] = run_misalign(a.gs, t.r_lo, H / 32);
-      misc->mis_gu[lane][1] = run_misalign(a.gb, t.r_lo, H / 32);
-      misc->mis_gu[lane][2] = run_misalign(a.us, t.r_lo, H / 32);
-      misc->mis_gu[lane][3] = run_misalign(a.ub, t.r_lo, H / 32);
-      misc->mis_d[lane][0] = run_misalign(a.ds, t.o_lo, I / 32);
-      misc->mis_d[lane][1] = run_misalign(a.db, t.o_lo, I / 32);
-      // arm this expert's two mbarriers with the bytes their copies bring
-      if (ok) {
-        const uint32_t ngu = fused_bar_bytes(g, H, I, K, t, misc->ea, bar_gu(lane));
-        const uint32_t nd = fused_bar_bytes(g, H, I, K, t, misc->ea, bar_down(K, lane));
-        if (ngu) mbar_arrive_expect_tx(&bars[bar_gu(lane)], ngu);
-        if (nd) mbar_arrive_expect_tx(&bars[bar_down(K, lane)], nd);
-      }
-    }
-    if (lane == 0) {
-      float m = 0.f;
-      for (int w = 0; w < kWarps; ++w) m = fmaxf(m, misc->redf[w]);
-      misc->Ex = fixed_scale_exponent(m);
-      misc->xK = pow2f(misc->Ex - 22);
-      int ub = misc->ex[0].gate.bits;
-      for (int k = 1; k < K; ++k)
-        if (misc->ex[k].gate.bits != ub) ub = 0;
-      misc->ubits = ub;
-    }
-  }
-  // the keys' generic stores and loads come before the bulk copies' writes
-  // into the same shared memory
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  __syncthreads();
-  if (tid == 0) QE_TRACE(kTrTopK);
-
-  // ------------------------------------------------------- issue the copies
-  // Every warp first copies scale/bias runs with cp.async (so they are ahead
-  // of the bulk traffic), then warp k < K issues expert k's bulk row copies:
-  // gate and up rows, and, after every such warp has issued those, its down
-  // rows.  The CTA barrier below waits for the scale/bias runs.
+  // Every warp of the CTA agrees on `issued` (the copies went out): warp 0
+  // from its lanes' checks, the others from the abort flag it sets before
+  // the hand-off barrier.
   bool issued = false;
-  if (!*abort_flag) {
-    issued = true;
-    const uint64_t pol = policy_evict_first();
-    // run r = 6k + u: u < 4 gate/up scale/bias segment u, u = 4, 5 down scales, biases
-    for (int r = warp; r < 6 * K; r += kWarps) {
-      const int k = r / 6, u = r - 6 * k;
-      if (u < 4 ? t.np > 0 : t.no > 0) {
-        const FusedCopy c =
-            fused_expert_copy(g, H, I, K, t, k, misc->ea[k], u < 4 ? 2 + u : gu_copies(t) + u - 3);
-        const unsigned char* src = (const unsigned char*)(uintptr_t)c.src;
-        for (uint32_t o = 16u * lane; o < c.bytes; o += 512u) cp_async16(smem + c.dst + o, src + o, pol);
-      }
-    }
-    cp_async_commit();
-    if (warp < K) {
-      const ExpertAddr& a = misc->ea[warp];
-      if (lane < 2 && t.np > 0) {
-        const FusedCopy c = fused_expert_copy(g, H, I, K, t, warp, a, lane);
-        bulk_g2s(smem + c.dst, (const void*)(uintptr_t)c.src, c.bytes, &bars[c.bar], pol);
-      }
-      named_barrier(1, 32 * K);
-      if (lane == 0 && t.no > 0) {
-        const FusedCopy c = fused_expert_copy(g, H, I, K, t, warp, a, gu_copies(t));
-        bulk_g2s(smem + c.dst, (const void*)(uintptr_t)c.src, c.bytes, &bars[c.bar], pol);
-      }
-      if (tid == 0) QE_TRACE(kTrIssued);
-    }
-    cp_async_wait<0>();
-  }
-  __syncthreads();
-
-  // ------------------------------------------------------------- gate/up
-  if (issued && warp < g.nq * g.nrg && t.np > 0) {
-    const int ub = misc->ubits;
-    if (ub == 4) gateup_phase<4>(p, t, misc, bars, xn_s, gred, smem, deadline, warp, lane);
-    else if (ub == 2) gateup_phase<2>(p, t, misc, bars, xn_s, gred, smem, deadline, warp, lane);
-    else gateup_phase<0>(p, t, misc, bars, xn_s, gred, smem, deadline, warp, lane);
-  }
-  __syncthreads();
-  if (tid == 0) QE_TRACE(kTrGateUp);
-  // h = silu(g) * u of this CTA's row pairs, then this CTA's h flag
-  if (issued && !*abort_flag) {
-    for (int P = tid; P < K * t.np; P += kFusedThreads) {
-      float gs = 0.f, us = 0.f;
-      for (int q = 0; q < g.nq; ++q) {
-        gs += gred[(P * g.nq + q) * 2];
-        us += gred[(P * g.nq + q) * 2 + 1];
-      }
-      const float hv = gs / (1.0f + expf(-gs)) * us;
-      const int k = P / t.np, j = P - k * t.np;
-      st_rec(&p.rec_h[(size_t)k * I + t.r_lo + j], rec_word(__float_as_uint(hv), tag));
-    }
-  }
-
-  // ------------------------------------------------ stage all of h
-  // This CTA's done record goes out after its h records (same threads'
-  // stores, behind a barrier); thread c < G polls CTA c's done record, then
-  // every thread reads its share of h (two records per 16-byte load) into
-  // the gate/up slots (free by now), re-polling any record still stale, and
-  // the CTA finds max |h_k| itself.
-  float* hst = (float*)(smem + g.off_gu);  // [K][I], 16-byte pieces swizzled per 32-column chunk (xswz)
-  if (issued && !*abort_flag) {
-    __syncthreads();
-    if (tid == 0) st_rec(&p.rec_done[kDoneStride * cta], rec_word(0u, tag));
-    bool ok = true;
-    if (tid < G) {
-      unsigned long long w = ld_rec(&p.rec_done[kDoneStride * tid]);
-      for (unsigned spins = 0; rec_tag(w) != tag; ++spins) {
-        if (*abort_flag || ((spins & 7u) == 7u && gtimer() > deadline)) {
-          ok = false;
-          break;
-        }
-        w = ld_rec(&p.rec_done[kDoneStride * tid]);
-      }
-    }
-    if (!ok) {
-      set_error(&ctl->err, QE_ERR_TIMEOUT);
-      misc->abort = 1;
-    }
-    __syncthreads();
-    if (tid == 0) QE_TRACE(kTrHPolled);
-    if (!*abort_flag) {
-      const int npair = K * I / 2;
-      for (int b0 = 0; b0 < npair; b0 += 4 * kFusedThreads) {
-        const unsigned long long* rp[4];
+  unsigned tag = 0;  // this launch's record tag (compute warps)
+  if (warp < kWarps) {
+    // ------------------------------------------------------------- routing
+    // The router dot s_e = sum_c W[e,c] x_c gamma_c does not depend on the
+    // RMSNorm scale, so it runs on the same x loads as the sum of squares; the
+    // logit is s_e * rinv (+ offset_e), in fp64.  CTA c owns rows c, c+G, ...;
+    // thread t covers float4 columns t and t + 512 of each of them.
+    const int nrows = (!given && E > cta) ? (E - cta + G - 1) / G : 0;
+    const int nf4 = H / 4;
+    {
+      // the first (usually only) batch of router rows is requested before x
+      float4 wv[4][2];
+      auto load_rows = [&](int r0) {
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int q = b0 + tid + m * kFusedThreads;
-          rp[m] = q < npair ? &p.rec_h[2 * q] : nullptr;
-        }
-        unsigned long long a[4], b[4];
-        ok = poll_rec2<4>(rp, tag, deadline, abort_flag, a, b) && ok;
-        float mv[4];
+        for (int m = 0; m < 4; ++m)
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int q = b0 + tid + m * kFusedThreads;
-          float2 v = make_float2(0.f, 0.f);
-          if (q < npair) {
-            v = make_float2(__uint_as_float(rec_val(a[m])), __uint_as_float(rec_val(b[m])));
-            *(float2*)(hst + xswz(2 * q)) = v;
+          for (int s = 0; s < 2; ++s) {
+            const int f = tid + s * kComputeThreads;
+            wv[m][s] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r0 + m < nrows && f < nf4)
+              wv[m][s] = __ldg((const float4*)(p.router_w + (size_t)(cta + G * (r0 + m)) * H) + f);
           }
-          mv[m] = fmaxf(fabsf(v.x), fabsf(v.y));
+      };
+      load_rows(0);
+      double xg[2][4];
+      double ss = 0.0;
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const int f = tid + s * kComputeThreads;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xg[s][i] = 0.0;
+        if (f < nf4) {
+          load_x4(p, 4 * f, xg[s]);
+          ss += xg[s][0] * xg[s][0] + xg[s][1] * xg[s][1] + xg[s][2] * xg[s][2] + xg[s][3] * xg[s][3];
+          // raw x for RMSNorm pass 2
+          *(float4*)(xn_s + xswz(4 * f)) = make_float4((float)xg[s][0], (float)xg[s][1], (float)xg[s][2], (float)xg[s][3]);
+          if (p.gamma) {
+            const float4 gm = *(const float4*)(p.gamma + 4 * f);
+            xg[s][0] *= (double)gm.x; xg[s][1] *= (double)gm.y; xg[s][2] *= (double)gm.z; xg[s][3] *= (double)gm.w;
+          }
         }
-        // the 32 lanes of a warp hold 64 consecutive values of one expert for
-        // each m: one transposed max over the four
-        const float am = warp_reduce_rows_max<4>(mv, lane);
-        const int m = reduced_row_of_lane<4>(lane);
-        const int q0 = b0 + warp * 32 + m * kFusedThreads;
-        if (lane == lane_of_reduced_row<4>(m) && q0 < npair) atomicMax(&misc->hamax[(2 * q0) / I], __float_as_uint(am));
       }
-      if (!ok) {
+      // one transposed warp reduction per batch of 4 rows; the first batch
+      // also carries the sum of squares (value 4 of 8)
+      for (int r0 = 0; r0 == 0 || r0 < nrows; r0 += 4) {
+        if (r0 > 0) load_rows(r0);
+        double a[8];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          a[m] = 0.0;  // rows past nrows were loaded as zeros
+#pragma unroll
+          for (int s = 0; s < 2; ++s) {
+            a[m] = fma((double)wv[m][s].x, xg[s][0], a[m]);
+            a[m] = fma((double)wv[m][s].y, xg[s][1], a[m]);
+            a[m] = fma((double)wv[m][s].z, xg[s][2], a[m]);
+            a[m] = fma((double)wv[m][s].w, xg[s][3], a[m]);
+          }
+        }
+        a[4] = r0 == 0 ? ss : 0.0;
+        a[5] = a[6] = a[7] = 0.0;
+        const double r = warp_reduce_rows<8>(a, lane);
+        const int row = reduced_row_of_lane<8>(lane);
+        if (lane == lane_of_reduced_row<8>(row)) {
+          if (row < 4 && r0 + row < nrows) misc->rpart[r0 + row][warp] = r;
+          if (row == 4 && r0 == 0) misc->redd[warp] = r;
+        }
+      }
+    }
+    if (tid == 0) {
+      const unsigned tg = 0x80000000u | ((epoch + 1u) & 0x7FFFFFFFu);
+      misc->tag = tg;
+      st_rec(&p.rec_done[(size_t)cta * kDoneStride], rec_word(0u, tg));  // this CTA has read the epoch
+    }
+    named_barrier(kBarCompute, kComputeThreads);
+    if (tid == 0) QE_TRACE(kTrRouter);
+    tag = misc->tag;
+    double rinv;
+    {
+      double tot = 0.0;
+      for (int w = 0; w < kWarps; ++w) tot += misc->redd[w];
+      rinv = 1.0 / sqrt(tot / (double)H + (double)p.eps);
+    }
+    if (tid < nrows && cta != p.skip_cta) {
+      double sl = 0.0;
+      for (int w = 0; w < kWarps; ++w) sl += misc->rpart[tid][w];
+      const int e = cta + G * tid;
+      const unsigned long long key = dkey(sl * rinv + (p.offset ? (double)p.offset[e] : 0.0));
+      st_rec2(&p.rec_logit[logit_rec(e, G)], rec_word((uint32_t)key, tag), rec_word((uint32_t)(key >> 32), tag));
+    }
+    // RMSNorm pass 2 (fp32 suffices: xn feeds the expert matvecs, not the
+    // routing) and max |xn|
+    {
+      const float rinv_f = (float)rinv;
+      float amax = 0.f;
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const int f = tid + s * kComputeThreads;
+        if (f < nf4) {
+          float4 v = *(const float4*)(xn_s + xswz(4 * f));
+          float4 gm = make_float4(1.f, 1.f, 1.f, 1.f);
+          if (p.gamma) gm = *(const float4*)(p.gamma + 4 * f);
+          v.x = v.x * rinv_f * gm.x; v.y = v.y * rinv_f * gm.y; v.z = v.z * rinv_f * gm.z; v.w = v.w * rinv_f * gm.w;
+          *(float4*)(xn_s + xswz(4 * f)) = v;
+          amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
+      }
+      amax = warp_max(amax);
+      if (lane == 0) atomicMax(&misc->amax_bits, __float_as_uint(amax));  // non-negative: ordered as integers
+    }
+
+    // ---------------------------------------------------------------- top-K
+    // Two levels.  Thread t polls the records of experts t and t + 512, and
+    // its warp takes the K largest of its keys at once (warp_topk_local);
+    // after the barrier warp 0 merges the 16 sorted lists: lane w holds the
+    // head of warp w's list, and in each of K rounds the winning lane takes
+    // its head and moves to its next one.  Equal keys: the lower expert
+    // index, at both levels.  As each winner is known its descriptor is
+    // requested (cp.async) into shared memory.
+    TopKCand* cand = (TopKCand*)(smem + g.off_cand);  // [kWarps][K]
+    if (!given) {
+      const unsigned iA = (unsigned)tid, iB = (unsigned)(tid + kComputeThreads);
+      const bool hasA = (int)iA < E, hasB = (int)iB < E;
+      const unsigned long long* const rp[2] = {hasA ? &p.rec_logit[logit_rec(iA, G)] : nullptr,
+                                               hasB ? &p.rec_logit[logit_rec(iB, G)] : nullptr};
+      unsigned long long lo[2], hi[2];
+      if (!poll_rec2<2>(rp, tag, deadline, abort_flag, lo, hi)) {
         set_error(&ctl->err, QE_ERR_TIMEOUT);
         misc->abort = 1;
       }
+      if (tid == 0) QE_TRACE(kTrLogits);
+      // a key of 0 stands for "none"; the one key a real logit could map to
+      // 0 (a negative NaN with every payload bit set) is raised to 1
+      unsigned long long kA = ((unsigned long long)rec_val(hi[0]) << 32) | rec_val(lo[0]);
+      unsigned long long kB = ((unsigned long long)rec_val(hi[1]) << 32) | rec_val(lo[1]);
+      kA = hasA ? (kA ? kA : 1ull) : 0ull;
+      kB = hasB ? (kB ? kB : 1ull) : 0ull;
+      warp_topk_local(kA, iA, kB, iB, K, lane, cand + warp * K);
     }
-  }
-  __syncthreads();
-  if (tid < K) {
-    const int Eh = fixed_scale_exponent(__uint_as_float(misc->hamax[tid]));
-    misc->hexp[tid] = Eh;
-    misc->hK[tid] = pow2f(Eh - 22);
-  }
-  __syncthreads();
-  if (tid == 0) QE_TRACE(kTrHStaged);
+    named_barrier(kBarCompute, kComputeThreads);
+    if (warp == 0 && !*abort_flag) {
+      if (given) {
+        // routing decided beforehand: take its experts and weights as they are
+        if (lane < K) {
+          const int e = p.given_idx[lane];
+          misc->idx[lane] = e;
+          misc->wk[lane] = p.given_w[lane];
+          if (e >= 0 && e < E) misc->ex[lane] = p.experts[e];
+        }
+      } else {
+        if (lane == 0) QE_TRACE(kTrPolledAll);
+        const TopKCand* cl = cand + lane * K;
+        int h = 0;
+        TopKCand c = lane < kWarps ? cl[0] : TopKCand{0ull, 0xffffffffu, 0u};
+        for (int k = 0; k < K; ++k) {
+          if (lane_wins_argmax(c.key, c.idx)) {
+            misc->idx[k] = (int)c.idx;
+            misc->selkey[k] = c.key;
+            if ((int)c.idx < E) {  // the descriptor, 8 bytes at a time
+              const unsigned char* src = (const unsigned char*)(p.experts + c.idx);
+              unsigned char* dst = (unsigned char*)&misc->ex[k];
+#pragma unroll
+              for (int q = 0; q < (int)sizeof(qe_expert); q += 8) cp_async8(dst + q, src + q);
+            }
+            ++h;
+            c = h < K ? cl[h] : TopKCand{0ull, 0xffffffffu, 0u};
+          }
+        }
+        cp_async_wait_all();
+        if (lane == 0) QE_TRACE(kTrRounds);
+      }
+      __syncwarp();
+      // the selected experts' descriptors, checked, and what the copies and
+      // the dequant cores need of them
+      bool ok = true;
+      qe_expert ex{};
+      if (lane < K) {
+        const int e = misc->idx[lane];
+        ok = e >= 0 && e < E;
+        if (ok) {
+          ex = misc->ex[lane];
+          ok = expert_ok(ex);
+        }
+        if (!ok) {
+          set_error(&ctl->err, QE_ERR_INVALID_ARG);
+          misc->abort = 1;
+        }
+        const ExpertAddr a = expert_addr(ex);
+        misc->ea[lane] = a;
+        misc->mis_gu[lane][0] = run_misalign(a.gs, t.r_lo, H / 32);
+        misc->mis_gu[lane][1] = run_misalign(a.gb, t.r_lo, H / 32);
+        misc->mis_gu[lane][2] = run_misalign(a.us, t.r_lo, H / 32);
+        misc->mis_gu[lane][3] = run_misalign(a.ub, t.r_lo, H / 32);
+        misc->mis_d[lane][0] = run_misalign(a.ds, t.o_lo, I / 32);
+        misc->mis_d[lane][1] = run_misalign(a.db, t.o_lo, I / 32);
+      }
+      if (lane == 0) {
+        misc->Ex = fixed_scale_exponent(__uint_as_float(misc->amax_bits));
+        misc->xK = pow2f(misc->Ex - 22);
+      }
+      // the descriptors are out: the copy warp issues every copy of the CTA,
+      // the compute warps go on to their gate/up work (and wait for its data
+      // on the mbarriers)
+      const bool all_ok = __all_sync(0xffffffffu, ok);
+      if (lane == 0) QE_TRACE(kTrTopK);
+      named_barrier_arrive(kBarHandoff, kFusedThreads);
+      issued = all_ok;
+      if (!given) {
+        // renormalised softmax over the K kept logits (sum in k order); the
+        // weights are needed at the combine only
+        const double lmax = dkey_inv(misc->selkey[0]);
+        const float ev = lane < K ? expf((float)(dkey_inv(misc->selkey[lane]) - lmax)) : 0.0f;
+        float sum = 0.0f;
+        for (int k = 0; k < K; ++k) sum += __shfl_sync(0xffffffffu, ev, k);
+        if (lane < K) misc->wk[lane] = ev / sum;
+      }
+      if (cta == 0 && lane < K) {
+        if (p.topk_idx) p.topk_idx[lane] = misc->idx[lane];
+        if (p.topk_w) p.topk_w[lane] = misc->wk[lane];
+      }
+      if (lane == 0) QE_TRACE(kTrMerged);
+    } else {
+      named_barrier(kBarHandoff, kFusedThreads);
+      issued = !*abort_flag;
+    }
 
-  // ------------------------------------------------------------------ down
-  // warp w: expert k = w % K, its owned rows wi, wi + nwk, ... (wi = w / K)
-  if (issued && !*abort_flag && t.no > 0 && warp < K * (kWarps / K)) {
-    if (misc->ex[warp % K].down.bits == 4) down_phase<4>(p, t, misc, bars, hst, ycomb, smem, deadline, warp, lane);
-    else down_phase<2>(p, t, misc, bars, hst, ycomb, smem, deadline, warp, lane);
-  }
-  __syncthreads();
-  if (tid == 0) QE_TRACE(kTrDown);
+    // ------------------------------------------ gate/up and down, pipelined
+    // Every warp does its gate/up pairs, then down rows of expert
+    // warp / (16 / K) as soon as that expert is ready; the last warp to finish
+    // an expert's pairs publishes its h.  Experts stream in one after the
+    // other and each group of warps works on its own expert, so the exchange
+    // and the down rows of the early experts overlap the later ones' data.
+    if (issued) {
+      bool ok = true;
+      if (warp < g.nq * g.nrg) {
+        gateup_phase(p, t, misc, bars, xn_s, gred, smem, deadline, warp, lane, tag);
+        if (warp == 0 && lane == 0) QE_TRACE(kTrGateUp);
+      }
+      if (warp < K * (kWarps / K)) {  // every warp of an expert calls it (named barrier inside)
+        ok = misc->ex[warp / (kWarps / K)].down.bits == 4
+                 ? down_phase<4>(p, t, misc, bars, ycomb, smem, deadline, warp, lane, tag)
+                 : down_phase<2>(p, t, misc, bars, ycomb, smem, deadline, warp, lane, tag);
+        if (!ok && lane == 0 && !*abort_flag) {
+          set_error(&ctl->err, QE_ERR_TIMEOUT);
+          misc->abort = 1;
+        }
+      }
+    }
+    named_barrier(kBarCompute, kComputeThreads);
+    if (tid == 0) QE_TRACE(kTrDown);
 
-  // ----------------------------------------------- combine of owned rows
-  if (issued && !*abort_flag) {
-    for (int i = tid; i < t.no; i += kFusedThreads) {
-      const int r = t.o_lo + i;
-      float acc = 0.f;
-      for (int k = 0; k < K; ++k) acc += misc->wk[k] * ycomb[k * g.no_max + i];
-      if (p.add_residual) acc += load_x(p, r);
-      p.out[r] = acc;
+    // ----------------------------------------------- combine of owned rows
+    if (issued && !*abort_flag) {
+      for (int i = tid; i < t.no; i += kComputeThreads) {
+        const int r = t.o_lo + i;
+        float acc = 0.f;
+        for (int k = 0; k < K; ++k) acc += misc->wk[k] * ycomb[k * g.no_max + i];
+        if (p.add_residual) acc += load_x(p, r);
+        p.out[r] = acc;
+      }
+    }
+    if (tid == 0) QE_TRACE(kTrCombined);
+  } else {
+    // ---------------------------------------------------- the copy warp
+    named_barrier(kBarHandoff, kFusedThreads);
+    issued = !*abort_flag;
+    if (issued) {
+      // Expert by expert, its gate/up copies (lane u takes copy u: gate
+      // rows, up rows, the four scale/bias runs), then expert by expert its
+      // down copies: each expert's gate/up bytes are ahead of the next
+      // expert's, and all of them ahead of the down rows.  A bulk copy's
+      // issue waits while the SM's queue of copies is full, so this warp
+      // keeps issuing for most of the stream; nothing else waits on it.
+      const uint64_t pol = policy_evict_first();
+      const int ng = gu_copies(t), nd = d_copies(t);
+      for (int k = 0; k < K; ++k) {
+        if (lane == 0 && ng) mbar_arrive_expect_tx(&bars[bar_gu(k)], fused_bar_bytes(g, H, I, K, t, misc->ea, bar_gu(k)));
+        __syncwarp();
+        if (lane < ng) {
+          const FusedCopy c = fused_expert_copy(g, H, I, K, t, k, misc->ea[k], lane);
+          bulk_g2s(smem + c.dst, (const void*)(uintptr_t)c.src, c.bytes, &bars[c.bar], pol);
+        }
+      }
+      for (int k = 0; k < K; ++k) {
+        if (lane == 0 && nd)
+          mbar_arrive_expect_tx(&bars[bar_down(K, k)], fused_bar_bytes(g, H, I, K, t, misc->ea, bar_down(K, k)));
+        __syncwarp();
+        if (lane < nd) {
+          const FusedCopy c = fused_expert_copy(g, H, I, K, t, k, misc->ea[k], ng + lane);
+          bulk_g2s(smem + c.dst, (const void*)(uintptr_t)c.src, c.bytes, &bars[c.bar], pol);
+        }
+      }
+      if (lane == 0) QE_TRACE(kTrIssued);
+    }
+    // CTA 0 advances the launch epoch at the end: check here, off the
+    // compute warps' path, that every CTA has read it (its "read the epoch"
+    // record, lanes polling CTAs lane, lane + 32, ...).  Every CTA writes
+    // that record right after its router whatever happens later, so this
+    // wait does not end early on an abort: an epoch advanced before a CTA
+    // read it would hand that CTA the next launch's tag.
+    if (cta == 0) {
+      const unsigned tg = misc->tag;  // written before the hand-off
+      for (int c0 = 0; c0 < G; c0 += 8 * 32) {
+        const unsigned long long* rp[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int c = c0 + lane + 32 * i;
+          rp[i] = c < G ? &p.rec_done[(size_t)c * kDoneStride] : nullptr;
+        }
+        volatile int no_abort = 0;
+        if (!poll_rec<8>(rp, tg, deadline, &no_abort)) {
+          set_error(&ctl->err, QE_ERR_TIMEOUT);
+          misc->abort = 1;
+        }
+      }
     }
   }
   // no copy may still be landing when the CTA exits (they all have, unless
   // a wait gave up): wait for every armed mbarrier, bounded
-  if (issued) {
+  if (warp == kWarps && issued) {
     volatile int no_abort = 0;
     const uint64_t dl2 = gtimer() + p.budget_ns;
-    for (int b = tid; b < g.nbar; b += kFusedThreads)
+    for (int b = lane; b < g.nbar; b += 32)
       if (fused_bar_bytes(g, H, I, K, t, misc->ea, b)) mbar_wait(&bars[b], 0, dl2, &no_abort);
   }
+  if (warp == kWarps && lane == 0) QE_TRACE(kTrBarsDone);
   __syncthreads();
   if (tid == 0) {
-    // every CTA has read the epoch (CTA 0 saw all done records, or gave up
-    // after the wait budget): advance it for the next launch
+    // every CTA has read the epoch (CTA 0 saw every CTA's record, or gave
+    // up after the wait budget): advance it for the next launch
     if (cta == 0) st_relaxed_u32(&ctl->epoch, tag & 0x7FFFFFFFu);
     QE_TRACE(kTrEnd);
   }
@@ -697,7 +820,7 @@ int fused_geometry(int H, int E, int K, int I, int sms, int smem_optin, FusedGeo
   // one 32-column chunk per lane: a gate/up row in at most 4 warps, a down
   // row in one
   if (H % 64 != 0 || I % 64 != 0 || H > 4096 || I > 1024) return QE_ERR_UNSUPPORTED;
-  if (K < 1 || K > kMaxK || E > 2 * kFusedThreads) return QE_ERR_UNSUPPORTED;
+  if (K < 1 || K > kMaxK || E > 2 * kComputeThreads) return QE_ERR_UNSUPPORTED;
   if (sms < 1 || sms > kMaxGrid || E > kRouterRows * sms) return QE_ERR_UNSUPPORTED;
   g.grid = sms;
   g.nq = (H / 32 + 31) / 32;
@@ -707,6 +830,7 @@ int fused_geometry(int H, int E, int K, int I, int sms, int smem_optin, FusedGeo
   g.gu_row = H / 2;
   g.gu_sc = align_up(g.np_max * (H / 32) + 30, 16);
   g.gu_bytes = 2 * g.np_max * g.gu_row + 4 * g.gu_sc;
+  if (g.gu_bytes < 4 * I) g.gu_bytes = 4 * I;  // h_k is staged in expert k's slot
   g.d_row = I / 2;
   g.d_sc = align_up(g.no_max * (I / 32) + 30, 16);
   g.d_bytes = g.no_max * g.d_row + 2 * g.d_sc;
@@ -715,15 +839,11 @@ int fused_geometry(int H, int E, int K, int I, int sms, int smem_optin, FusedGeo
   g.off_misc = off; off = align_up(off + (int)sizeof(FusedMisc), 128);
   g.off_bar = off; off = align_up(off + 8 * g.nbar, 128);
   g.off_xn = off; off = align_up(off + 4 * H, 128);
-  g.off_xsum = off; off = align_up(off + 4 * (H / 32), 128);
+  g.off_cand = off; off = align_up(off + (int)sizeof(TopKCand) * kWarps * K, 128);  // top-K candidates
   g.off_gred = off; off = align_up(off + 4 * 2 * g.nq * K * g.np_max, 128);
   g.off_ycomb = off; off = align_up(off + 4 * K * g.no_max, 128);
   g.off_gu = off;
-  // the top-K keys (8 bytes per expert) and, later, all of h are staged here too
-  int gu_total = K * g.gu_bytes;
-  if (gu_total < 4 * K * I) gu_total = 4 * K * I;
-  if (gu_total < 8 * E) gu_total = 8 * E;
-  off = align_up(off + gu_total, 128);
+  off = align_up(off + K * g.gu_bytes, 128);
   g.off_down = off;
   off += K * g.d_bytes;
   g.smem_bytes = align_up(off, 128);
@@ -749,9 +869,14 @@ cudaError_t launch_fused_layer(const FusedParams& p, cudaStream_t s) {
   cfg.blockDim = dim3(kFusedThreads);
   cfg.dynamicSmemBytes = p.g.smem_bytes;
   cfg.stream = s;
+  // Every CTA must be resident at once (one per SM; the CTAs wait on one
+  // another with bounded waits).  No cooperative attribute: with it the
+  // launch does not overlap the previous kernel's tail.  Programmatic
+  // dependent launch lets the CTAs start their prologue on SMs the
+  // previous kernel has left, before that kernel has finished.
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, qe_fused_layer_kernel, p);
@@ -766,7 +891,7 @@ cudaError_t launch_fused_layer(const FusedParams& p, cudaStream_t s) {
 // uses.  The CPU tests check the copies against the buffers and every read
 // against the copies.
 extern "C" QE_API int qe_fused_plan_probe(int H, int E, int K, int I, int sms, int smem_optin, int cta,
-                                          const int* bits, const uint64_t* seg /* [K][9] */, int* geom /* [24] */,
+                                          const int* bits, const uint64_t* seg /* [K][9] */, int* geom /* [64] */,
                                           long long* copies /* [max_copies][4] */, int max_copies,
                                           long long* reads /* [max_reads][6] */, int max_reads) {
   using namespace qe;
@@ -774,7 +899,7 @@ extern "C" QE_API int qe_fused_plan_probe(int H, int E, int K, int I, int sms, i
   const int rc = fused_geometry(H, E, K, I, sms, smem_optin, &g);
   if (rc != QE_OK) return rc;
   const int gv[24] = {g.grid, g.nq, g.nrg, g.np_max, g.no_max, g.gu_row, g.gu_sc, g.gu_bytes,
-                      g.d_row, g.d_sc, g.d_bytes, g.nbar, g.off_xn, g.off_xsum, g.off_misc, g.off_bar,
+                      g.d_row, g.d_sc, g.d_bytes, g.nbar, g.off_xn, g.off_cand, g.off_misc, g.off_bar,
                       g.off_gred, g.off_ycomb, g.off_gu, g.off_down, g.smem_bytes, 0, 0, 0};
   for (int i = 0; i < 24; ++i) geom[i] = gv[i];
   const FusedCta t = fused_cta(H, I, sms, cta);
@@ -792,6 +917,7 @@ extern "C" QE_API int qe_fused_plan_probe(int H, int E, int K, int I, int sms, i
     copies[4 * v + 2] = c.bytes;
     copies[4 * v + 3] = c.bar;
   }
+  for (int b = 0; b < 40; ++b) geom[24 + b] = b < g.nbar ? (int)fused_bar_bytes(g, H, I, K, t, a, b) : 0;
   // reads: {kind, k, a, b, smem offset, bytes}; kind 0 gate/up word (a =
   // 2j + m, b = chunk), 1 gate/up scale/bias (a = 4j + s, b = group),
   // 2 down word (a = row, b = chunk), 3 down scale/bias (a = 2i + s, b = group)

@@ -19,12 +19,12 @@
 //   down slot:    the owned down rows back to back (no_max rows), then two
 //                 segment slots (scales, biases) of d_sc bytes.
 // A bulk copy (TMA engine) costs tens of nanoseconds of issue whatever its
-// size, so every run of consecutive packed rows is ONE bulk copy: the gate
-// rows and the up rows of an expert (on its gate/up mbarrier) and its down
-// rows (on its down mbarrier).  The short scale/bias runs (four per expert
-// for gate/up, two for down, under a kilobyte each at the model's sizes) are
-// copied 16 bytes per thread with cp.async instead, and waited for with the
-// CTA barrier that follows the issue (bar = -1 in the plan).
+// size, so every run of consecutive rows is ONE bulk copy: per expert, the
+// gate rows, the up rows and the four gate/up scale/bias runs (on its
+// gate/up mbarrier), the down rows and the two down scale/bias runs (on its
+// down mbarrier), each mbarrier counting the bytes of its copies.  (Copying
+// the short scale/bias runs with cp.async instead stalls the issuing warp
+// behind the bulk traffic already queued at the SM.)
 // A scale/bias run of consecutive rows starts wherever the rows start; its
 // copy is widened to 16-byte boundaries (every segment is 16-byte aligned
 // and a multiple of 16 bytes long, so the widened copy stays inside it) and
@@ -124,7 +124,7 @@ struct FusedCopy {
   int dst;        // shared-memory offset
   uint64_t src;   // global address
   uint32_t bytes;
-  int bar;        // mbarrier of a bulk copy; -1: a cp.async run
+  int bar;        // the mbarrier that counts the copy's bytes
 };
 
 QE_HD int gu_copies(const FusedCta& t) { return t.np > 0 ? 6 : 0; }
@@ -155,8 +155,6 @@ QE_HD FusedCopy fused_expert_copy(const FusedGeometry& g, int H, int I, int K, c
       const uint64_t seg = sidx == 0 ? a.gs : sidx == 1 ? a.gb : sidx == 2 ? a.us : a.ub;
       c = widened(seg, t.r_lo, t.np, H / 32);
       c.dst = gu_sc_off(g, k, sidx);
-      c.bar = -1;
-      return c;
     } else {
       const uint64_t rowb = (uint64_t)H * (uint64_t)a.bits / 8;
       c.dst = gu_mat_off(g, k, u);
@@ -175,8 +173,6 @@ QE_HD FusedCopy fused_expert_copy(const FusedGeometry& g, int H, int I, int K, c
   } else {
     c = widened(u == 1 ? a.ds : a.db, t.o_lo, t.no, I / 32);
     c.dst = d_sc_off(g, k, u - 1);
-    c.bar = -1;
-    return c;
   }
   c.bar = bar_down(K, k);
   return c;
@@ -191,13 +187,15 @@ QE_HD FusedCopy fused_copy_at(const FusedGeometry& g, int H, int I, int K, const
   return fused_expert_copy(g, H, I, K, t, v / nd, a[v / nd], ng + v % nd);
 }
 
-// Bytes that complete mbarrier b (0 if no copy completes on it): the bulk
-// row copies only.
+// Bytes mbarrier b is armed with: the sum over the copies that complete on
+// it (0 if none does).
 QE_HD uint32_t fused_bar_bytes(const FusedGeometry& g, int H, int I, int K, const FusedCta& t, const ExpertAddr* a,
                                int b) {
-  if (b < K) return t.np > 0 ? 2u * (uint32_t)((uint64_t)H * (uint64_t)a[b].bits / 8 * (uint64_t)t.np) : 0u;
-  const int k = b - K;
-  return t.no > 0 ? (uint32_t)((uint64_t)I * (uint64_t)a[k].bits / 8 * (uint64_t)t.no) : 0u;
+  const int k = b < K ? b : b - K;
+  const int u0 = b < K ? 0 : gu_copies(t), n = b < K ? gu_copies(t) : d_copies(t);
+  uint32_t sum = 0;
+  for (int u = u0; u < u0 + n; ++u) sum += fused_expert_copy(g, H, I, K, t, k, a[k], u).bytes;
+  return sum;
 }
 
 }  // namespace qe

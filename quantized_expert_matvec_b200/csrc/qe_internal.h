@@ -52,9 +52,9 @@ struct WsLayout {
   size_t xh;        // fp16   [T*H]  xn for the tensor-core gate/up
   size_t xin;       // float  [T*H]  device copy of a host x (moe_layer_step_host)
   size_t xout;      // float  [T*H]  device result before its copy to the host
-  size_t f_logit;   // u64 [2E]        single-token kernel: tagged router logits (16 B each)
+  size_t f_logit;   // u64 [kMaxGrid*16] single-token kernel: tagged router logits, one 128-byte line per CTA
   size_t f_h;       // u64 [K*I]       single-token kernel: tagged SwiGLU outputs
-  size_t f_done;    // u64 [kMaxGrid * kDoneStride] single-token kernel: per-CTA "h published" records
+  size_t f_done;    // u64 [kMaxGrid * kDoneStride] single-token kernel: per-CTA "read the epoch" records
   size_t total;
 };
 
@@ -65,10 +65,10 @@ WsLayout ws_layout(int H, int E, int K, int I, int T);
 // memory: per expert a gate/up slot (np_max row pairs + four scale/bias
 // segments) and a down slot (no_max output rows + two segments).
 constexpr int kMaxGrid = 256;
-// one done record per 128-byte line: every CTA polls all of them, and
+// one done record per 32-byte sector: every CTA polls all of them, and
 // records packed into a few lines would put all that polling on a few L2
 // slices
-constexpr int kDoneStride = 16;
+constexpr int kDoneStride = 4;
 struct FusedGeometry {
   int grid;
   int nq, nrg;       // column quarters of a gate/up row; row groups (nq * nrg <= 16 warps)
@@ -80,8 +80,8 @@ struct FusedGeometry {
   int d_row;         // bytes of a down row (4-bit: I / 2)
   int d_sc;          // bytes of a down scale or bias segment slot
   int d_bytes;       // bytes of one expert's down slot
-  int nbar;          // mbarriers: K (scales) + K * np_max (row pairs) + K (down)
-  int off_xn, off_xsum, off_misc, off_bar, off_gred, off_ycomb, off_gu, off_down;
+  int nbar;          // mbarriers: K (gate/up rows) + K (down rows)
+  int off_xn, off_cand, off_misc, off_bar, off_gred, off_ycomb, off_gu, off_down;
   int smem_bytes;
 };
 
@@ -99,9 +99,9 @@ struct FusedParams {
   int32_t* topk_idx;
   float* topk_w;
   WsControl* ctl;
-  unsigned long long* rec_logit;  // [E][2] {low half | tag, high half | tag} of each fp64 logit
+  unsigned long long* rec_logit;  // [kMaxGrid][8][2] per CTA line: {low half | tag, high half | tag} of each fp64 logit
   unsigned long long* rec_h;      // [K*I] {h bits | tag}
-  unsigned long long* rec_done;   // [grid * kDoneStride] {0 | tag} at c * kDoneStride: CTA c published its h
+  unsigned long long* rec_done;   // {0 | tag} at c * kDoneStride: CTA c has read the launch epoch
   // routing decided beforehand (device [K] each), or null: the kernel then
   // skips the router and the top-K
   const int32_t* given_idx;

@@ -8,7 +8,8 @@ and several shapes:
 
 * every copy is 16-byte aligned at both ends, a positive multiple of 16
   bytes, inside its source segment, inside its own shared-memory slot, and
-  overlaps no other copy;
+  overlaps no other copy; each mbarrier is armed with exactly the bytes of
+  the copies that complete on it;
 * every read the kernel makes lies inside one copy, on the mbarrier the
   kernel waits for before that read, and maps back through that copy to
   exactly the global element it is meant to read (computed here from the
@@ -53,7 +54,7 @@ def seg_layout(H, I, bits, k, rng):
 
 
 def probe(lib, H, E, K, I, bits, segs, cta, sms=B200_SMS, optin=B200_OPTIN):
-    geom = (ctypes.c_int * 24)()
+    geom = (ctypes.c_int * 64)()
     maxc, maxr = 4096, 1 << 19
     copies = (ctypes.c_longlong * (4 * maxc))()
     reads = (ctypes.c_longlong * (6 * maxr))()
@@ -66,9 +67,11 @@ def probe(lib, H, E, K, I, bits, segs, cta, sms=B200_SMS, optin=B200_OPTIN):
     cp = np.frombuffer(copies, dtype=np.int64)[: 4 * nc].reshape(nc, 4)
     rd = np.frombuffer(reads, dtype=np.int64)[: 6 * nr].reshape(nr, 6)
     names = ["grid", "nq", "nrg", "np_max", "no_max", "gu_row", "gu_sc", "gu_bytes", "d_row", "d_sc", "d_bytes",
-             "nbar", "off_xn", "off_xsum", "off_misc", "off_bar", "off_gred", "off_ycomb", "off_gu", "off_down",
+             "nbar", "off_xn", "off_cand", "off_misc", "off_bar", "off_gred", "off_ycomb", "off_gu", "off_down",
              "smem_bytes"]
-    return dict(zip(names, g)), cp, rd
+    d = dict(zip(names, g))
+    d["armed"] = g[24:24 + d["nbar"]]
+    return d, cp, rd
 
 
 @pytest.fixture(scope="module")
@@ -96,23 +99,26 @@ def test_plan_copies_and_reads(plib, shape):
         g, cp, rd = probe(plib, H, E, K, I, bits, segs, cta)
         assert g["smem_bytes"] <= B200_OPTIN
         assert g["nq"] * g["nrg"] <= 16 and g["nq"] * 32 * 32 >= H
-        assert g["off_down"] - g["off_gu"] >= 4 * K * I  # h is staged in the gate/up slots
-        assert g["off_down"] - g["off_gu"] >= 8 * E  # so are the top-K keys
+        assert g["off_cand"] + 16 * 16 * K <= g["off_gred"]  # the top-K candidates have their own region
+        assert g["nrg"] * g["nq"] <= 16 and g["gu_bytes"] >= 4 * I  # h_k is staged in expert k's slot
         r_lo, np_ = cta * I // G, (cta + 1) * I // G - cta * I // G
         o_lo, no = cta * H // G, (cta + 1) * H // G - cta * H // G
         assert np_ <= g["np_max"] and no <= g["no_max"]
         # ---- copies
         spans = []
+        armed = np.zeros(g["nbar"], dtype=np.int64)
         for dst, src, nb, bar in cp:
             assert dst % 16 == 0 and src % 16 == 0 and nb % 16 == 0 and nb > 0
-            assert -1 <= bar < g["nbar"]
+            assert 0 <= bar < g["nbar"]
             inside = [(a, n) for s in segs for a, n in s if a <= src and src + nb <= a + n]
             assert len(inside) == 1, (hex(src), nb)
-            if 0 <= bar < K or (bar == -1 and dst < g["off_down"]):
+            if bar < K:
                 assert g["off_gu"] <= dst and dst + nb <= g["off_down"]
             else:
                 assert g["off_down"] <= dst and dst + nb <= g["smem_bytes"]
+            armed[bar] += nb
             spans.append((dst, dst + nb))
+        assert list(armed) == list(g["armed"]), "an mbarrier is armed with other bytes than its copies bring"
         spans.sort()
         for (a0, a1), (b0, _) in zip(spans, spans[1:]):
             assert a1 <= b0, "copies overlap in shared memory"
@@ -141,7 +147,7 @@ def test_plan_copies_and_reads(plib, shape):
         m1 = kind == 1  # gate/up scale or bias: a = 4j + s, b = group
         j, sidx = a // 4, a % 4
         want[m1] = (seg[k, 3 + np.minimum(sidx, 3)] + (r_lo + j) * (H // 32) + 2 * b)[m1]
-        want_bar[m1] = -1  # scale/bias runs: cp.async, then the CTA barrier
+        want_bar[m1] = k[m1]  # scale/bias runs: on the expert's gate/up mbarrier
         m2 = kind == 2  # down word: a = owned row, b = chunk
         want[m2] = (seg[k, 2] + (o_lo + a) * (I * bk // 8) + b * cwb)[m2]
         want_bar[m2] = (K + k)[m2]
@@ -149,7 +155,7 @@ def test_plan_copies_and_reads(plib, shape):
         m3 = kind == 3  # down scale or bias: a = 2i + s, b = group
         i, sidx = a // 2, a % 2
         want[m3] = (seg[k, 7 + np.minimum(sidx, 1)] + (o_lo + i) * (I // 32) + 2 * b)[m3]
-        want_bar[m3] = -1
+        want_bar[m3] = (K + k)[m3]
         assert (m0 | m1 | m2 | m3).all()
         bad = np.nonzero(got != want)[0]
         assert bad.size == 0, rd[bad[:5]]
@@ -159,7 +165,7 @@ def test_plan_copies_and_reads(plib, shape):
 
 
 def test_plan_rejects_shapes_beyond_the_kernel(plib):
-    geom = (ctypes.c_int * 24)()
+    geom = (ctypes.c_int * 64)()
     cp = (ctypes.c_longlong * 4)()
     rd = (ctypes.c_longlong * 6)()
     bits = (ctypes.c_int * 16)(*([4] * 16))
