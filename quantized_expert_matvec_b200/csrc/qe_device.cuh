@@ -115,11 +115,12 @@ QE_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.
+// Bounded wait for the phase with the given parity to complete.  Each try
+// suspends the thread in hardware (up to 10 us, resuming as soon as the
+// phase completes), so waiting warps take no issue slots from working ones.
 QE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t deadline, volatile int* abort_flag) {
-  unsigned spins = 0;
-  while (!mbar_try_wait(bar, parity)) {
-    if ((++spins & 15u) == 0 && (*abort_flag || gtimer() > deadline)) return false;
+  while (!mbar_try_wait_sleep(bar, parity, 10000u)) {
+    if (*abort_flag || gtimer() > deadline) return false;
   }
   return true;
 }

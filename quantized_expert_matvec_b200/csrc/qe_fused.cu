@@ -219,6 +219,9 @@ static __device__ __forceinline__ float ld_bf16(const unsigned char* p) { return
 // A gate/up warp has finished its row pairs of expert k: count it, and the
 // last of the CTA's gate/up warps to do so turns the quarter sums of expert
 // k's rows into h = silu(g) * u and publishes them as tagged records.
+// (Unlike the logits, giving each CTA its own lines here measured slower:
+// the readers' loads of h_k, coalesced four lines a warp in this layout,
+// weigh more than the writers sharing a line.)
 static __device__ __forceinline__ void gateup_expert_done(const FusedParams& p, const FusedCta& t, FusedMisc* misc,
                                                           const float* gred, int k, int ngu, int lane,
                                                           unsigned tag) {

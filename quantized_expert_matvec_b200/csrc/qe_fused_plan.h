@@ -48,12 +48,14 @@ struct FusedCta {
   int o_lo, no;  // output rows [o_lo, o_lo + no)
 };
 
+// 32-bit arithmetic: c <= 256 and H, I <= 4096 in this kernel (a 64-bit
+// division is a long instruction sequence on the GPU).
 QE_HD FusedCta fused_cta(int H, int I, int G, int c) {
   FusedCta t;
-  t.r_lo = (int)((long long)c * I / G);
-  t.np = (int)((long long)(c + 1) * I / G) - t.r_lo;
-  t.o_lo = (int)((long long)c * H / G);
-  t.no = (int)((long long)(c + 1) * H / G) - t.o_lo;
+  t.r_lo = c * I / G;
+  t.np = (c + 1) * I / G - t.r_lo;
+  t.o_lo = c * H / G;
+  t.no = (c + 1) * H / G - t.o_lo;
   return t;
 }
 

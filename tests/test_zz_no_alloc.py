@@ -95,7 +95,7 @@ def test_noalloc_rejects_oversized_scratch(cuda):
 
 def test_noalloc_at_the_scratch_limit(cuda):
     """top_k * inter exactly at the built-in limit (16 x 1024): the SwiGLU
-    records fill the scratch array to its end; the result matches the
+    records fill their part of the scratch array; the result matches the
     workspace entry point."""
     import quantized_expert_matvec_b200 as q
     cfg = q.Cfg(256, 32, 16, 1024)
