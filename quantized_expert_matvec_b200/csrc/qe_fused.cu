@@ -144,7 +144,10 @@ static __device__ __forceinline__ bool lane_wins_argmax(unsigned long long key, 
   const bool eq = top && lo == lmax;
   const unsigned m = __ballot_sync(0xffffffffu, eq);
   if (__popc(m) == 1) return eq;
-  return eq && idx == __reduce_min_sync(0xffffffffu, eq ? idx : 0xffffffffu);
+  // every lane takes part in the collective (a full-mask reduction that
+  // some lanes skipped, as under a short-circuited &&, would never finish)
+  const unsigned imin = __reduce_min_sync(0xffffffffu, eq ? idx : 0xffffffffu);
+  return eq && idx == imin;
 }
 
 // First level of the top-K, in every compute warp: the K largest of the
