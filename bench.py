@@ -68,17 +68,17 @@ def expert_bytes(H, I, bits):
 
 
 KERNEL_SOURCES = {  # the sources the dominant kernel of each workload is compiled from
-    "c1": ("qe_fused.cu", "qe_device.cuh"),
-    "c0": ("qe_fused.cu", "qe_device.cuh"),
-    "c2": ("qe_fused.cu", "qe_device.cuh"),
-    "c4": ("qe_grouped.cu", "qe_device.cuh"),
+    "c1": ("qe_fused.cu", "qe_device.cuh", "qe_fused_plan.h", "qe_internal.h"),
+    "c0": ("qe_fused.cu", "qe_device.cuh", "qe_fused_plan.h", "qe_internal.h"),
+    "c2": ("qe_fused.cu", "qe_device.cuh", "qe_fused_plan.h", "qe_internal.h"),
+    "c4": ("qe_grouped.cu", "qe_device.cuh", "qe_internal.h"),
 }
 
 
 def kernel_source_hash(workload="c1"):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "quantized_expert_matvec_b200", "csrc")
-    for f in KERNEL_SOURCES.get(workload, ("qe_fused.cu", "qe_device.cuh")):
+    for f in KERNEL_SOURCES.get(workload, KERNEL_SOURCES["c1"]):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 

@@ -41,8 +41,8 @@ def test_committed_traffic_records_are_well_formed():
 def test_kernel_source_hash_follows_the_sources(tmp_path, monkeypatch):
     csrc = tmp_path / "quantized_expert_matvec_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "qe_fused.cu").write_text("a")
-    (csrc / "qe_device.cuh").write_text("b")
+    for i, f in enumerate(bench.KERNEL_SOURCES["c1"]):
+        (csrc / f).write_text(str(i))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     h1 = bench.kernel_source_hash("c1")
     (csrc / "qe_device.cuh").write_text("c")
