@@ -163,6 +163,11 @@ QE_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"
 QE_DEV void cp_async_mbar_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+// The same arrival counted against the barrier's expected count (its init
+// count must include it).
+QE_DEV void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 template <int N>
 QE_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 // Programmatic dependent launch: wait until the kernels this one depends on

@@ -66,6 +66,9 @@ struct FusedMisc {
   qe_expert ex[kMaxK];    // descriptors of the selected experts
   ExpertAddr ea[kMaxK];   // the same descriptors as addresses (copy plan)
   unsigned long long selkey[kMaxK];  // keys of the selected experts, in rank order
+  // expert k's index and descriptor are in (ex[k] landed by cp.async):
+  // count 2, the selecting lane's cp.async arrival and its own arrival
+  uint64_t dbar[kMaxK];
   unsigned amax_bits;  // max |xn| (float bits)
   double redd[kWarps];
   double rpart[kRouterRows][kWarps];
@@ -462,6 +465,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
     misc->abort = 0;
     misc->amax_bits = 0u;
     for (int b = 0; b < g.nbar; ++b) mbar_init(&bars[b], 1);
+    for (int k = 0; k < K; ++k) mbar_init(&misc->dbar[k], 2);
     fence_mbar_init();
   }
   if (tid < kMaxK) misc->gu_cnt[tid] = 0;
@@ -483,7 +487,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   // from its lanes' checks, the others from the abort flag it sets before
   // the hand-off barrier.
   bool issued = false;
-  unsigned tag = 0;  // this launch's record tag (compute warps)
+  unsigned tag = 0;    // this launch's record tag (compute warps)
+  unsigned armed = 0;  // copy warp: bit k, expert k's copies were issued
   if (warp < kWarps) {
     // ------------------------------------------------------------- routing
     // The router dot s_e = sum_c W[e,c] x_c gamma_c does not depend on the
@@ -623,13 +628,33 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
     }
     named_barrier(kBarCompute, kComputeThreads);
     if (warp == 0 && !*abort_flag) {
+      // the compute warps need only xn's exponent to start: hand off now;
+      // each expert's descriptor follows through its dbar mbarrier
+      if (lane == 0) {
+        misc->Ex = fixed_scale_exponent(__uint_as_float(misc->amax_bits));
+        misc->xK = pow2f(misc->Ex - 22);
+      }
+      __syncwarp();
+      named_barrier_arrive(kBarHandoff, kFusedThreads);
+      issued = true;
+      // expert k is decided: record it, fetch its descriptor into ex[k]
+      // (cp.async), arrive twice on dbar[k]
+      auto publish = [&](int k, int e) {
+        misc->idx[k] = e;
+        if (e >= 0 && e < E) {
+          const unsigned char* src = (const unsigned char*)(p.experts + e);
+          unsigned char* dst = (unsigned char*)&misc->ex[k];
+#pragma unroll
+          for (int q = 0; q < (int)sizeof(qe_expert); q += 8) cp_async8(dst + q, src + q);
+        }
+        cp_async_mbar_arrive_noinc(&misc->dbar[k]);
+        mbar_arrive(&misc->dbar[k]);
+      };
       if (given) {
         // routing decided beforehand: take its experts and weights as they are
         if (lane < K) {
-          const int e = p.given_idx[lane];
-          misc->idx[lane] = e;
           misc->wk[lane] = p.given_w[lane];
-          if (e >= 0 && e < E) misc->ex[lane] = p.experts[e];
+          publish(lane, p.given_idx[lane]);
         }
       } else {
         if (lane == 0) QE_TRACE(kTrPolledAll);
@@ -638,58 +663,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
         TopKCand c = lane < kWarps ? cl[0] : TopKCand{0ull, 0xffffffffu, 0u};
         for (int k = 0; k < K; ++k) {
           if (lane_wins_argmax(c.key, c.idx)) {
-            misc->idx[k] = (int)c.idx;
             misc->selkey[k] = c.key;
-            if ((int)c.idx < E) {  // the descriptor, 8 bytes at a time
-              const unsigned char* src = (const unsigned char*)(p.experts + c.idx);
-              unsigned char* dst = (unsigned char*)&misc->ex[k];
-#pragma unroll
-              for (int q = 0; q < (int)sizeof(qe_expert); q += 8) cp_async8(dst + q, src + q);
-            }
+            publish(k, (int)c.idx);
             ++h;
             c = h < K ? cl[h] : TopKCand{0ull, 0xffffffffu, 0u};
           }
         }
-        cp_async_wait_all();
         if (lane == 0) QE_TRACE(kTrRounds);
-      }
-      __syncwarp();
-      // the selected experts' descriptors, checked, and what the copies and
-      // the dequant cores need of them
-      bool ok = true;
-      qe_expert ex{};
-      if (lane < K) {
-        const int e = misc->idx[lane];
-        ok = e >= 0 && e < E;
-        if (ok) {
-          ex = misc->ex[lane];
-          ok = expert_ok(ex);
-        }
-        if (!ok) {
-          set_error(&ctl->err, QE_ERR_INVALID_ARG);
-          misc->abort = 1;
-        }
-        const ExpertAddr a = expert_addr(ex);
-        misc->ea[lane] = a;
-        misc->mis_gu[lane][0] = run_misalign(a.gs, t.r_lo, H / 32);
-        misc->mis_gu[lane][1] = run_misalign(a.gb, t.r_lo, H / 32);
-        misc->mis_gu[lane][2] = run_misalign(a.us, t.r_lo, H / 32);
-        misc->mis_gu[lane][3] = run_misalign(a.ub, t.r_lo, H / 32);
-        misc->mis_d[lane][0] = run_misalign(a.ds, t.o_lo, I / 32);
-        misc->mis_d[lane][1] = run_misalign(a.db, t.o_lo, I / 32);
-      }
-      if (lane == 0) {
-        misc->Ex = fixed_scale_exponent(__uint_as_float(misc->amax_bits));
-        misc->xK = pow2f(misc->Ex - 22);
-      }
-      // the descriptors are out: the copy warp issues every copy of the CTA,
-      // the compute warps go on to their gate/up work (and wait for its data
-      // on the mbarriers)
-      const bool all_ok = __all_sync(0xffffffffu, ok);
-      if (lane == 0) QE_TRACE(kTrTopK);
-      named_barrier_arrive(kBarHandoff, kFusedThreads);
-      issued = all_ok;
-      if (!given) {
+        __syncwarp();
         // renormalised softmax over the K kept logits (sum in k order); the
         // weights are needed at the combine only
         const double lmax = dkey_inv(misc->selkey[0]);
@@ -698,6 +679,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
         for (int k = 0; k < K; ++k) sum += __shfl_sync(0xffffffffu, ev, k);
         if (lane < K) misc->wk[lane] = ev / sum;
       }
+      __syncwarp();
       if (cta == 0 && lane < K) {
         if (p.topk_idx) p.topk_idx[lane] = misc->idx[lane];
         if (p.topk_w) p.topk_w[lane] = misc->wk[lane];
@@ -721,7 +703,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
         if (warp == 0 && lane == 0) QE_TRACE(kTrGateUp);
       }
       if (warp < K * (kWarps / K)) {  // every warp of an expert calls it (named barrier inside)
-        ok = misc->ex[warp / (kWarps / K)].down.bits == 4
+        // the expert's descriptor (a warp without gate/up rows has not
+        // waited for it yet)
+        const int kd = warp / (kWarps / K);
+        mbar_wait(&misc->dbar[kd], 0, deadline, abort_flag);
+        ok = misc->ex[kd].down.bits == 4
                  ? down_phase<4>(p, t, misc, bars, ycomb, smem, deadline, warp, lane, tag)
                  : down_phase<2>(p, t, misc, bars, ycomb, smem, deadline, warp, lane, tag);
         if (!ok && lane == 0 && !*abort_flag) {
@@ -749,24 +735,63 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
     named_barrier(kBarHandoff, kFusedThreads);
     issued = !*abort_flag;
     if (issued) {
-      // Expert by expert, its gate/up copies (lane u takes copy u: gate
-      // rows, up rows, the four scale/bias runs), then expert by expert its
-      // down copies: each expert's gate/up bytes are ahead of the next
+      // Expert by expert, as warp 0 decides them: wait for the descriptor,
+      // check it, write what the compute warps read of it, arm the expert's
+      // gate/up mbarrier and issue its gate/up copies (lane u takes copy u:
+      // gate rows, up rows, the four scale/bias runs).  Then the down copies
+      // of every expert.  Each expert's gate/up bytes are ahead of the next
       // expert's, and all of them ahead of the down rows.  A bulk copy's
       // issue waits while the SM's queue of copies is full, so this warp
       // keeps issuing for most of the stream; nothing else waits on it.
       const uint64_t pol = policy_evict_first();
       const int ng = gu_copies(t), nd = d_copies(t);
       for (int k = 0; k < K; ++k) {
-        if (lane == 0 && ng) mbar_arrive_expect_tx(&bars[bar_gu(k)], fused_bar_bytes(g, H, I, K, t, misc->ea, bar_gu(k)));
+        if (!__all_sync(0xffffffffu, mbar_wait(&misc->dbar[k], 0, deadline, abort_flag))) {
+          if (lane == 0) {
+            set_error(&ctl->err, QE_ERR_TIMEOUT);
+            __threadfence_block();
+            misc->abort = 1;
+          }
+          break;
+        }
+        const int e = misc->idx[k];
+        qe_expert ex{};
+        bool ok = e >= 0 && e < E;
+        if (ok) {
+          ex = misc->ex[k];
+          ok = expert_ok(ex);
+        }
+        if (!ok) {  // the same decision in every lane
+          if (lane == 0) {
+            set_error(&ctl->err, QE_ERR_INVALID_ARG);
+            __threadfence_block();  // the error word before the flag others act on
+            misc->abort = 1;
+          }
+          break;
+        }
+        const ExpertAddr ak = expert_addr(ex);
+        if (lane == 0) {
+          misc->ea[k] = ak;
+          misc->mis_gu[k][0] = run_misalign(ak.gs, t.r_lo, H / 32);
+          misc->mis_gu[k][1] = run_misalign(ak.gb, t.r_lo, H / 32);
+          misc->mis_gu[k][2] = run_misalign(ak.us, t.r_lo, H / 32);
+          misc->mis_gu[k][3] = run_misalign(ak.ub, t.r_lo, H / 32);
+          misc->mis_d[k][0] = run_misalign(ak.ds, t.o_lo, I / 32);
+          misc->mis_d[k][1] = run_misalign(ak.db, t.o_lo, I / 32);
+          // releases the writes above to the warps that wait on the barrier
+          if (ng) mbar_arrive_expect_tx(&bars[bar_gu(k)], fused_bar_bytes(g, H, I, K, t, misc->ea, bar_gu(k)));
+        }
         __syncwarp();
         if (lane < ng) {
-          const FusedCopy c = fused_expert_copy(g, H, I, K, t, k, misc->ea[k], lane);
+          const FusedCopy c = fused_expert_copy(g, H, I, K, t, k, ak, lane);
           bulk_g2s(smem + c.dst, (const void*)(uintptr_t)c.src, c.bytes, &bars[c.bar], pol);
         }
+        armed |= 1u << k;
+        if (k == 0 && lane == 0) QE_TRACE(kTrTopK);
       }
-      for (int k = 0; k < K; ++k) {
-        if (lane == 0 && nd)
+      for (int k = 0; k < K && nd; ++k) {
+        if (!(armed >> k & 1u)) break;
+        if (lane == 0)
           mbar_arrive_expect_tx(&bars[bar_down(K, k)], fused_bar_bytes(g, H, I, K, t, misc->ea, bar_down(K, k)));
         __syncwarp();
         if (lane < nd) {
@@ -804,9 +829,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1) qe_fused_layer_kernel(const 
   if (warp == kWarps && issued) {
     volatile int no_abort = 0;
     const uint64_t dl2 = gtimer() + p.budget_ns;
-    for (int b = lane; b < g.nbar; b += 32)
-      if (fused_bar_bytes(g, H, I, K, t, misc->ea, b)) mbar_wait(&bars[b], 0, dl2, &no_abort);
+    for (int b = lane; b < g.nbar; b += 32) {
+      const int k = b < K ? b : b - K;
+      if ((armed >> k & 1u) && fused_bar_bytes(g, H, I, K, t, misc->ea, b)) mbar_wait(&bars[b], 0, dl2, &no_abort);
+    }
   }
+  // the descriptor copies warp 0 started (normally long landed)
+  if (warp == 0) cp_async_wait_all();
   if (warp == kWarps && lane == 0) QE_TRACE(kTrBarsDone);
   __syncthreads();
   if (tid == 0) {
