@@ -10,7 +10,9 @@ order); this module only marshals numpy arrays and sequences the steps of one
 layer as the Flash-MoE pages order them (lilting.ch article on Flash-MoE,
 sections "Model architecture" and "Metal Compute Shaders"): RMSNorm, router,
 softmax + top-K, per-expert gate/up dequant-matvec, SwiGLU, down
-dequant-matvec, weighted combine.
+dequant-matvec, weighted combine.  ``gdn_step`` is the GatedDeltaNet decode
+step of the same model (lilting.ch article, section "GatedDeltaNet
+acceleration"), stated in ``oracle.c``.
 """
 from __future__ import annotations
 
@@ -76,6 +78,8 @@ def _L():
         lib.or_expert_ffn.restype = None
         lib.or_expert_ffn.argtypes = [ctypes.POINTER(_QMat)] * 3 + [ctypes.c_int, ctypes.c_int, _D, _D, _D,
                                                                     ctypes.c_int]
+        lib.or_gdn_step.restype = None
+        lib.or_gdn_step.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _D, _D, _D, _D, _D, _D, _D]
         lib.or_combine.restype = None
         lib.or_combine.argtypes = [_D, _D, ctypes.c_int, ctypes.c_int, _D, _D]
         _lib = lib
@@ -220,3 +224,17 @@ def layer_step(x, router_w, experts, bits_of, K: int, eps: float = 1e-6, gamma=N
     y = np.stack([expert_ffn(experts(int(e)), bits_of(int(e)), xn, nthreads) for e in idx])
     out = combine(y, w, x if residual else None)
     return {"xn": xn, "logits": logits, "idx": idx, "w": w, "y": y, "out": out}
+
+
+def gdn_step(S, q, k, v, alpha, beta):
+    """One gated-delta-rule decode step (scal, gemv, ger, gemv per head).
+
+    S [n_heads, dv, dk], q and k [n_heads, dk], v [n_heads, dv], alpha and
+    beta [n_heads].  Returns (S', o) as new float64 arrays; S is not changed."""
+    S2 = np.array(S, dtype=np.float64, copy=True, order="C")
+    nh, dv, dk = S2.shape
+    q, k, v = _f64(q).reshape(nh, dk), _f64(k).reshape(nh, dk), _f64(v).reshape(nh, dv)
+    a, b = _f64(alpha).reshape(nh), _f64(beta).reshape(nh)
+    o = np.empty((nh, dv), np.float64)
+    _L().or_gdn_step(nh, dk, dv, _d(S2), _d(q), _d(k), _d(v), _d(a), _d(b), _d(o))
+    return S2, o

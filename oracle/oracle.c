@@ -1,6 +1,8 @@
 /*
  * oracle.c -- TEST INFRASTRUCTURE.  A plain, slow, fp64 CPU statement of the
- * MoE expert step of Flash-MoE decode, used only to check the CUDA library.
+ * MoE expert step of Flash-MoE decode, and of the GatedDeltaNet decode step
+ * that precedes it in 45 of the model's 60 layers, used only to check the
+ * CUDA library.
  * Only the tests, the smoke check and the CPU-baseline leg of the benchmark
  * may load it; the product path never does.  It shares no code, header,
  * table or helper with the CUDA library.
@@ -21,6 +23,11 @@
  *          (nibble*scale + bias)*x  ->  fma(nibble, scale*x, bias*x).
  *  [QUANT] tomo3141592653.github.io summary, section "Hybrid quantisation":
  *          MLX 4-bit quantisation of the experts.
+ *  [GDN]   lilting.ch, same article, section "GatedDeltaNet acceleration":
+ *          per layer a recurrent update of 64 heads x 128x128 state
+ *          matrices, done with the BLAS calls scal, gemv and ger; and the
+ *          tomo3141592653.github.io summary, section "GatedDeltaNet": a fixed,
+ *          O(1) state in place of a KV cache.
  *
  * Readings where the pages are silent (each is a convention of the problem
  * statement this library implements; the pins in tests/ hold them):
@@ -191,4 +198,43 @@ void or_combine(const double* y, const double* w, int K, int H, const double* re
     for (int k = 0; k < K; ++k) acc += w[k] * y[(size_t)k * H + r];
     out[r] = acc + (residual ? residual[r] : 0.0);
   }
+}
+
+/* One decode step of the gated delta rule for n_heads independent heads
+ * [GDN].  The pages name the recurrence and its three BLAS calls but print
+ * no formula; the reading taken here is the gated delta rule
+ *   S' = alpha S (I - beta k k^T) + beta v k^T,   o = S' q,
+ * carried out as the BLAS sequence the pages name, in this order:
+ *   scal  S <- alpha S
+ *   gemv  u <- S k                    (what the decayed state recalls for k)
+ *   ger   S <- S + beta (v - u) k^T   (write the correction at key k)
+ *   gemv  o <- S q                    (read out with the query)
+ * S is [n_heads][dv][dk] row-major (row i answers value component i), q and
+ * k are [n_heads][dk], v and o are [n_heads][dv], alpha and beta one value per
+ * head.  S is updated in place. */
+void or_gdn_step(int n_heads, int dk, int dv, double* S, const double* q, const double* k,
+                 const double* v, const double* alpha, const double* beta, double* o) {
+  double* u = (double*)malloc(sizeof(double) * (size_t)(dv > 0 ? dv : 1));
+  for (int h = 0; h < n_heads; ++h) {
+    double* Sh = S + (size_t)h * dv * dk;
+    const double* qh = q + (size_t)h * dk;
+    const double* kh = k + (size_t)h * dk;
+    const double* vh = v + (size_t)h * dv;
+    for (size_t e = 0; e < (size_t)dv * dk; ++e) Sh[e] *= alpha[h];
+    for (int i = 0; i < dv; ++i) {
+      double acc = 0.0;
+      for (int j = 0; j < dk; ++j) acc += Sh[(size_t)i * dk + j] * kh[j];
+      u[i] = acc;
+    }
+    for (int i = 0; i < dv; ++i) {
+      const double c = beta[h] * (vh[i] - u[i]);
+      for (int j = 0; j < dk; ++j) Sh[(size_t)i * dk + j] += c * kh[j];
+    }
+    for (int i = 0; i < dv; ++i) {
+      double acc = 0.0;
+      for (int j = 0; j < dk; ++j) acc += Sh[(size_t)i * dk + j] * qh[j];
+      o[(size_t)h * dv + i] = acc;
+    }
+  }
+  free(u);
 }

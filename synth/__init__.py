@@ -12,7 +12,11 @@ Value distributions follow the workload shapes of the Flash-MoE pages
   field is U{0..15} (U{0..3});
 * scales: bf16(U(0.005, 0.02)); biases: bf16(N(0, 0.01));
 * x: N(0, 1) fp32 (bf16 for the batched workload); router W: N(0, 0.02) fp32;
-* Zipf(s=1.1) expert popularity enters the router as a per-layer logit offset.
+* Zipf(s=1.1) expert popularity enters the router as a per-layer logit offset;
+* GatedDeltaNet decode step (64 heads x 128x128 state per layer): state
+  N(0, 0.1) fp32, q and k uniform on the unit sphere (normalised N(0,1) draws,
+  rounded to fp32), v N(0, 1) fp32, decay alpha bf16(U(0.9, 1)) and write
+  strength beta bf16(U(0, 1)), both as fp32.
 
 Host fills (numpy) come from ``libsynth_host.so`` and device fills (torch
 CUDA tensors) from ``libsynth_dev.so``; both evaluate the same counter-based
@@ -35,6 +39,7 @@ T_GATE_WQ, T_GATE_S, T_GATE_B = 1, 2, 3
 T_UP_WQ, T_UP_S, T_UP_B = 4, 5, 6
 T_DOWN_WQ, T_DOWN_S, T_DOWN_B = 7, 8, 9
 T_ROUTER, T_X, T_PERM = 10, 11, 12
+T_GDN_S, T_GDN_Q, T_GDN_K, T_GDN_V, T_GDN_ALPHA, T_GDN_BETA = 13, 14, 15, 16, 17, 18
 
 # value kinds
 K_U32, K_BF16_UNIFORM, K_BF16_NORMAL, K_F32_NORMAL = 0, 1, 2, 3
@@ -228,3 +233,36 @@ def zipf_logit_offset(seed: int, layer: int, n_experts: int, s: float = 1.1,
 def hot_set(seed: int, layer: int, n_experts: int, n_hot: int) -> np.ndarray:
     """Boolean mask of the n_hot most popular experts of a layer (ranks < n_hot)."""
     return expert_permutation(seed, layer, n_experts) < n_hot
+
+
+GDN_STATE_STD = 0.1
+GDN_ALPHA_LO, GDN_ALPHA_HI = 0.9, 1.0
+
+
+def _unit_rows(z: np.ndarray) -> np.ndarray:
+    """Rows of z scaled to unit length in float64, then rounded to fp32 (a
+    sample from the uniform distribution on the sphere)."""
+    z = z.astype(np.float64)
+    n = np.sqrt((z * z).sum(axis=1, keepdims=True))
+    return (z / np.where(n > 0, n, 1.0)).astype(np.float32)
+
+
+def host_gdn_state(seed: int, layer: int, n_heads: int, dk: int, dv: int) -> np.ndarray:
+    """Initial recurrent state S fp32 [n_heads, dv, dk] ~ N(0, 0.1)."""
+    return host_fill(n_heads * dv * dk, K_F32_NORMAL, seed, layer, 0, T_GDN_S,
+                     GDN_STATE_STD).reshape(n_heads, dv, dk)
+
+
+def host_gdn_token(seed: int, layer: int, t: int, n_heads: int, dk: int, dv: int) -> dict:
+    """Inputs of one decode step of one layer: q, k [n_heads, dk] unit rows,
+    v [n_heads, dv] ~ N(0,1), alpha, beta [n_heads] (fp32)."""
+    def bf16_uniform(tensor, lo, hi):
+        b = host_fill(n_heads, K_BF16_UNIFORM, seed, layer, t, tensor, lo, hi)
+        return (b.astype(np.uint32) << 16).view(np.float32).copy()
+    return {
+        "q": _unit_rows(host_fill(n_heads * dk, K_F32_NORMAL, seed, layer, t, T_GDN_Q, 1.0).reshape(n_heads, dk)),
+        "k": _unit_rows(host_fill(n_heads * dk, K_F32_NORMAL, seed, layer, t, T_GDN_K, 1.0).reshape(n_heads, dk)),
+        "v": host_fill(n_heads * dv, K_F32_NORMAL, seed, layer, t, T_GDN_V, 1.0).reshape(n_heads, dv),
+        "alpha": bf16_uniform(T_GDN_ALPHA, GDN_ALPHA_LO, GDN_ALPHA_HI),
+        "beta": bf16_uniform(T_GDN_BETA, 0.0, 1.0),
+    }

@@ -37,7 +37,10 @@ enum {
   SY_T_GATE_WQ = 1, SY_T_GATE_S = 2, SY_T_GATE_B = 3,
   SY_T_UP_WQ = 4,   SY_T_UP_S = 5,   SY_T_UP_B = 6,
   SY_T_DOWN_WQ = 7, SY_T_DOWN_S = 8, SY_T_DOWN_B = 9,
-  SY_T_ROUTER = 10, SY_T_X = 11,     SY_T_PERM = 12
+  SY_T_ROUTER = 10, SY_T_X = 11,     SY_T_PERM = 12,
+  /* GatedDeltaNet decode step: state, query, key, value, decay, write strength */
+  SY_T_GDN_S = 13, SY_T_GDN_Q = 14, SY_T_GDN_K = 15, SY_T_GDN_V = 16,
+  SY_T_GDN_ALPHA = 17, SY_T_GDN_BETA = 18
 };
 
 /* Value kinds a fill can produce. */
