@@ -10,8 +10,10 @@ top-K, 4 expert FFNs, combine) = one launch of the fused kernel.  Tokens are
 distinct seeded N(0,1) vectors, so routing scatters over the 3.6 GB expert
 pool, far larger than L2.
 
-Other workloads (--workload): c0 tiny layer, c4 batched decode (256 tokens
-per step, grouped experts).  Prints one JSON line; ``--impl reference`` times
+Other workloads (--workload): c0 tiny layer, c2 40-layer stack, c3 tiered
+layers, c4 batched decode (256 tokens per step, grouped experts), gdn the
+GatedDeltaNet decode step of the same model (45 layers of 64 heads x 128x128
+recurrent state).  Prints one JSON line; ``--impl reference`` times
 the fp64 CPU oracle on the host cores instead.
 """
 from __future__ import annotations
@@ -56,6 +58,16 @@ WORKLOADS = {
                name="batched decode of the one-layer workload: 256 bf16 tokens per step, own top-4 of 512 each, "
                     "grouped per expert, 4-bit g64 experts in HBM, uniform routing",
                metric="MoE-layer batched decode tokens/s at 1 B200"),
+    "gdn": dict(heads=64, dk=128, dv=128, layers=45, T=1,
+                name="GatedDeltaNet decode: one token through the recurrent state of 45 linear-attention layers, "
+                     "64 heads x 128x128 fp32 state per layer (180 MiB of state in HBM, larger than L2), gated "
+                     "delta rule (scal, gemv, ger, gemv per head), batch 1 sequence",
+                metric="GatedDeltaNet decode tokens/s at 1 B200 (45 layers)"),
+    "gdn8": dict(heads=64, dk=128, dv=128, layers=45, T=8, seqs=8,
+                 name="GatedDeltaNet batched decode: one token of each of 8 sequences through the recurrent state "
+                      "of 45 linear-attention layers, 8 x 64 heads x 128x128 fp32 state per layer (1.4 GiB of "
+                      "state in HBM), gated delta rule, one launch per layer for all 8 sequences",
+                 metric="GatedDeltaNet batched decode tokens/s at 1 B200 (45 layers, 8 sequences)"),
 }
 
 UNIT = "tokens/s"
@@ -72,6 +84,8 @@ KERNEL_SOURCES = {  # the sources the dominant kernel of each workload is compil
     "c0": ("qe_fused.cu", "qe_device.cuh", "qe_fused_plan.h", "qe_internal.h"),
     "c2": ("qe_fused.cu", "qe_device.cuh", "qe_fused_plan.h", "qe_internal.h"),
     "c4": ("qe_grouped.cu", "qe_device.cuh", "qe_internal.h"),
+    "gdn": ("qe_gdn.cu", "qe_device.cuh", "qe_internal.h"),
+    "gdn8": ("qe_gdn.cu", "qe_device.cuh", "qe_internal.h"),
 }
 
 
@@ -266,6 +280,9 @@ def run_reference(args, wl, rank, world):
     timed steps take about 150 s."""
     if rank != 0:
         return
+    if "heads" in wl:
+        run_reference_gdn(args, wl)
+        return
     K, W, T = args.steps, args.warmup, wl["T"]
     per_step_units = T * wl_layers(wl)   # layer steps in one step
     probe = OracleSample(wl, args.seed, 1.0, n_pool=1)
@@ -297,6 +314,70 @@ def run_reference(args, wl, rank, world):
                              "sample": f"each step: {t_timed} of its {per_step_units} layer step(s) timed, "
                                        f"routing in full, expert rows sampled at fraction {frac:.4f} and "
                                        f"extrapolated; {wall:.1f} s wall for the timed steps"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+class GdnOracleSample:
+    """The oracle's GatedDeltaNet step on a few layers of the workload: fp64
+    state per layer, a pool of seeded tokens, one whole layer step per call."""
+
+    def __init__(self, wl, seed, n_layers=2, n_tok=4):
+        import oracle
+        import synth
+        self.oracle = oracle
+        nh, dk, dv = wl["heads"], wl["dk"], wl["dv"]
+        self.S = [synth.host_gdn_state(seed, l, nh, dk, dv).astype(np.float64) for l in range(n_layers)]
+        self.toks = [[synth.host_gdn_token(seed, l, t, nh, dk, dv) for t in range(n_tok)] for l in range(n_layers)]
+        self.i = 0
+
+    def layer_step_seconds(self):
+        l = self.i % len(self.S)
+        tok = self.toks[l][(self.i // len(self.S)) % len(self.toks[l])]
+        self.i += 1
+        t0 = time.perf_counter()
+        self.S[l], _ = self.oracle.gdn_step(self.S[l], tok["q"], tok["k"], tok["v"], tok["alpha"], tok["beta"])
+        return time.perf_counter() - t0
+
+
+def gdn_cpu_baseline(wl, seed, budget_s=10.0):
+    smp = GdnOracleSample(wl, seed)
+    per = smp.layer_step_seconds()
+    n = max(2, min(4000, int(budget_s / max(per, 1e-9))))
+    t0 = time.perf_counter()
+    tot = sum(smp.layer_step_seconds() for _ in range(n))
+    spent = time.perf_counter() - t0
+    per_token = tot / n * wl["layers"]      # one sequence's token; the oracle step is per sequence
+    return {"value": 1.0 / per_token, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} whole layer steps (64 heads x 128x128, fp64 oracle, one thread) over 2 layers' "
+                      f"states and 4 tokens each, scaled to {wl['layers']} layers per token; {spent:.1f} s"}
+
+
+def run_reference_gdn(args, wl):
+    """Reference arm of the GatedDeltaNet workload: the oracle's step, at
+    most 4 layer steps timed per step and scaled to the 45 layers."""
+    K, W = args.steps, args.warmup
+    smp = GdnOracleSample(wl, args.seed)
+    per = min(smp.layer_step_seconds() for _ in range(2))
+    t_timed = max(1, min(4, int((150.0 / (K + W)) / max(per, 1e-9))))
+    for _ in range(W * t_timed):
+        smp.layer_step_seconds()
+    t0 = time.perf_counter()
+    total = 0.0
+    seqs = wl.get("seqs", 1)
+    for _ in range(K):
+        # a step: every sequence's token through every layer (the oracle
+        # takes one sequence's layer step at a time)
+        total += sum(smp.layer_step_seconds() for _ in range(t_timed)) * (wl["layers"] * seqs / t_timed)
+    wall = time.perf_counter() - t0
+    value = K * seqs / total
+    line = {"metric": wl["metric"], "value": value, "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": W,
+            "ms_per_step": 1000.0 * total / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl["name"], "tokens_per_step": seqs, "layers": wl["layers"]},
+            "cpu_baseline": {"kind": "oracle", "cores": 1, "value": value, "unit": UNIT,
+                             "sample": f"each step: {t_timed} of its {wl['layers'] * seqs} layer steps timed (fp64 "
+                                       f"oracle, one thread), scaled; {wall:.2f} s wall for the timed steps"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -679,6 +760,137 @@ def mem_available():
     return 0
 
 
+def run_gdn(args, wl, rank, world, local_rank):
+    """One step = one token through the GatedDeltaNet recurrence of every
+    layer: one gdn_decode_step launch per layer on that layer's resident
+    state.  CUDA graphs of 32 tokens; the launches overlap their neighbours'
+    tails through programmatic dependent launch."""
+    import torch
+    import quantized_expert_matvec_b200 as q
+    import synth
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    seqs = wl.get("seqs", 1)
+    nh, dk, dv, L = wl["heads"] * seqs, wl["dk"], wl["dv"], wl["layers"]
+    S = torch.empty((L, nh, dv, dk), dtype=torch.float32, device=dev)
+    for l in range(L):
+        S[l].copy_(torch.from_numpy(synth.host_gdn_state(args.seed, l, nh, dk, dv)))
+    # per (token, layer) one flat fp32 record: q [nh,dk], k [nh,dk], v [nh,dv], alpha [nh], beta [nh]
+    oq, ok_, ov, oa, ob = 0, nh * dk, 2 * nh * dk, 2 * nh * dk + nh * dv, 2 * nh * dk + nh * dv + nh
+    rec = ob + nh
+    chunk = 32 if seqs == 1 else 8
+    tok0 = rank_token_base(20_000_000, rank)
+    host_in = np.empty((chunk, L, rec), np.float32)
+    for t in range(chunk):
+        for l in range(L):
+            d = synth.host_gdn_token(args.seed, l, tok0 + t, nh, dk, dv)
+            host_in[t, l, oq:ok_] = d["q"].ravel()
+            host_in[t, l, ok_:ov] = d["k"].ravel()
+            host_in[t, l, ov:oa] = d["v"].ravel()
+            host_in[t, l, oa:ob] = d["alpha"]
+            host_in[t, l, ob:] = d["beta"]
+    inp = torch.from_numpy(host_in).to(dev)
+    out = torch.empty((chunk, L, nh, dv), dtype=torch.float32, device=dev)
+    s = torch.cuda.Stream(device=dev)
+
+    def token(t, src, dst):
+        for l in range(L):
+            r = src[t, l]
+            q.gdn_decode_step(S[l], r[oq:ok_], r[ok_:ov], r[ov:oa], r[oa:ob], r[ob:], dst[t, l], stream=s)
+
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        token(0, inp, out)
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for t in range(chunk):
+                token(t, inp, out)
+    torch.cuda.synchronize()
+    reps = max(1, args.steps // chunk)
+    args.steps = reps * chunk
+    with torch.cuda.stream(s):
+        for _ in range(max(1, -(-args.warmup // chunk))):
+            g.replay()
+    s.synchronize()
+    barrier(world)
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        ev0.record(s)
+        for _ in range(reps):
+            g.replay()
+        ev1.record(s)
+    s.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    ms = ev0.elapsed_time(ev1)
+    ms_max = sync_max(world, dev, ms)
+    if not bool(torch.isfinite(S).all().item()):
+        raise RuntimeError("non-finite recurrent state after timing")
+    del g
+
+    # e2e: per token, the layers' inputs copied from pinned host memory, the
+    # 45 launches, the read-outs copied back, one synchronisation
+    n_e2e = min(args.steps, 256 if seqs == 1 else 64)
+    pin_in = torch.from_numpy(host_in).pin_memory()
+    pin_out = torch.empty((1, L, nh, dv), dtype=torch.float32).pin_memory()
+    stage_in = torch.empty((1, L, rec), dtype=torch.float32, device=dev)
+    stage_out = torch.empty((1, L, nh, dv), dtype=torch.float32, device=dev)
+
+    def e2e_token(i):
+        with torch.cuda.stream(s):
+            stage_in.copy_(pin_in[i % chunk:i % chunk + 1], non_blocking=True)
+            token(0, stage_in, stage_out)
+            pin_out.copy_(stage_out, non_blocking=True)
+        s.synchronize()
+
+    for i in range(4):
+        e2e_token(i)
+    barrier(world)
+    t0 = time.perf_counter()
+    for i in range(n_e2e):
+        e2e_token(i)
+    e2e_s = sync_max(world, dev, time.perf_counter() - t0)
+    if rank != 0:
+        return
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks["hbm_gbs"])
+    per_launch_s = (ms / 1000.0) / (args.steps * L)
+    alg = 2 * nh * dv * dk * 4 + rec * 4 + nh * dv * 4
+    achieved = alg / per_launch_s / 1e9
+    cpu = None if args.no_cpu_baseline else gdn_cpu_baseline(wl, args.seed)
+    line = {
+        "metric": wl["metric"], "value": world * args.steps * seqs / (ms_max / 1000.0), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl["name"], "tokens_per_step": seqs, "sequences": seqs, "layers": L,
+                   "distinct_token_inputs": chunk,
+                   "l2": f"inputs larger than L2: {S.numel() * 4 / 2**20:.0f} MiB of recurrent state plus "
+                         f"{inp.numel() * 4 / 1e6:.0f} MB of token inputs",
+                   "launch": f"CUDA graphs of {chunk} tokens x {L} launches, programmatic dependent launch",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": load_traffic(args.workload), "peak_source": peak_kind,
+                     "kernel": "qe_gdn_step_kernel", "algorithmic_bytes_per_launch": alg,
+                     "duration": f"whole step / {L} launches (gaps between launches included)",
+                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                     "frac_basis": "frac: of the measured copy peak; frac_of_nominal_8tbs: of B200's nominal 8 TB/s"},
+        "us_per_layer_step": 1e6 * per_launch_s,
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * n_e2e * seqs / e2e_s, "unit": UNIT, "h2d_bytes_per_step": L * rec * 4,
+                "d2h_bytes_per_step": L * nh * dv * 4, "steps": n_e2e,
+                "how": f"per token: pinned H2D of the {L} layers' q, k, v, alpha, beta; {L} gdn_decode_step "
+                       f"calls; D2H of the read-outs; stream sync"},
+        "gpu_launches": args.steps * L,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_tiered(args, wl, rank, world, local_rank):
     """One step = one token through all tiered layers: per layer routing, one
     host synchronisation, cache resolve (misses copied host->device on the
@@ -831,7 +1043,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
-    defaults = {"c2": (1024, 32), "c3": (224, 32)}
+    defaults = {"c2": (1024, 32), "c3": (224, 32), "gdn": (4096, 32), "gdn8": (1024, 8)}
     if args.steps is None:
         args.steps = defaults.get(args.workload, (32768 if wl["T"] == 1 else 64, 0))[0]
     if args.warmup is None:
@@ -854,6 +1066,8 @@ def main():
             run_stack(args, wl, rank, world, local_rank)
         elif args.workload == "c3":
             run_tiered(args, wl, rank, world, local_rank)
+        elif args.workload in ("gdn", "gdn8"):
+            run_gdn(args, wl, rank, world, local_rank)
         else:
             run_ours(args, wl, rank, world, local_rank)
     finally:

@@ -366,6 +366,35 @@ QE_API int qe_fused_plan_probe(int H, int E, int K, int I, int sms, int smem_opt
  * reach keep their old value.  NULL disables tracing. */
 QE_API void qe_trace_fused(void* dev_buf);
 
+/* ---------------------------------------------------------------------
+ * GatedDeltaNet decode step (the linear-attention recurrence of 45 of the
+ * model's 60 layers): lilting.ch, "Flash-MoE: running a 397B-parameter model
+ * on a 48 GB MacBook", section "GatedDeltaNet acceleration" (64 heads x
+ * 128x128 state matrices updated per token with the BLAS calls scal, gemv
+ * and ger); tomo3141592653.github.io summary "Running a 400B-parameter LLM
+ * on iPhone 17 Pro", section "GatedDeltaNet" (a fixed O(1) state).  The pages
+ * print no formula; the recurrence is read as the gated delta rule, per head
+ *   S <- alpha S;  u = S k;  S <- S + beta (v - u) k^T;  o = S q,
+ * i.e. S' = alpha S (I - beta k k^T) + beta v k^T and o = S' q.
+ *
+ *   state  device fp32 [n_heads][dv][dk], row-major (row i is value
+ *          component i); updated in place.  16-byte aligned.
+ *   q, k   device fp32 [n_heads][dk]; 16-byte aligned.  (Unit-length keys
+ *          keep the recurrence non-expansive; nothing here requires it.)
+ *   v      device fp32 [n_heads][dv].
+ *   alpha, beta  device fp32 [n_heads]: decay and write strength per head.
+ *   out    device fp32 [n_heads][dv]: o of every head.  Must not overlap any
+ *          input.
+ * n_heads counts independent heads (a batch of sequences is n_seq * heads
+ * heads).  Shapes: n_heads >= 0 (0 launches nothing), dv >= 1, 4 <= dk <= 512,
+ * dk % 4 == 0; anything else returns QE_ERR_INVALID_ARG before any launch,
+ * as do NULL, misaligned or overlapping pointers.  Asynchronous on `stream`,
+ * one kernel launch, graph-capturable; the launch may overlap the tail of the
+ * previous kernel in the stream but reads nothing before that kernel has
+ * finished.  The arithmetic is fp32 (the pages use single-precision BLAS). */
+QE_API int gdn_decode_step(int n_heads, int dk, int dv, float* state, const float* q, const float* k,
+                           const float* v, const float* alpha, const float* beta, float* out, qe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

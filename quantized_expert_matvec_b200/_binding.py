@@ -29,6 +29,7 @@ __all__ = [
     "qe_workspace_init", "qe_workspace_status", "qe_set_wait_budget_ns", "qe_test_skip_arrival", "qe_trace_fused",
     "moe_route", "moe_expert_ffn_q4", "moe_expert_ffn_q2", "moe_expert_ffn_mixed", "moe_combine",
     "moe_layer_step", "moe_layer_step_noalloc", "moe_layer_step_host", "workspace", "Tier", "TierDesc",
+    "gdn_decode_step",
 ]
 
 
@@ -104,6 +105,7 @@ def _load():
         "qe_tier_stats": (i32, [vp, P(ctypes.c_uint64), P(ctypes.c_uint64), P(ctypes.c_uint64)]),
         "qe_tier_slots": (i32, [vp]),
         "qe_tier_destroy": (None, [vp]),
+        "gdn_decode_step": (i32, [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -349,3 +351,18 @@ class ExpertPool:
     def seg_ptr(self, seg: int, expert: int = 0) -> int:
         """Device address of segment `seg` (0..8, qe_pool_table order) of an expert."""
         return self.base + expert * self.stride + self.seg[seg]
+
+
+def gdn_decode_step(state, q, k, v, alpha, beta, out, stream=None):
+    """One GatedDeltaNet decode step for every head, in place on ``state``
+    (fp32 CUDA tensors: state [n_heads, dv, dk], q and k [n_heads, dk], v and
+    out [n_heads, dv], alpha and beta [n_heads])."""
+    if state.dim() != 3:
+        raise ValueError("state must be [n_heads, dv, dk]")
+    nh, dv, dk = (int(d) for d in state.shape)
+    for name, t, n in (("q", q, nh * dk), ("k", k, nh * dk), ("v", v, nh * dv), ("alpha", alpha, nh),
+                       ("beta", beta, nh), ("out", out, nh * dv)):
+        if t.numel() != n:
+            raise ValueError(f"{name} has {t.numel()} elements, expected {n}")
+    _check(lib.gdn_decode_step(nh, dk, dv, _ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                               _ptr(out), _stream(stream)))

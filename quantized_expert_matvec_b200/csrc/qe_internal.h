@@ -203,6 +203,11 @@ struct DevInfo {
   int sms = 0, optin = 0;
 };
 DevInfo dev_info();
+// GatedDeltaNet decode step (qe_gdn.cu): one launch over all heads.
+cudaError_t launch_gdn_step(long long n_heads, int dk, int dv, float* S, const float* q, const float* k,
+                            const float* v, const float* alpha, const float* beta, float* o, int sms,
+                            cudaStream_t s);
+
 int fail(int code, const char* fmt, ...);
 int cuda_fail(cudaError_t e, const char* what);
 int check_cfg(const qe_cfg* c);

@@ -140,3 +140,30 @@ def test_build_script_loads_without_the_library():
             "assert 'quantized_expert_matvec_b200' not in sys.modules, 'package imported'; print('ok')")
     r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
+
+
+@pytest.mark.parametrize("nh,dk,dv,what", [
+    (-1, 128, 128, "n_heads"), (4, 6, 8, "dk"), (4, 516, 8, "dk"), (4, 0, 8, "dk"), (4, 128, 0, "dv"),
+])
+def test_gdn_bad_shapes_rejected_before_launch(q, nh, dk, dv, what):
+    rc = q.lib.gdn_decode_step(nh, dk, dv, 1 << 20, 2 << 20, 3 << 20, 4 << 20, 5 << 20, 6 << 20, 7 << 20, None)
+    assert rc == q.QE_ERR_INVALID_ARG
+    assert "gdn_decode_step" in q.qe_last_error()
+
+
+def test_gdn_bad_pointers_rejected_before_launch(q):
+    L = q.lib
+    M = 1 << 20
+    # NULL, misaligned state / k (16 bytes needed), misaligned v (4 bytes)
+    assert L.gdn_decode_step(2, 128, 8, None, 2 * M, 3 * M, 4 * M, 5 * M, 6 * M, 7 * M, None) == q.QE_ERR_INVALID_ARG
+    assert L.gdn_decode_step(2, 128, 8, M + 8, 2 * M, 3 * M, 4 * M, 5 * M, 6 * M, 7 * M, None) == q.QE_ERR_INVALID_ARG
+    assert "16-byte" in q.qe_last_error()
+    assert L.gdn_decode_step(2, 128, 8, M, 2 * M, 3 * M + 4, 4 * M, 5 * M, 6 * M, 7 * M, None) == q.QE_ERR_INVALID_ARG
+    assert L.gdn_decode_step(2, 128, 8, M, 2 * M, 3 * M, 4 * M + 2, 5 * M, 6 * M, 7 * M, None) == q.QE_ERR_INVALID_ARG
+    assert "4-byte" in q.qe_last_error()
+    # out inside the state, and out overlapping v by one element
+    assert L.gdn_decode_step(2, 128, 8, M, 2 * M, 3 * M, 4 * M, 5 * M, 6 * M, M + 4096, None) == q.QE_ERR_INVALID_ARG
+    assert "overlaps" in q.qe_last_error()
+    assert L.gdn_decode_step(2, 128, 8, M, 2 * M, 3 * M, 4 * M + 60, 5 * M, 6 * M, 4 * M, None) == q.QE_ERR_INVALID_ARG
+    # no heads: nothing to do, no pointer looked at
+    assert L.gdn_decode_step(0, 128, 8, None, None, None, None, None, None, None, None) == q.QE_OK
