@@ -273,11 +273,15 @@ QE_API int moe_layer_step_noalloc(const qe_cfg* cfg, const qe_layer* layer, cons
  * from slow storage on demand through a cache; nzkcom.pages.dev
  * "flash-moe-romance-vs-utility", adopted optimisations: hot experts at 4
  * bits, cold experts at 2 bits).  Hot experts stay resident in HBM (the
- * caller's descriptors); cold experts live in pinned host memory and are
- * copied on demand into a pool of HBM slots with least-recently-used
- * replacement, on a side stream.  qe_tier_create is the one call of this
- * library that allocates device memory (the slot pool) and pinned host
- * memory (small staging arrays). */
+ * caller's descriptors); cold experts live in page-locked host memory mapped
+ * into the device's address space and are copied on demand into a pool of
+ * HBM slots with least-recently-used replacement.  The replacement state (the
+ * slot map, last-use stamps, counters) lives on the device and is updated by
+ * kernels in stream order, so no call waits for the host: a tiered layer step
+ * is a fixed sequence of kernel launches and can be captured in a CUDA graph.
+ * All calls on one tier must be ordered on the device (one stream, or
+ * streams ordered with events).  qe_tier_create is the one call of this
+ * library that allocates device memory (the slot pool and its state). */
 typedef struct qe_tier qe_tier;
 
 typedef struct {
@@ -288,47 +292,55 @@ typedef struct {
   int32_t reserved;
   /* HOST array [n_layers * n_experts]: for a cold expert (l, e), entry
    * l*E+e is the base of its qe_expert_bytes(cfg, cold_bits) bytes in the
-   * standard pool layout, in host memory (page-locked, so that the copies run
-   * asynchronously); NULL marks a hot expert.  The array is copied; the
+   * standard pool layout, in page-locked host memory that the device can
+   * read (cudaHostAlloc, or cudaHostRegister with cudaHostRegisterMapped),
+   * 16-byte aligned; NULL marks a hot expert.  The array is copied; the
    * memory it points to must outlive the tier. */
   const void* const* cold_host;
   size_t cache_bytes;  /* HBM for cold-expert slots: floor(cache_bytes / expert bytes) slots */
 } qe_tier_desc;
 
 /* Create a tier on the current device.  QE_ERR_OOM if the slot pool cannot
- * be allocated. */
+ * be allocated; QE_ERR_INVALID_ARG if a cold expert is not 16-byte aligned
+ * or not device-readable page-locked memory.  Synchronous. */
 QE_API int qe_tier_create(const qe_tier_desc* desc, qe_tier** out);
 
 /* Make the experts host_idx[0..n) (HOST array, indices into layer `layer`)
- * usable from dev_table (device, E descriptors of that layer): for each
- * distinct cold expert a hit reuses its slot, a miss evicts the least
- * recently used slot not needed by this call and copies the expert in on
- * the tier's side stream; `stream` waits for those copies, then the cold
- * experts' descriptors are written into dev_table on `stream`.  Hot entries
- * of dev_table are left as they are.  QE_ERR_OOM if one call needs more cold
- * experts than there are slots.  Calls on one tier are serialised. */
+ * usable from dev_table (device, E descriptors of that layer), on `stream`:
+ * for each distinct cold expert, in call order, a hit reuses its slot and a
+ * miss takes the least recently used slot not needed by this call; then the
+ * misses are copied in from host memory by a kernel and every cold expert's
+ * descriptor is written into dev_table.  Hot entries of dev_table are left
+ * as they are.  The indices are checked on the host first: QE_ERR_INVALID_ARG
+ * for one out of range, QE_ERR_OOM if the call needs more distinct cold
+ * experts than there are slots; a refused call changes nothing. */
 QE_API int qe_tier_resolve(qe_tier* t, int layer, const int32_t* host_idx, int n, qe_expert* dev_table,
                            qe_stream_t stream);
 
-/* The layer step with tiered experts: routing (as moe_route), then one host
- * synchronisation to read the K chosen experts per token, qe_tier_resolve on
- * layer->experts, then the expert FFNs and the combine (+ x if
- * add_residual) as moe_layer_step's batched path.  Arguments as
- * moe_layer_step; T <= max_tokens.  Synchronises the calling thread with
- * `stream` once. */
+/* The layer step with tiered experts, all on `stream` with no host
+ * synchronisation: routing (as moe_route), the resolve of the routed experts
+ * into layer->experts on the device (as qe_tier_resolve), the copy of the
+ * misses, then the expert FFNs and the combine (+ x if add_residual): the
+ * single-token kernel with this routing for T = 1, moe_layer_step's batched
+ * path otherwise.  Arguments as moe_layer_step; T <= max_tokens, and
+ * QE_ERR_OOM before any launch if T * top_k exceeds the number of slots (the
+ * routing, unknown to the host, could need that many cold experts). */
 QE_API int qe_tier_layer_step(qe_tier* t, int layer, const qe_layer* layer_w, const void* x, int x_dtype, int T,
                               float* out, int add_residual, int32_t* topk_idx, float* topk_w, void* dev_ws,
                               size_t ws_bytes, qe_stream_t stream);
 
 /* Counters since creation: distinct cold experts found in the cache (hits),
- * copied in (misses), and bytes copied host->device. */
+ * copied in (misses), and bytes copied host->device.  Synchronises the
+ * device first (the counters live there).  Returns the first error a resolve
+ * met on the device, if any (QE_ERR_INVALID_ARG for an index out of range,
+ * QE_ERR_OOM), after filling the counters. */
 QE_API int qe_tier_stats(const qe_tier* t, uint64_t* hits, uint64_t* misses, uint64_t* h2d_bytes);
 
 /* Number of HBM slots of the tier (0 for NULL). */
 QE_API int qe_tier_slots(const qe_tier* t);
 
-/* Wait for the tier's copies, then free everything it allocated.  NULL is a
- * no-op. */
+/* Synchronise the device, then free everything the tier allocated.  NULL is
+ * a no-op. */
 QE_API void qe_tier_destroy(qe_tier* t);
 
 /* Test hook: make CTA `cta` of the next fused single-token launches skip

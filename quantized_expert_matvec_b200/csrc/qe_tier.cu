@@ -1,6 +1,6 @@
 // qe_tier.cu -- two-tier expert residency: hot experts resident in HBM, cold
-// experts in pinned host memory behind an HBM cache of expert slots with LRU
-// replacement, misses copied host->device on a side stream.
+// experts in page-locked host memory behind an HBM cache of expert slots with
+// least-recently-used replacement.
 //
 // Follows the tiering of the Flash-MoE pages (lilting.ch "Flash-MoE: running
 // a 397B-parameter model on a 48 GB MacBook", sections "Core technique: SSD
@@ -9,59 +9,459 @@
 // adopted optimisations: frequently used experts kept at 4 bits, the rest
 // at 2 bits).  On B200 the storage tier is pinned host memory over PCIe and
 // the cache is a pool of HBM slots managed here instead of by an OS.
-#include <list>
+//
+// The cache's bookkeeping lives on the device, so that a layer whose experts
+// are all cached never waits for the host:
+//   - a slot map (cold expert -> slot or -1), per-slot last-use stamps and
+//     per-slot claim marks (the last call that claimed the slot), all in
+//     device memory;
+//   - tier_resolve_kernel (one CTA) replays the replacement policy in stream
+//     order: the call's distinct cold experts are found, hits claim their
+//     slots (stamped most recent), then each miss takes the unclaimed slot
+//     with the oldest stamp and queues a copy task; every cold expert's
+//     descriptor is written into the layer's table;
+//   - tier_fill_kernel copies the queued experts from host memory, which is
+//     mapped into the device's address space, into their slots.
+// A tiered layer step is therefore a fixed sequence of kernel launches
+// (routing, resolve, fill, experts; for one token the routing and the resolve
+// are one kernel, tier_route_kernel) and can be captured in a CUDA graph.
 #include <mutex>
 #include <vector>
 
+#include "qe_device.cuh"
 #include "qe_internal.h"
+
+namespace qe {
+
+struct TierState {                // device
+  unsigned call;                  // calls resolved so far; claim marks compare to it
+  int status;                     // first error found on the device (QE_OK if none)
+  unsigned long long clock;       // last stamp given to a slot
+  unsigned long long hits, misses, h2d_bytes;
+  int n_tasks;                    // copies queued by the last resolve
+  unsigned route_done;            // CTAs of the running routing launch that are done (0 between launches)
+};
+
+struct TierDev {                  // device pointers and constants, passed by value
+  TierState* st;
+  int32_t* key_slot;              // [L*E] slot of a cold expert, -1 if not cached
+  const unsigned long long* cold_src;  // [L*E] device-visible address of a cold expert, 0 if hot
+  int32_t* slot_key;              // [S] expert held by a slot, -1 if none
+  uint32_t* slot_call;            // [S] call that last claimed the slot
+  unsigned long long* slot_stamp; // [S] last use; unique, larger is more recent
+  unsigned long long* task_src;   // [max selections] source of a queued copy
+  int32_t* task_slot;             // [max selections] its slot
+  unsigned char* cache;           // S * slot_bytes
+  unsigned long long slot_bytes, expert_bytes;
+  int n_slots, E;
+  qe_expert tmpl;                 // descriptor of an expert stored at cache + 0
+};
+
+constexpr int kResolveThreads = 1024;
+constexpr int kFillThreads = 512;
+constexpr int kMaxTierSel = 4096;  // selections one call may resolve (max_tokens * top_k)
+
+__device__ __forceinline__ qe_expert slot_descriptor(const TierDev& d, int slot) {
+  qe_expert x = d.tmpl;
+  const size_t off = (size_t)slot * d.slot_bytes;
+  x.gate.wq = (const uint32_t*)((const char*)x.gate.wq + off);
+  x.gate.scales = (const uint16_t*)((const char*)x.gate.scales + off);
+  x.gate.biases = (const uint16_t*)((const char*)x.gate.biases + off);
+  x.up.wq = (const uint32_t*)((const char*)x.up.wq + off);
+  x.up.scales = (const uint16_t*)((const char*)x.up.scales + off);
+  x.up.biases = (const uint16_t*)((const char*)x.up.biases + off);
+  x.down.wq = (const uint32_t*)((const char*)x.down.wq + off);
+  x.down.scales = (const uint16_t*)((const char*)x.down.scales + off);
+  x.down.biases = (const uint16_t*)((const char*)x.down.biases + off);
+  return x;
+}
+
+// One CTA.  The call's selections are loaded in parallel into shared memory
+// (expert key, cold or not, slot at the start of the call) and deduplicated
+// there; thread 0 then replays the replacement policy over the distinct cold
+// experts in call order, reading shared memory only; the whole CTA searches
+// for each miss's victim; finally every first occurrence writes its
+// descriptor.  Every __syncthreads below is reached by all threads: the
+// branches around them test shared values written before the preceding
+// barrier.  n <= kMaxTierSel.
+// (A __device__ function so that the single-token routing kernel's last CTA
+// can run it too; called by all kResolveThreads threads of one CTA.)
+__device__ __noinline__ void tier_resolve_body(const TierDev& d, int layer, const int32_t* idx, int n,
+                                               qe_expert* table) {
+  __shared__ int s_key[kMaxTierSel];    // expert key of selection i
+  __shared__ int s_slot[kMaxTierSel];   // its slot: < 0 if not cached; -2 hot or duplicate
+  __shared__ unsigned s_call;
+  __shared__ int s_bad, s_kind, s_cur;
+  __shared__ unsigned long long s_best[kResolveThreads / 32];
+  __shared__ int s_besti[kResolveThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  TierState* st = d.st;
+  __syncthreads();  // the caller's shared memory may still be in use
+  if (tid == 0) {
+    s_call = st->call + 1u;  // 0 after 2^32 calls
+    s_bad = QE_OK;
+  }
+  __syncthreads();
+  for (int i = tid; i < n; i += blockDim.x) {
+    const int e = idx[i];
+    if (e < 0 || e >= d.E) {
+      s_key[i] = -1;
+      s_slot[i] = -2;
+      atomicCAS(&s_bad, QE_OK, QE_ERR_INVALID_ARG);
+      continue;
+    }
+    const int key = layer * d.E + e;
+    s_key[i] = key;
+    s_slot[i] = d.cold_src[key] ? d.key_slot[key] : -2;
+  }
+  __syncthreads();
+  if (s_call == 0) {  // wrapped: forget every claim mark
+    for (int s = tid; s < d.n_slots; s += blockDim.x) d.slot_call[s] = 0u;
+    __syncthreads();
+    if (tid == 0) s_call = 1u;
+  }
+  // later occurrences of an expert are dropped (marked hot) so that each
+  // distinct cold expert is handled once, at its first occurrence
+  int dup[kMaxTierSel / kResolveThreads];
+#pragma unroll
+  for (int r = 0; r < kMaxTierSel / kResolveThreads; ++r) {
+    const int i = tid + r * kResolveThreads;
+    dup[r] = 0;
+    if (i < n && s_slot[i] != -2)
+      for (int j = 0; j < i; ++j)
+        if (s_key[j] == s_key[i]) {
+          dup[r] = 1;
+          break;
+        }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kMaxTierSel / kResolveThreads; ++r)
+    if (dup[r]) s_slot[tid + r * kResolveThreads] = -2;
+  __syncthreads();
+  const unsigned call = s_call;
+  unsigned long long clock = 0, hits = 0, misses = 0, bytes = 0;
+  int n_tasks = 0;
+  if (tid == 0) {
+    st->call = call;
+    st->n_tasks = 0;
+    clock = st->clock;
+    int n_cold = 0;
+    // hits claim their slots (most recent in call order) before any miss
+    // chooses a victim, so that no miss of this call evicts them
+    for (int i = 0; i < n; ++i) {
+      if (s_slot[i] == -2) continue;
+      ++n_cold;
+      const int sl = s_slot[i];
+      if (sl >= 0) {
+        d.slot_call[sl] = call;
+        d.slot_stamp[sl] = ++clock;
+        ++hits;
+      }
+    }
+    if (s_bad == QE_OK && n_cold > d.n_slots) s_bad = QE_ERR_OOM;
+    if (s_bad != QE_OK) atomicCAS(&st->status, QE_OK, s_bad);
+    s_cur = -1;
+  }
+  __syncthreads();
+  if (s_bad != QE_OK) return;  // resolve nothing (the host refuses such calls before launching)
+  // misses in call order: each takes the least recently used unclaimed slot
+  for (;;) {
+    if (tid == 0) {
+      int i = s_cur + 1;
+      while (i < n && s_slot[i] != -1) ++i;  // the next miss (cached slots are >= 0)
+      s_cur = i;
+      s_kind = i < n;
+    }
+    __syncthreads();
+    if (!s_kind) break;
+    unsigned long long best = ~0ull;
+    int bi = -1;
+    for (int s = tid; s < d.n_slots; s += blockDim.x) {
+      const unsigned long long stamp = d.slot_stamp[s];
+      if (d.slot_call[s] != call && stamp < best) {
+        best = stamp;
+        bi = s;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob < best) {
+        best = ob;
+        bi = oi;
+      }
+    }
+    if (lane == 0) {
+      s_best[warp] = best;
+      s_besti[warp] = bi;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      for (int w = 1; w < kResolveThreads / 32; ++w)
+        if (s_best[w] < best) {
+          best = s_best[w];
+          bi = s_besti[w];
+        }
+      const int i = s_cur;
+      if (bi < 0) {  // every slot claimed: cannot happen once n_cold <= n_slots
+        atomicCAS(&st->status, QE_OK, QE_ERR_OOM);
+        s_slot[i] = -2;
+      } else {
+        const int key = s_key[i];
+        const int old = d.slot_key[bi];
+        if (old >= 0) d.key_slot[old] = -1;
+        d.slot_key[bi] = key;
+        d.key_slot[key] = bi;
+        d.slot_call[bi] = call;
+        d.slot_stamp[bi] = ++clock;
+        d.task_src[n_tasks] = d.cold_src[key];
+        d.task_slot[n_tasks] = bi;
+        ++n_tasks;
+        ++misses;
+        bytes += d.expert_bytes;
+        s_slot[i] = bi;
+      }
+    }
+    __syncthreads();
+  }
+  // descriptors of every distinct cold expert of the call
+  for (int i = tid; i < n; i += blockDim.x)
+    if (s_slot[i] >= 0) table[idx[i]] = slot_descriptor(d, s_slot[i]);
+  if (tid == 0) {
+    st->clock = clock;
+    st->hits += hits;
+    st->misses += misses;
+    st->h2d_bytes += bytes;
+    st->n_tasks = n_tasks;
+  }
+}
+
+__global__ void __launch_bounds__(kResolveThreads) tier_resolve_kernel(TierDev d, int layer, const int32_t* idx,
+                                                                        int n, qe_expert* table) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  tier_resolve_body(d, layer, idx, n, table);
+}
+
+// Copy the queued experts from host memory (device-visible addresses) into
+// their slots, 16 bytes per access, four accesses in flight per thread.
+__global__ void __launch_bounds__(kFillThreads) tier_fill_kernel(TierDev d) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int n = d.st->n_tasks;
+  const unsigned long long per = d.expert_bytes / 16;  // expert bytes are a multiple of 256
+  const unsigned long long total = (unsigned long long)n * per;
+  const unsigned long long stride = (unsigned long long)gridDim.x * blockDim.x;
+  for (unsigned long long j0 = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x; j0 < total;
+       j0 += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const unsigned long long j = j0 + u * stride;
+      if (j < total) {
+        const unsigned long long t = j / per, o = j - t * per;
+        v[u] = reinterpret_cast<const uint4*>(d.task_src[t])[o];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const unsigned long long j = j0 + u * stride;
+      if (j < total) {
+        const unsigned long long t = j / per, o = j - t * per;
+        reinterpret_cast<uint4*>(d.cache + (size_t)d.task_slot[t] * d.slot_bytes)[o] = v[u];
+      }
+    }
+  }
+}
+
+
+// Routing of one token for the tiered step, with the resolve folded in:
+// RMSNorm scale, router logits (fp64), top-K with renormalised softmax
+// weights, then tier_resolve_body on the chosen experts.  Each CTA takes
+// kRouteRows router rows, kRouteSplit warps per row, each warp one
+// 1/kRouteSplit of the columns; every CTA also sums x^2 itself (x is small
+// and in L2), so no CTA waits for another.  The last CTA to finish its
+// logits (an arrival counter after a fence) takes the top-K and the resolve;
+// the others just exit.  The logit and weight formulas are moe_route's:
+// l_e = (sum_c W[e,c] * x_c * gamma_c) / sqrt(mean(x^2) + eps) + offset_e,
+// sums in fp64, ties to the lower index.
+constexpr int kRouteSplit = 8;
+constexpr int kRouteRows = kResolveThreads / 32 / kRouteSplit;  // 4
+constexpr int kRouteUnroll = 4;
+
+struct TierRoute {
+  const void* x;
+  int x_bf16;
+  const float* gamma;
+  const float* router_w;
+  const float* offset;
+  int H, E, K;
+  float eps;
+  double* logits;  // [E], workspace
+  int32_t* idx;    // [K]
+  float* w;        // [K]
+};
+
+// x[c..c+3] as floats (c % 4 == 0; fp32 rows are 16-byte aligned here, bf16
+// rows 8-byte aligned)
+__device__ __forceinline__ float4 load_x4(const TierRoute& r, int c) {
+  if (!r.x_bf16) return *reinterpret_cast<const float4*>((const float*)r.x + c);
+  const uint2 u = *reinterpret_cast<const uint2*>((const uint16_t*)r.x + c);
+  return make_float4(bf16f(u.x & 0xffffu), bf16f(u.x >> 16), bf16f(u.y & 0xffffu), bf16f(u.y >> 16));
+}
+
+__global__ void __launch_bounds__(kResolveThreads) tier_route_kernel(TierRoute r, TierDev d, int layer,
+                                                                      qe_expert* table) {
+  __shared__ double s_part[kRouteRows][kRouteSplit];
+  __shared__ double s_ss[kResolveThreads / 32];
+  __shared__ double s_lg[kMaxE];
+  __shared__ int s_last;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  grid_dependency_wait();  // x comes from the previous kernel
+  grid_launch_dependents();
+  auto ldx = [&](int c) -> double {
+    return r.x_bf16 ? (double)bf16f(((const uint16_t*)r.x)[c]) : (double)((const float*)r.x)[c];
+  };
+  // sum of squares: all of a thread's loads first (H <= 8192: at most 8)
+  double xs[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int c = tid + u * kResolveThreads;
+    xs[u] = c < r.H ? ldx(c) : 0.0;
+  }
+  double ss = 0.0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) ss += xs[u] * xs[u];
+  ss = warp_sum_d(ss);
+  if (lane == 0) s_ss[warp] = ss;
+  // this warp's part of one router row: all of a lane's loads are issued
+  // before its FMAs (4 float4 of W and 4 of x at a time)
+  const int row = warp / kRouteSplit, part = warp % kRouteSplit;
+  const int e = blockIdx.x * kRouteRows + row;
+  double acc = 0.0;
+  if (e < r.E) {
+    const int q4 = r.H / 4 / kRouteSplit;  // float4 per part (H % 64 == 0, so whole); <= 256
+    const float4* wrow = reinterpret_cast<const float4*>(r.router_w + (size_t)e * r.H) + part * q4;
+    const int c0 = part * q4 * 4;
+    for (int i0 = lane; i0 < q4; i0 += 32 * kRouteUnroll) {
+      float4 wv[kRouteUnroll], xv[kRouteUnroll];
+#pragma unroll
+      for (int u = 0; u < kRouteUnroll; ++u) {
+        const int i = i0 + 32 * u;
+        if (i < q4) {
+          wv[u] = __ldg(wrow + i);
+          xv[u] = load_x4(r, c0 + 4 * i);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kRouteUnroll; ++u) {
+        const int i = i0 + 32 * u;
+        if (i < q4) {
+          const int c = c0 + 4 * i;
+          double g0 = 1.0, g1 = 1.0, g2 = 1.0, g3 = 1.0;
+          if (r.gamma) {
+            const float4 gv = *reinterpret_cast<const float4*>(r.gamma + c);
+            g0 = gv.x, g1 = gv.y, g2 = gv.z, g3 = gv.w;
+          }
+          acc = fma((double)wv[u].x, (double)xv[u].x * g0, acc);
+          acc = fma((double)wv[u].y, (double)xv[u].y * g1, acc);
+          acc = fma((double)wv[u].z, (double)xv[u].z * g2, acc);
+          acc = fma((double)wv[u].w, (double)xv[u].w * g3, acc);
+        }
+      }
+    }
+  }
+  acc = warp_sum_d(acc);
+  if (lane == 0) s_part[row][part] = acc;
+  __syncthreads();
+  if (tid < kRouteRows && blockIdx.x * kRouteRows + tid < r.E) {
+    double a = 0.0, q = 0.0;
+    for (int p = 0; p < kRouteSplit; ++p) a += s_part[tid][p];
+    for (int w = 0; w < kResolveThreads / 32; ++w) q += s_ss[w];
+    const double rinv = 1.0 / sqrt(q / (double)r.H + (double)r.eps);
+    const int ee = blockIdx.x * kRouteRows + tid;
+    r.logits[ee] = a * rinv + (r.offset ? (double)r.offset[ee] : 0.0);
+    __threadfence();  // the logit is visible before this CTA counts itself done
+  }
+  __syncthreads();
+  if (tid == 0) {
+    s_last = atomicAdd(&d.st->route_done, 1u) == gridDim.x - 1;
+    __threadfence();
+  }
+  __syncthreads();
+  if (!s_last) return;  // uniform: the whole CTA leaves
+  // every logit into shared memory (read past L1: other CTAs wrote them)
+  for (int ex = tid; ex < r.E; ex += kResolveThreads) s_lg[ex] = __ldcg(r.logits + ex);
+  __syncthreads();
+  if (warp == 0) {
+    // top-K, ties to the lower index
+    const int E = r.E, K = r.K;
+    unsigned taken = 0;
+    int sel[kMaxK];
+    for (int k = 0; k < K; ++k) {
+      double bv = 0.0;
+      int bi = 0x7fffffff;
+      for (int i = 0, ex = lane; ex < E; ++i, ex += 32) {
+        if (taken & (1u << i)) continue;
+        const double v = s_lg[ex];
+        if (bi == 0x7fffffff || v > bv) {
+          bv = v;
+          bi = ex;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      sel[k] = bi;
+    }
+    if (lane == 0) {
+      const double lmax = s_lg[sel[0]];
+      double ev[kMaxK];
+      double sum = 0.0;
+      for (int k = 0; k < K; ++k) {
+        ev[k] = exp(s_lg[sel[k]] - lmax);
+        sum += ev[k];
+      }
+      for (int k = 0; k < K; ++k) {
+        r.idx[k] = sel[k];
+        r.w[k] = (float)(ev[k] / sum);
+      }
+      d.st->route_done = 0u;  // ready for the next launch
+    }
+  }
+  __syncthreads();  // idx written by warp 0 is visible to the CTA
+  tier_resolve_body(d, layer, r.idx, r.K, table);
+}
+
+}  // namespace qe
 
 struct qe_tier {
   qe_cfg cfg;
-  int L = 0, E = 0, bits = 2, dev = 0, max_tokens = 0;
-  size_t slot_bytes = 0, expert_bytes = 0;
+  int L = 0, E = 0, bits = 2, dev = 0, max_tokens = 0, sms = 148;
+  size_t expert_bytes = 0;
   int n_slots = 0;
-  std::vector<const void*> cold_host;  // [L*E], NULL for a hot expert
-  unsigned char* cache = nullptr;      // device, n_slots * slot_bytes
-  // LRU over slots: head = most recently used.  Free slots sit at the tail.
-  std::vector<int> slot_key, key_slot, prev, next;
-  std::vector<unsigned> slot_call;  // slot claimed by call number slot_call[s]
-  std::vector<unsigned> key_call;   // key seen in call number key_call[k]
-  int head = -1, tail = -1;
-  unsigned call = 0;
-  cudaStream_t copy_stream = nullptr;
-  cudaEvent_t ev_main = nullptr, ev_copy = nullptr, ev_idx = nullptr, ev_stage = nullptr;
-  int32_t* idx_host = nullptr;      // pinned [max_tokens * K]
-  qe_expert* stage_host = nullptr;  // pinned [max_tokens * K] descriptors
-  int32_t* pos_host = nullptr;      // pinned [max_tokens * K] table positions
-  qe_expert* stage_dev = nullptr;   // device copies of the two arrays above
-  int32_t* pos_dev = nullptr;
-  unsigned long long hits = 0, misses = 0, h2d_bytes = 0;
+  std::vector<unsigned char> is_cold;  // [L*E], host copy for argument checks
+  std::vector<unsigned> mark;          // [L*E], host scratch for counting distinct experts
+  unsigned mark_gen = 0;
+  unsigned char* cache = nullptr;      // device, n_slots * expert_bytes
+  void* state_mem = nullptr;           // device: TierState and the arrays of TierDev
+  int32_t* idx_dev = nullptr;          // device staging of host indices [max selections]
+  qe::TierDev d{};
   std::mutex mu;
 };
 
 namespace qe {
 
-// Scatter n descriptors into a device table: table[pos[j]] = desc[j].
-__global__ void tier_scatter_kernel(const qe_expert* desc, const int32_t* pos, int n, qe_expert* table) {
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j < n) table[pos[j]] = desc[j];
-}
-
-static void lru_unlink(qe_tier* t, int s) {
-  if (t->prev[s] >= 0) t->next[t->prev[s]] = t->next[s];
-  else t->head = t->next[s];
-  if (t->next[s] >= 0) t->prev[t->next[s]] = t->prev[s];
-  else t->tail = t->prev[s];
-  t->prev[s] = t->next[s] = -1;
-}
-
-static void lru_push_front(qe_tier* t, int s) {
-  t->prev[s] = -1;
-  t->next[s] = t->head;
-  if (t->head >= 0) t->prev[t->head] = s;
-  t->head = s;
-  if (t->tail < 0) t->tail = s;
-}
+static size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 static int check_device(const qe_tier* t) {
   int dev = -1;
@@ -73,102 +473,36 @@ static int check_device(const qe_tier* t) {
 
 static void tier_free(qe_tier* t) {
   if (!t) return;
-  if (t->copy_stream) cudaStreamSynchronize(t->copy_stream);
-  if (t->ev_stage) cudaEventSynchronize(t->ev_stage);
+  if (t->cache || t->state_mem) cudaDeviceSynchronize();  // kernels queued on the tier may still run
   if (t->cache) cudaFree(t->cache);
-  if (t->stage_dev) cudaFree(t->stage_dev);
-  if (t->pos_dev) cudaFree(t->pos_dev);
-  if (t->idx_host) cudaFreeHost(t->idx_host);
-  if (t->stage_host) cudaFreeHost(t->stage_host);
-  if (t->pos_host) cudaFreeHost(t->pos_host);
-  for (cudaEvent_t ev : {t->ev_main, t->ev_copy, t->ev_idx, t->ev_stage})
-    if (ev) cudaEventDestroy(ev);
-  if (t->copy_stream) cudaStreamDestroy(t->copy_stream);
+  if (t->state_mem) cudaFree(t->state_mem);
   delete t;
 }
 
-// Resolve the experts of one call (caller holds t->mu).
-static int resolve_locked(qe_tier* t, int layer, const int32_t* idx, int n, qe_expert* dev_table, cudaStream_t s) {
-  const int E = t->E;
-  ++t->call;
-  if (t->call == 0) {  // wrapped: forget old claims
-    std::fill(t->slot_call.begin(), t->slot_call.end(), 0u);
-    std::fill(t->key_call.begin(), t->key_call.end(), 0u);
-    t->call = 1;
-  }
-  for (int i = 0; i < n; ++i)
-    if (idx[i] < 0 || idx[i] >= E) return fail(QE_ERR_INVALID_ARG, "expert index %d out of range [0, %d)", idx[i], E);
-  // pass 1: hits claim their slots, so that no miss of this call evicts them
-  int n_cold = 0;
-  for (int i = 0; i < n; ++i) {
-    const int key = layer * E + idx[i];
-    if (!t->cold_host[key] || t->key_call[key] == t->call) continue;
-    t->key_call[key] = t->call;
-    ++n_cold;
-    const int sl = t->key_slot[key];
-    if (sl >= 0) {
-      t->slot_call[sl] = t->call;
-      lru_unlink(t, sl);
-      lru_push_front(t, sl);
-    }
-  }
-  if (n_cold > t->n_slots)
-    return fail(QE_ERR_OOM, "one call needs %d cold experts but the cache holds %d slots", n_cold, t->n_slots);
-  // pass 2: misses take the least recently used unclaimed slot
-  int nd = 0, n_miss = 0;
-  for (int i = 0; i < n; ++i) {
-    const int key = layer * E + idx[i];
-    if (!t->cold_host[key] || t->key_call[key] != t->call) continue;
-    t->key_call[key] = t->call - 1;  // emit each distinct expert once (call - 1 != call)
-    int sl = t->key_slot[key];
-    if (sl >= 0) {
-      ++t->hits;
-    } else {
-      sl = t->tail;
-      while (sl >= 0 && t->slot_call[sl] == t->call) sl = t->prev[sl];
-      if (sl < 0) return fail(QE_ERR_OOM, "no free cache slot");
-      if (t->slot_key[sl] >= 0) t->key_slot[t->slot_key[sl]] = -1;
-      t->slot_key[sl] = key;
-      t->key_slot[key] = sl;
-      t->slot_call[sl] = t->call;
-      lru_unlink(t, sl);
-      lru_push_front(t, sl);
-      if (n_miss == 0) {
-        // the copy may overwrite a slot that work already queued on `s` reads
-        cudaError_t e = cudaEventRecord(t->ev_main, s);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(t->copy_stream, t->ev_main, 0);
-        if (e != cudaSuccess) return cuda_fail(e, "tier: order the copy stream after the compute stream");
-      }
-      cudaError_t e = cudaMemcpyAsync(t->cache + (size_t)sl * t->slot_bytes, t->cold_host[key], t->expert_bytes,
-                                      cudaMemcpyHostToDevice, t->copy_stream);
-      if (e != cudaSuccess) return cuda_fail(e, "tier: expert copy");
-      ++t->misses;
-      t->h2d_bytes += t->expert_bytes;
-      ++n_miss;
-    }
-    if (nd == 0) {
-      // the staging arrays of the previous call must have been consumed
-      cudaError_t e = cudaEventSynchronize(t->ev_stage);
-      if (e != cudaSuccess) return cuda_fail(e, "tier: staging wait");
-    }
-    t->stage_host[nd] = pool_descriptor(&t->cfg, t->cache + (size_t)sl * t->slot_bytes, t->bits);
-    t->pos_host[nd] = idx[i];
-    ++nd;
-  }
-  if (n_miss > 0) {
-    cudaError_t e = cudaEventRecord(t->ev_copy, t->copy_stream);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, t->ev_copy, 0);
-    if (e != cudaSuccess) return cuda_fail(e, "tier: order the compute stream after the copies");
-  }
-  if (nd > 0) {
-    cudaError_t e = cudaMemcpyAsync(t->stage_dev, t->stage_host, sizeof(qe_expert) * nd, cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(t->pos_dev, t->pos_host, sizeof(int32_t) * nd, cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return cuda_fail(e, "tier: descriptor upload");
-    tier_scatter_kernel<<<(nd + 127) / 128, 128, 0, s>>>(t->stage_dev, t->pos_dev, nd, dev_table);
-    e = cudaGetLastError();
-    if (e == cudaSuccess) e = cudaEventRecord(t->ev_stage, s);
-    if (e != cudaSuccess) return cuda_fail(e, "tier: descriptor scatter");
-  }
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous one drains; each of these kernels waits for it
+// (griddepcontrol.wait) before touching memory.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Resolve + fill for `n` device indices of layer `layer` on stream s.
+static int launch_resolve(qe_tier* t, int layer, const int32_t* idx_dev, int n, qe_expert* dev_table,
+                          cudaStream_t s) {
+  cudaError_t e = launch_pdl(tier_resolve_kernel, 1, kResolveThreads, s, t->d, layer, idx_dev, n, dev_table);
+  if (e != cudaSuccess) return cuda_fail(e, "tier resolve launch");
+  e = launch_pdl(tier_fill_kernel, t->sms, kFillThreads, s, t->d);
+  if (e != cudaSuccess) return cuda_fail(e, "tier fill launch");
   return QE_OK;
 }
 
@@ -187,52 +521,104 @@ int qe_tier_create(const qe_tier_desc* d, qe_tier** out) {
   if (d->n_layers <= 0) return fail(QE_ERR_INVALID_ARG, "n_layers must be positive");
   if (!(d->cold_bits == 2 || d->cold_bits == 4)) return fail(QE_ERR_INVALID_ARG, "cold_bits must be 2 or 4");
   if (!d->cold_host) return fail(QE_ERR_INVALID_ARG, "cold_host is NULL");
-  if (d->max_tokens <= 0) return fail(QE_ERR_INVALID_ARG, "max_tokens must be positive");
+  if (d->max_tokens <= 0 || (long long)d->max_tokens * d->cfg.top_k > kMaxTierSel)
+    return fail(QE_ERR_INVALID_ARG, "max_tokens * top_k must be in [1, %d]", kMaxTierSel);
   const size_t eb = qe_expert_bytes(&d->cfg, d->cold_bits);
   const size_t nkeys = (size_t)d->n_layers * d->cfg.n_experts;
   if (nkeys > (size_t)0x7fffffff) return fail(QE_ERR_INVALID_ARG, "too many experts");
   const size_t n_slots = d->cache_bytes / eb;
   if (n_slots < 1) return fail(QE_ERR_INVALID_ARG, "cache_bytes %zu holds no %zu-byte expert", d->cache_bytes, eb);
   if (n_slots > (size_t)0x7fffffff) return fail(QE_ERR_INVALID_ARG, "cache too large");
+  for (size_t k = 0; k < nkeys; ++k)
+    if (((uintptr_t)d->cold_host[k] & 15) != 0)
+      return fail(QE_ERR_INVALID_ARG, "cold expert %zu is not 16-byte aligned", k);
   qe_tier* t = new qe_tier();
   t->cfg = d->cfg;
   t->L = d->n_layers;
   t->E = d->cfg.n_experts;
   t->bits = d->cold_bits;
   t->max_tokens = d->max_tokens;
-  t->expert_bytes = eb;
-  t->slot_bytes = eb;  // segments are 256-byte multiples already
+  t->expert_bytes = eb;  // segments are 256-byte multiples already
   t->n_slots = (int)n_slots;
-  t->cold_host.assign(d->cold_host, d->cold_host + nkeys);
-  t->key_slot.assign(nkeys, -1);
-  t->key_call.assign(nkeys, 0u);
-  t->slot_key.assign(n_slots, -1);
-  t->slot_call.assign(n_slots, 0u);
-  t->prev.assign(n_slots, -1);
-  t->next.assign(n_slots, -1);
-  for (int s = (int)n_slots - 1; s >= 0; --s) lru_push_front(t, s);
+  t->is_cold.assign(nkeys, 0);
+  t->mark.assign(nkeys, 0u);
+  // the device reads cold experts through their device-visible addresses
+  std::vector<unsigned long long> src(nkeys, 0ull);
   cudaError_t e = cudaGetDevice(&t->dev);
-  const size_t nst = (size_t)d->max_tokens * d->cfg.top_k;
-  if (e == cudaSuccess) {
-    e = cudaMalloc(&t->cache, n_slots * t->slot_bytes);
-    if (e != cudaSuccess) {
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&t->sms, cudaDevAttrMultiProcessorCount, t->dev);
+  for (size_t k = 0; k < nkeys && e == cudaSuccess; ++k) {
+    if (!d->cold_host[k]) continue;
+    cudaPointerAttributes pa{};
+    e = cudaPointerGetAttributes(&pa, d->cold_host[k]);
+    if (e != cudaSuccess || pa.type != cudaMemoryTypeHost || !pa.devicePointer) {
       cudaGetLastError();
-      tier_free(t);
-      return fail(QE_ERR_OOM, "tier: cudaMalloc of the %zu-byte expert cache failed", n_slots * eb);
+      delete t;
+      return fail(QE_ERR_INVALID_ARG,
+                  "cold expert %zu is not page-locked host memory mapped for the device (allocate it with "
+                  "cudaHostAlloc, or register it with cudaHostRegisterMapped)", k);
     }
+    src[k] = (unsigned long long)(uintptr_t)pa.devicePointer;
+    t->is_cold[k] = 1;
   }
-  if (e == cudaSuccess) e = cudaMalloc(&t->stage_dev, sizeof(qe_expert) * nst);
-  if (e == cudaSuccess) e = cudaMalloc(&t->pos_dev, sizeof(int32_t) * nst);
-  if (e == cudaSuccess) e = cudaHostAlloc(&t->idx_host, sizeof(int32_t) * nst, cudaHostAllocDefault);
-  if (e == cudaSuccess) e = cudaHostAlloc(&t->stage_host, sizeof(qe_expert) * nst, cudaHostAllocDefault);
-  if (e == cudaSuccess) e = cudaHostAlloc(&t->pos_host, sizeof(int32_t) * nst, cudaHostAllocDefault);
-  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&t->copy_stream, cudaStreamNonBlocking);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t->ev_main, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t->ev_copy, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t->ev_idx, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&t->ev_stage, cudaEventDisableTiming);
   if (e != cudaSuccess) {
     const int r = cuda_fail(e, "qe_tier_create");
+    delete t;
+    return r;
+  }
+  const size_t nsel = (size_t)d->max_tokens * d->cfg.top_k;
+  // one device block: state, then the arrays, each 256-byte aligned
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off = al256(off + bytes); return o; };
+  const size_t o_st = take(sizeof(TierState)), o_ks = take(4 * nkeys),
+               o_src = take(8 * nkeys), o_sk = take(4 * n_slots), o_sc = take(4 * n_slots),
+               o_stamp = take(8 * n_slots), o_tsrc = take(8 * nsel), o_tslot = take(4 * nsel),
+               o_idx = take(4 * nsel);
+  e = cudaMalloc(&t->cache, n_slots * eb);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    t->cache = nullptr;
+    tier_free(t);
+    return fail(QE_ERR_OOM, "tier: cudaMalloc of the %zu-byte expert cache failed", n_slots * eb);
+  }
+  e = cudaMalloc(&t->state_mem, off);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    t->state_mem = nullptr;
+    tier_free(t);
+    return fail(QE_ERR_OOM, "tier: cudaMalloc of %zu bytes of cache state failed", off);
+  }
+  char* b = (char*)t->state_mem;
+  TierDev& dv = t->d;
+  dv.st = (TierState*)(b + o_st);
+  dv.key_slot = (int32_t*)(b + o_ks);
+  dv.cold_src = (const unsigned long long*)(b + o_src);
+  dv.slot_key = (int32_t*)(b + o_sk);
+  dv.slot_call = (uint32_t*)(b + o_sc);
+  dv.slot_stamp = (unsigned long long*)(b + o_stamp);
+  dv.task_src = (unsigned long long*)(b + o_tsrc);
+  dv.task_slot = (int32_t*)(b + o_tslot);
+  dv.cache = t->cache;
+  dv.slot_bytes = eb;
+  dv.expert_bytes = eb;
+  dv.n_slots = (int)n_slots;
+  dv.E = t->E;
+  dv.tmpl = pool_descriptor(&t->cfg, t->cache, t->bits);
+  t->idx_dev = (int32_t*)(b + o_idx);
+  // initial state: nothing cached; slot s stamped n_slots - s, so that the
+  // highest slot is the least recently used (free slots are taken from the top)
+  TierState st0{};
+  st0.clock = n_slots;
+  std::vector<int32_t> minus1(nkeys > n_slots ? nkeys : n_slots, -1);
+  std::vector<unsigned long long> stamps(n_slots);
+  for (size_t s = 0; s < n_slots; ++s) stamps[s] = n_slots - s;
+  e = cudaMemcpy(dv.st, &st0, sizeof(st0), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(dv.key_slot, minus1.data(), 4 * nkeys, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy((void*)dv.cold_src, src.data(), 8 * nkeys, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(dv.slot_key, minus1.data(), 4 * n_slots, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemset(dv.slot_call, 0, 4 * n_slots);
+  if (e == cudaSuccess) e = cudaMemcpy(dv.slot_stamp, stamps.data(), 8 * n_slots, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    const int r = cuda_fail(e, "qe_tier_create: initial state");
     tier_free(t);
     return r;
   }
@@ -252,7 +638,27 @@ int qe_tier_resolve(qe_tier* t, int layer, const int32_t* host_idx, int n, qe_ex
   if ((rc = check_ptr(dev_table, "dev_table", false, 8))) return rc;
   if ((rc = check_device(t))) return rc;
   std::lock_guard<std::mutex> lock(t->mu);
-  return resolve_locked(t, layer, host_idx, n, dev_table, (cudaStream_t)stream);
+  // checked on the host first, so that a refused call changes nothing
+  if (++t->mark_gen == 0) {
+    std::fill(t->mark.begin(), t->mark.end(), 0u);
+    t->mark_gen = 1;
+  }
+  int n_cold = 0;
+  for (int i = 0; i < n; ++i) {
+    if (host_idx[i] < 0 || host_idx[i] >= t->E)
+      return fail(QE_ERR_INVALID_ARG, "expert index %d out of range [0, %d)", host_idx[i], t->E);
+    const size_t key = (size_t)layer * t->E + host_idx[i];
+    if (t->is_cold[key] && t->mark[key] != t->mark_gen) {
+      t->mark[key] = t->mark_gen;
+      ++n_cold;
+    }
+  }
+  if (n_cold > t->n_slots)
+    return fail(QE_ERR_OOM, "one call needs %d cold experts but the cache holds %d slots", n_cold, t->n_slots);
+  const cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(t->idx_dev, host_idx, sizeof(int32_t) * n, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "qe_tier_resolve: index upload");
+  return launch_resolve(t, layer, t->idx_dev, n, dev_table, s);
 }
 
 int qe_tier_layer_step(qe_tier* t, int layer, const qe_layer* lw, const void* x, int x_dtype, int T, float* out,
@@ -273,38 +679,58 @@ int qe_tier_layer_step(qe_tier* t, int layer, const qe_layer* lw, const void* x,
       (rc = check_ws(c, T, ws, ws_bytes)))
     return rc;
   if ((const void*)out == x) return fail(QE_ERR_INVALID_ARG, "out must not alias x");
+  // the routing is not known on the host: a call may need up to T * top_k
+  // cold experts at once, and the cache must be able to hold them all
+  if (T * c->top_k > t->n_slots)
+    return fail(QE_ERR_OOM, "T * top_k = %d may exceed the cache's %d slots", T * c->top_k, t->n_slots);
   if ((rc = check_device(t))) return rc;
   cudaStream_t s = (cudaStream_t)stream;
   const WsLayout L = ws_layout(c->hidden, c->n_experts, c->top_k, c->inter, T);
   int32_t* idx = topk_idx ? topk_idx : (int32_t*)((char*)ws + L.idx);
   float* w = topk_w ? topk_w : (float*)((char*)ws + L.w);
-  rc = route_impl(c, x, x_dtype, lw->gamma, lw->router_w, lw->logit_offset, T, nullptr, idx, w, ws, ws_bytes,
-                  !(T == 1 && fused_fits(c, x, x_dtype, lw->gamma)), s);
-  if (rc) return rc;
-  std::lock_guard<std::mutex> lock(t->mu);
-  const int n = T * c->top_k;
-  // the one host synchronisation of the tiered step: the routing decides
-  // which cold experts must be copied in
-  cudaError_t e = cudaMemcpyAsync(t->idx_host, idx, sizeof(int32_t) * n, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaEventRecord(t->ev_idx, s);
-  if (e == cudaSuccess) e = cudaEventSynchronize(t->ev_idx);
-  if (e != cudaSuccess) return cuda_fail(e, "qe_tier_layer_step: read routing");
-  rc = resolve_locked(t, layer, t->idx_host, n, const_cast<qe_expert*>(lw->experts), s);
-  if (rc) return rc;
-  // one token: the fused kernel with this routing (it does not route again,
-  // so it reads exactly the experts resolved above)
-  if (T == 1 && fused_fits(c, x, x_dtype, lw->gamma))
+  qe_expert* table = const_cast<qe_expert*>(lw->experts);
+  if (T == 1 && fused_fits(c, x, x_dtype, lw->gamma)) {
+    // one token: routing and resolve in one kernel, the fill, then the
+    // single-token kernel with this routing (it does not route again, so it
+    // reads exactly the experts resolved here)
+    TierRoute r{x, x_dtype == QE_BF16, lw->gamma, lw->router_w, lw->logit_offset, c->hidden, c->n_experts,
+                c->top_k, c->eps, (double*)((char*)ws + L.logits), idx, w};
+    cudaError_t e;
+    {
+      std::lock_guard<std::mutex> lock(t->mu);
+      e = launch_pdl(tier_route_kernel, (c->n_experts + kRouteRows - 1) / kRouteRows, kResolveThreads, s, r, t->d,
+                     layer, table);
+      if (e == cudaSuccess) e = launch_pdl(tier_fill_kernel, t->sms, kFillThreads, s, t->d);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "tier routing launch");
     return fused_step(c, lw, x, x_dtype, out, add_residual, nullptr, nullptr, ws, idx, w, s);
+  }
+  // several tokens (or a token the single-token kernel does not take): the
+  // route kernels, resolve + fill, then the batched experts and combine
+  rc = route_impl(c, x, x_dtype, lw->gamma, lw->router_w, lw->logit_offset, T, nullptr, idx, w, ws, ws_bytes,
+                  true, s);
+  if (rc) return rc;
+  {
+    std::lock_guard<std::mutex> lock(t->mu);
+    rc = launch_resolve(t, layer, idx, T * c->top_k, table, s);
+  }
+  if (rc) return rc;
   return experts_and_combine(c, lw->experts, idx, w, x, x_dtype, T, out, add_residual, ws, s);
 }
 
 int qe_tier_stats(const qe_tier* t, uint64_t* hits, uint64_t* misses, uint64_t* h2d_bytes) {
   if (!t) return fail(QE_ERR_INVALID_ARG, "tier is NULL");
-  qe_tier* m = const_cast<qe_tier*>(t);
-  std::lock_guard<std::mutex> lock(m->mu);
-  if (hits) *hits = t->hits;
-  if (misses) *misses = t->misses;
-  if (h2d_bytes) *h2d_bytes = t->h2d_bytes;
+  int rc = check_device(t);
+  if (rc) return rc;
+  // the counters are updated by kernels on the caller's streams: wait for them
+  cudaError_t e = cudaDeviceSynchronize();
+  TierState st{};
+  if (e == cudaSuccess) e = cudaMemcpy(&st, t->d.st, sizeof(st), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "qe_tier_stats");
+  if (hits) *hits = st.hits;
+  if (misses) *misses = st.misses;
+  if (h2d_bytes) *h2d_bytes = st.h2d_bytes;
+  if (st.status != QE_OK) return fail(st.status, "tier: a resolve on the device failed (status %d)", st.status);
   return QE_OK;
 }
 

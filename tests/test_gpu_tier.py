@@ -175,3 +175,70 @@ def test_tiered_full_layer_shape(q):
     assert (hits, misses) == (model.hits, model.misses)
     assert n_ok == 12
     st.tier.close()
+
+
+def test_tiered_tokens_captured_in_a_cuda_graph(q):
+    """Hits and misses are resolved on the device, so whole tokens through
+    the tiered stack capture into one CUDA graph (a host synchronisation
+    inside would fail the capture).  Replayed once, the graph gives the same
+    routing, outputs and cache counters as the LRU model and the oracle."""
+    import torch
+    cfg = q.Cfg(1024, 32, 4, 256)
+    st = TieredStack(q, cfg, n_layers=3, n_hot=8, seed=5, cache_slots=6, max_tokens=1)
+    model = LruModel(6)
+    K, H, E, L, NT = cfg.top_k, cfg.hidden, cfg.n_experts, 3, 5
+    x = dev_tokens(5, 700, NT, H)
+    acts = torch.empty((NT, L, H), dtype=torch.float32, device="cuda")
+    idx = torch.empty((NT, L, K), dtype=torch.int32, device="cuda")
+    s = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for t in range(NT):
+            cur = x[t:t + 1]
+            for l in range(L):
+                st.tier.layer_step(l, st.layers[l], cur, acts[t, l:l + 1], True, idx[t, l:l + 1], None, st.ws,
+                                   stream=s)
+                cur = acts[t, l:l + 1]
+    assert st.tier.stats() == (0, 0, 0)  # capturing ran nothing
+    g.replay()
+    torch.cuda.synchronize()
+    assert q.qe_workspace_status(st.ws) == q.QE_OK, q.qe_last_error()
+    ih, ah = idx.cpu().numpy(), acts.cpu().numpy()
+    for t in range(NT):
+        cur = x[t].cpu().numpy().astype(np.float64)
+        for l in range(L):
+            model.call([l * E + int(e) for e in ih[t, l] if not st.hot[l][int(e)]])
+            ref = st.oracle(l, cur)
+            assert_same_routing(ih[t, l], ref["idx"], ref["logits"])
+            assert normwise_err(ah[t, l], ref["out"]) <= TOL, (t, l)
+            cur = ah[t, l].astype(np.float64)
+    hits, misses, h2d = st.tier.stats()
+    assert (hits, misses) == (model.hits, model.misses)
+    assert misses > 6 and hits > 0
+    del g
+    st.tier.close()
+
+
+def test_tiered_refusals_before_launch(q):
+    """A layer step whose T * top_k cold experts might not fit the cache is
+    refused on the host; cold experts in pageable (not page-locked) memory are
+    refused at creation, since the device cannot read them."""
+    import torch
+    cfg = q.Cfg(1024, 32, 4, 256)
+    st = TieredStack(q, cfg, n_layers=1, n_hot=8, seed=6, cache_slots=6, max_tokens=2)
+    x = dev_tokens(6, 10, 2, cfg.hidden)
+    out = torch.empty((2, cfg.hidden), dtype=torch.float32, device="cuda")
+    with pytest.raises(q.QEError) as ei:
+        st.tier.layer_step(0, st.layers[0], x, out, True, None, None, st.ws)  # 2 * 4 > 6 slots
+    assert ei.value.code == q.QE_ERR_OOM
+    assert st.tier.stats() == (0, 0, 0)
+    st.tier.close()
+    cold_b = q.qe_expert_bytes(cfg, 2)
+    pageable = np.zeros(cold_b + 256, np.uint8)
+    base = (pageable.ctypes.data + 255) // 256 * 256
+    cold = [[base if e == 0 else None for e in range(cfg.n_experts)]]
+    with pytest.raises(q.QEError) as ei:
+        q.Tier(cfg, cold, 2, 4 * cold_b, max_tokens=1)
+    assert ei.value.code == q.QE_ERR_INVALID_ARG
+    assert "page-locked" in str(ei.value)
