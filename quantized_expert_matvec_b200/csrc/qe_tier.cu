@@ -86,33 +86,36 @@ __device__ __forceinline__ qe_expert slot_descriptor(const TierDev& d, int slot)
 // barrier.  n <= kMaxTierSel.
 // (A __device__ function so that the single-token routing kernel's last CTA
 // can run it too; called by all kResolveThreads threads of one CTA.)
-__device__ __noinline__ void tier_resolve_body(const TierDev& d, int layer, const int32_t* idx, int n,
-                                               qe_expert* table) {
+__device__ __forceinline__ void tier_resolve_body(const TierDev& d, int layer, const int32_t* idx, int n,
+                                                 qe_expert* table) {
   __shared__ int s_key[kMaxTierSel];    // expert key of selection i
-  __shared__ int s_slot[kMaxTierSel];   // its slot: < 0 if not cached; -2 hot or duplicate
+  __shared__ int s_slot[kMaxTierSel];   // its slot: -1 not cached; -2 hot or duplicate; -3 index out of range
   __shared__ unsigned s_call;
+  __shared__ unsigned long long s_clock;
   __shared__ int s_bad, s_kind, s_cur;
   __shared__ unsigned long long s_best[kResolveThreads / 32];
   __shared__ int s_besti[kResolveThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   TierState* st = d.st;
   __syncthreads();  // the caller's shared memory may still be in use
+  // every load of the hit path in one round trip: the state's call counter
+  // and clock, and each selection's slot (idx may be shared memory)
   if (tid == 0) {
     s_call = st->call + 1u;  // 0 after 2^32 calls
-    s_bad = QE_OK;
+    s_clock = st->clock;
   }
-  __syncthreads();
   for (int i = tid; i < n; i += blockDim.x) {
     const int e = idx[i];
     if (e < 0 || e >= d.E) {
       s_key[i] = -1;
-      s_slot[i] = -2;
-      atomicCAS(&s_bad, QE_OK, QE_ERR_INVALID_ARG);
+      s_slot[i] = -3;
       continue;
     }
     const int key = layer * d.E + e;
     s_key[i] = key;
-    s_slot[i] = d.cold_src[key] ? d.key_slot[key] : -2;
+    const unsigned long long src = d.cold_src[key];
+    const int sl = d.key_slot[key];  // loaded with src, not after it
+    s_slot[i] = src ? sl : -2;
   }
   __syncthreads();
   if (s_call == 0) {  // wrapped: forget every claim mark
@@ -127,7 +130,7 @@ __device__ __noinline__ void tier_resolve_body(const TierDev& d, int layer, cons
   for (int r = 0; r < kMaxTierSel / kResolveThreads; ++r) {
     const int i = tid + r * kResolveThreads;
     dup[r] = 0;
-    if (i < n && s_slot[i] != -2)
+    if (i < n && s_slot[i] >= -1)
       for (int j = 0; j < i; ++j)
         if (s_key[j] == s_key[i]) {
           dup[r] = 1;
@@ -145,12 +148,13 @@ __device__ __noinline__ void tier_resolve_body(const TierDev& d, int layer, cons
   if (tid == 0) {
     st->call = call;
     st->n_tasks = 0;
-    clock = st->clock;
-    int n_cold = 0;
+    clock = s_clock;
+    int n_cold = 0, bad = QE_OK;
     // hits claim their slots (most recent in call order) before any miss
     // chooses a victim, so that no miss of this call evicts them
     for (int i = 0; i < n; ++i) {
-      if (s_slot[i] == -2) continue;
+      if (s_slot[i] == -3) bad = QE_ERR_INVALID_ARG;
+      if (s_slot[i] < -1) continue;
       ++n_cold;
       const int sl = s_slot[i];
       if (sl >= 0) {
@@ -159,8 +163,9 @@ __device__ __noinline__ void tier_resolve_body(const TierDev& d, int layer, cons
         ++hits;
       }
     }
-    if (s_bad == QE_OK && n_cold > d.n_slots) s_bad = QE_ERR_OOM;
-    if (s_bad != QE_OK) atomicCAS(&st->status, QE_OK, s_bad);
+    if (bad == QE_OK && n_cold > d.n_slots) bad = QE_ERR_OOM;
+    if (bad != QE_OK) atomicCAS(&st->status, QE_OK, bad);
+    s_bad = bad;
     s_cur = -1;
   }
   __syncthreads();
@@ -229,11 +234,11 @@ __device__ __noinline__ void tier_resolve_body(const TierDev& d, int layer, cons
   // descriptors of every distinct cold expert of the call
   for (int i = tid; i < n; i += blockDim.x)
     if (s_slot[i] >= 0) table[idx[i]] = slot_descriptor(d, s_slot[i]);
-  if (tid == 0) {
+  if (tid == 0) {  // stores and reductions only: nothing left to wait for
     st->clock = clock;
-    st->hits += hits;
-    st->misses += misses;
-    st->h2d_bytes += bytes;
+    if (hits) atomicAdd(&st->hits, hits);
+    if (misses) atomicAdd(&st->misses, misses);
+    if (bytes) atomicAdd(&st->h2d_bytes, bytes);
     st->n_tasks = n_tasks;
   }
 }
@@ -284,7 +289,8 @@ __global__ void __launch_bounds__(kFillThreads) tier_fill_kernel(TierDev d) {
 // 1/kRouteSplit of the columns; every CTA also sums x^2 itself (x is small
 // and in L2), so no CTA waits for another.  The last CTA to finish its
 // logits (an arrival counter after a fence) takes the top-K and the resolve;
-// the others just exit.  The logit and weight formulas are moe_route's:
+// the others just exit.  The last CTA's top-K runs over the whole block,
+// one logit per thread.  The logit and weight formulas are moe_route's:
 // l_e = (sum_c W[e,c] * x_c * gamma_c) / sqrt(mean(x^2) + eps) + offset_e,
 // sums in fp64, ties to the lower index.
 constexpr int kRouteSplit = 8;
@@ -316,7 +322,10 @@ __global__ void __launch_bounds__(kResolveThreads) tier_route_kernel(TierRoute r
                                                                       qe_expert* table) {
   __shared__ double s_part[kRouteRows][kRouteSplit];
   __shared__ double s_ss[kResolveThreads / 32];
-  __shared__ double s_lg[kMaxE];
+  __shared__ double s_wv[kResolveThreads / 32];
+  __shared__ int s_wi[kResolveThreads / 32];
+  __shared__ double s_selv[kMaxK];
+  __shared__ int s_sel[kMaxK];
   __shared__ int s_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   grid_dependency_wait();  // x comes from the previous kernel
@@ -376,41 +385,51 @@ __global__ void __launch_bounds__(kResolveThreads) tier_route_kernel(TierRoute r
   acc = warp_sum_d(acc);
   if (lane == 0) s_part[row][part] = acc;
   __syncthreads();
-  if (tid < kRouteRows && blockIdx.x * kRouteRows + tid < r.E) {
-    double a = 0.0, q = 0.0;
-    for (int p = 0; p < kRouteSplit; ++p) a += s_part[tid][p];
+  if (tid == 0) {
+    // this CTA's logits, then its arrival: the acquire-release add orders the
+    // stores before it for whichever CTA arrives last
+    double q = 0.0;
     for (int w = 0; w < kResolveThreads / 32; ++w) q += s_ss[w];
     const double rinv = 1.0 / sqrt(q / (double)r.H + (double)r.eps);
-    const int ee = blockIdx.x * kRouteRows + tid;
-    r.logits[ee] = a * rinv + (r.offset ? (double)r.offset[ee] : 0.0);
-    __threadfence();  // the logit is visible before this CTA counts itself done
-  }
-  __syncthreads();
-  if (tid == 0) {
-    s_last = atomicAdd(&d.st->route_done, 1u) == gridDim.x - 1;
-    __threadfence();
+    for (int rr = 0; rr < kRouteRows; ++rr) {
+      const int ee = blockIdx.x * kRouteRows + rr;
+      if (ee < r.E) {
+        double a = 0.0;
+        for (int p = 0; p < kRouteSplit; ++p) a += s_part[rr][p];
+        r.logits[ee] = a * rinv + (r.offset ? (double)r.offset[ee] : 0.0);
+      }
+    }
+    unsigned prev;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(&d.st->route_done) : "memory");
+    s_last = prev == gridDim.x - 1;
   }
   __syncthreads();
   if (!s_last) return;  // uniform: the whole CTA leaves
-  // every logit into shared memory (read past L1: other CTAs wrote them)
-  for (int ex = tid; ex < r.E; ex += kResolveThreads) s_lg[ex] = __ldcg(r.logits + ex);
-  __syncthreads();
-  if (warp == 0) {
-    // top-K, ties to the lower index
-    const int E = r.E, K = r.K;
-    unsigned taken = 0;
-    int sel[kMaxK];
-    for (int k = 0; k < K; ++k) {
-      double bv = 0.0;
-      int bi = 0x7fffffff;
-      for (int i = 0, ex = lane; ex < E; ++i, ex += 32) {
-        if (taken & (1u << i)) continue;
-        const double v = s_lg[ex];
-        if (bi == 0x7fffffff || v > bv) {
-          bv = v;
-          bi = ex;
-        }
+  // top-K over the block: one logit per thread (E <= kResolveThreads), K
+  // rounds of a warp arg-max and an arg-max over the warps' winners; ties go
+  // to the lower index
+  const double lv = tid < r.E ? __ldcg(r.logits + tid) : 0.0;
+  bool alive = tid < r.E;
+  for (int k = 0; k < r.K; ++k) {
+    double bv = lv;
+    int bi = alive ? tid : 0x7fffffff;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+        bv = ov;
+        bi = oi;
       }
+    }
+    if (lane == 0) {
+      s_wv[warp] = bv;
+      s_wi[warp] = bi;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      bv = s_wv[lane];
+      bi = s_wi[lane];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -420,26 +439,29 @@ __global__ void __launch_bounds__(kResolveThreads) tier_route_kernel(TierRoute r
           bi = oi;
         }
       }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      sel[k] = bi;
-    }
-    if (lane == 0) {
-      const double lmax = s_lg[sel[0]];
-      double ev[kMaxK];
-      double sum = 0.0;
-      for (int k = 0; k < K; ++k) {
-        ev[k] = exp(s_lg[sel[k]] - lmax);
-        sum += ev[k];
+      if (lane == 0) {
+        s_sel[k] = bi;
+        s_selv[k] = bv;
       }
-      for (int k = 0; k < K; ++k) {
-        r.idx[k] = sel[k];
-        r.w[k] = (float)(ev[k] / sum);
-      }
-      d.st->route_done = 0u;  // ready for the next launch
     }
+    __syncthreads();
+    if (tid == s_sel[k]) alive = false;
   }
-  __syncthreads();  // idx written by warp 0 is visible to the CTA
-  tier_resolve_body(d, layer, r.idx, r.K, table);
+  if (warp == 0) {
+    // renormalised softmax weights: lane k takes expert k's exponential,
+    // lane 0 sums them in k order
+    const int K = r.K;
+    const double ev = lane < K ? exp(s_selv[lane] - s_selv[0]) : 0.0;
+    double sum = 0.0;
+    for (int k = 0; k < K; ++k) sum += __shfl_sync(0xffffffffu, ev, k);
+    if (lane < K) {
+      r.idx[lane] = s_sel[lane];
+      r.w[lane] = (float)(ev / sum);
+    }
+    if (lane == 0) d.st->route_done = 0u;  // ready for the next launch
+  }
+  __syncthreads();
+  tier_resolve_body(d, layer, s_sel, r.K, table);
 }
 
 }  // namespace qe
