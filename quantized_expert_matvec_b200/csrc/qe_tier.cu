@@ -288,9 +288,12 @@ __global__ void __launch_bounds__(kFillThreads) tier_fill_kernel(TierDev d) {
 // kRouteRows router rows, kRouteSplit warps per row, each warp one
 // 1/kRouteSplit of the columns; every CTA also sums x^2 itself (x is small
 // and in L2), so no CTA waits for another.  The last CTA to finish its
-// logits (an arrival counter after a fence) takes the top-K and the resolve;
-// the others just exit.  The last CTA's top-K runs over the whole block,
-// one logit per thread.  The logit and weight formulas are moe_route's:
+// logits (an acquire-release arrival counter in the tier's state, reset by
+// that CTA for the next launch) takes the top-K and the resolve; the others
+// just exit.  The last CTA's top-K runs over the whole block, one logit per
+// thread.  Two routing launches on one tier must not overlap (all calls on a
+// tier are ordered on the device).  The logit and weight formulas are
+// moe_route's:
 // l_e = (sum_c W[e,c] * x_c * gamma_c) / sqrt(mean(x^2) + eps) + offset_e,
 // sums in fp64, ties to the lower index.
 constexpr int kRouteSplit = 8;
