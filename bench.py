@@ -52,7 +52,8 @@ WORKLOADS = {
     "c3": dict(H=4096, E=512, K=4, I=1024, bits=4, T=1, layers=60, zipf=True, hot=128, cache_gb=24.0,
                name="60 tiered layers of the one-layer shape: per layer the 128 most popular experts 4-bit in "
                     "HBM, the other 384 2-bit in pinned host memory behind a 24 GB HBM LRU expert cache "
-                    "(async H2D on a side stream), Zipf routing, sequential decode tokens with residual",
+                    "(misses copied by a kernel from mapped host memory, cache resolved on the device), Zipf routing, "
+                    "sequential decode tokens with residual",
                metric="60-layer tiered MoE decode tokens/s at 1 B200"),
     "c4": dict(H=4096, E=512, K=4, I=1024, bits=4, T=256,
                name="batched decode of the one-layer workload: 256 bf16 tokens per step, own top-4 of 512 each, "
@@ -893,9 +894,11 @@ def run_gdn(args, wl, rank, world, local_rank):
 
 
 def run_tiered(args, wl, rank, world, local_rank):
-    """One step = one token through all tiered layers: per layer routing, one
-    host synchronisation, cache resolve (misses copied host->device on the
-    side stream), grouped expert FFNs and the combine with residual."""
+    """One step = one token through all tiered layers: per layer the routing
+    kernel (router, top-K and the cache resolve on the device), the fill
+    kernel (misses copied from mapped host memory into their slots) and the
+    single-token kernel with the given routing, residual added; no host
+    synchronisation, so tokens run from CUDA graphs."""
     import torch
     import quantized_expert_matvec_b200 as q
     from _util import dev_router, dev_tokens, fill_pool, fill_pool_slots
