@@ -357,11 +357,14 @@ def gdn_decode_step(state, q, k, v, alpha, beta, out, stream=None):
     """One GatedDeltaNet decode step for every head, in place on ``state``
     (fp32 CUDA tensors: state [n_heads, dv, dk], q and k [n_heads, dk], v and
     out [n_heads, dv], alpha and beta [n_heads])."""
+    import torch
     if state.dim() != 3:
         raise ValueError("state must be [n_heads, dv, dk]")
     nh, dv, dk = (int(d) for d in state.shape)
-    for name, t, n in (("q", q, nh * dk), ("k", k, nh * dk), ("v", v, nh * dv), ("alpha", alpha, nh),
-                       ("beta", beta, nh), ("out", out, nh * dv)):
+    for name, t, n in (("state", state, nh * dv * dk), ("q", q, nh * dk), ("k", k, nh * dk), ("v", v, nh * dv),
+                       ("alpha", alpha, nh), ("beta", beta, nh), ("out", out, nh * dv)):
+        if t.dtype != torch.float32:
+            raise ValueError(f"{name} must be float32, got {t.dtype}")
         if t.numel() != n:
             raise ValueError(f"{name} has {t.numel()} elements, expected {n}")
     _check(lib.gdn_decode_step(nh, dk, dv, _ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),

@@ -167,3 +167,15 @@ def test_gdn_bad_pointers_rejected_before_launch(q):
     assert L.gdn_decode_step(2, 128, 8, M, 2 * M, 3 * M, 4 * M + 60, 5 * M, 6 * M, 4 * M, None) == q.QE_ERR_INVALID_ARG
     # no heads: nothing to do, no pointer looked at
     assert L.gdn_decode_step(0, 128, 8, None, None, None, None, None, None, None, None) == q.QE_OK
+
+
+def test_gdn_binding_checks_dtypes_and_sizes_first(q):
+    import torch
+    S = torch.zeros((2, 8, 16), dtype=torch.float32)
+    f = lambda n, dt=torch.float32: torch.zeros(n, dtype=dt)  # noqa: E731
+    with pytest.raises(ValueError, match="float32"):
+        q.gdn_decode_step(S, f(32, torch.float64), f(32), f(16), f(2), f(2), f(16))
+    with pytest.raises(ValueError, match="elements"):
+        q.gdn_decode_step(S, f(32), f(31), f(16), f(2), f(2), f(16))
+    with pytest.raises(ValueError, match="CUDA"):
+        q.gdn_decode_step(S, f(32), f(32), f(16), f(2), f(2), f(16))  # host tensors never reach the library
